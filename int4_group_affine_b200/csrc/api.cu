@@ -1,0 +1,481 @@
+// api.cu - the extern "C" entry points of libmoeq: argument validation on the
+// host, workspace layout, and the launch sequence of each call.
+#include <string.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace moeq {
+cudaError_t launch_index_build_counts(const Work& wk, const int32_t* adapter_id, int n_adapters, int32_t* counts_out,
+                                      cudaStream_t s);
+}
+
+using namespace moeq;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+#define CHECK_ARG(cond) \
+    do {                \
+        if (!(cond)) return MOE_ERR_INVALID_ARG; \
+    } while (0)
+#define CHECK_CUDA(expr)                              \
+    do {                                              \
+        if ((expr) != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+// A launch on stream `s` followed by its timing mark.
+#define LAUNCH(kind, expr)                            \
+    do {                                              \
+        if ((expr) != cudaSuccess) return MOE_ERR_CUDA; \
+        timing_mark(kind, s);                         \
+    } while (0)
+
+// Shape check of an affine tensor: group a multiple of 32 that divides `in`,
+// 16-byte aligned packed rows.
+bool qtensor_ok(const moe_qtensor& t, int n, int out, int in, int bits) {
+    if (!t.packed || !t.scales || !t.biases) return false;
+    if (t.n != n || t.out != out || t.in != in || t.bits != bits) return false;
+    if (t.group <= 0 || t.group % 32 != 0 || in % t.group != 0) return false;
+    if (!aligned(t.packed, 16) || !aligned(t.scales, 2) || !aligned(t.biases, 2)) return false;
+    return true;
+}
+
+bool lora_proj_ok(const moe_lora_proj& p, int in) {
+    if (!p.A && !p.B) return true;
+    if (!p.A || !p.B) return false;
+    return aligned(p.A, 16) && aligned(p.B, 2) && in % 8 == 0;
+}
+
+moe_status validate_layer(const moe_layer* L) {
+    if (!L) return MOE_ERR_INVALID_ARG;
+    const int H = L->hidden, E = L->n_experts, K = L->top_k, I = L->inter, Is = L->shared_inter;
+    if (H <= 0 || E <= 0 || K <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+    if (E > MOEQ_MAX_EXPERTS || K > MOEQ_MAX_TOPK || K > E || H > MOEQ_MAX_HIDDEN || I > MOEQ_MAX_INTER)
+        return MOE_ERR_UNSUPPORTED;
+    if (H % 32 || I % 32) return MOE_ERR_INVALID_ARG;
+    if (!qtensor_ok(L->router, 1, E, H, 8)) return MOE_ERR_INVALID_ARG;
+    if (L->shared_gate.packed && !qtensor_ok(L->shared_gate, 1, 1, H, 8)) return MOE_ERR_INVALID_ARG;
+    if (!qtensor_ok(L->gate, E, I, H, 4) || !qtensor_ok(L->up, E, I, H, 4) || !qtensor_ok(L->down, E, H, I, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (L->gate.group != L->up.group) return MOE_ERR_UNSUPPORTED;
+    if (L->s_gate.packed) {
+        if (Is <= 0 || Is % 32 || Is > MOEQ_MAX_INTER) return MOE_ERR_INVALID_ARG;
+        if (!qtensor_ok(L->s_gate, 1, Is, H, 4) || !qtensor_ok(L->s_up, 1, Is, H, 4) ||
+            !qtensor_ok(L->s_down, 1, H, Is, 4))
+            return MOE_ERR_INVALID_ARG;
+        if (L->s_gate.group != L->s_up.group) return MOE_ERR_UNSUPPORTED;
+    }
+    if (L->n_adapters < 0 || L->n_adapters > MOEQ_MAX_ADAPTERS) return MOE_ERR_INVALID_ARG;
+    if (L->n_adapters > 0) {
+        if (L->rank <= 0 || L->rank > MOEQ_MAX_RANK) return MOE_ERR_INVALID_ARG;
+        for (int a = 0; a < L->n_adapters; ++a) {
+            const moe_lora_ptrs& p = L->lora[a];
+            if (!lora_proj_ok(p.gate, H) || !lora_proj_ok(p.up, H) || !lora_proj_ok(p.down, I) ||
+                !lora_proj_ok(p.s_gate, H) || !lora_proj_ok(p.s_up, H) || !lora_proj_ok(p.s_down, Is > 0 ? Is : 8))
+                return MOE_ERR_INVALID_ARG;
+        }
+    }
+    return MOE_OK;
+}
+
+struct Dims {
+    int T, K, E, H, I, Is, Imax, A1, C, nb, J, r;
+};
+
+Dims dims_of(const moe_layer* L, int T) {
+    Dims d;
+    d.T = T;
+    d.K = L->top_k;
+    d.E = L->n_experts;
+    d.H = L->hidden;
+    d.I = L->inter;
+    d.Is = L->s_gate.packed ? L->shared_inter : 0;
+    d.Imax = std::max(d.I, d.Is);
+    d.A1 = L->n_adapters + 1;
+    d.C = (T + 31) / 32;
+    d.nb = (d.E + 1) * d.A1;
+    d.J = T * (d.K + 1);
+    d.r = L->n_adapters > 0 ? L->rank : 1;
+    return d;
+}
+
+WsPlan plan_of(const Dims& d) {
+    WsPlan p;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align_up(o + bytes);
+        return at;
+    };
+    p.status = take(8);  // status word + n_active share the first 256 bytes
+    p.n_active = p.status + 4;
+    p.idx = take((size_t)d.T * d.K * 4);
+    p.w = take((size_t)d.T * d.K * 4);
+    p.sg = take((size_t)d.T * 4);
+    p.logits = take((size_t)d.T * d.E * 4);
+    p.gs = take((size_t)d.T * 4);
+    p.cnt = take((size_t)d.nb * d.C * 4);
+    p.goff = take((size_t)(d.E + 2) * 4);
+    p.active = take((size_t)(d.E + 1) * 4);
+    p.perm = take((size_t)d.J * 16);
+    p.wperm = take((size_t)d.J * 4);
+    p.inv = take((size_t)d.J * 4);
+    p.tgu = take((size_t)d.J * 2 * d.r * 4);
+    p.td = take((size_t)d.J * d.r * 4);
+    p.h = take((size_t)d.J * d.Imax * 4);
+    p.ypart = take((size_t)d.J * d.H * 4);
+    p.xn = take((size_t)d.T * d.H * 2);
+    p.total = o;
+    return p;
+}
+
+Work work_of(const Dims& d, const WsPlan& p, void* ws) {
+    char* b = (char*)ws;
+    Work w;
+    w.status = (int32_t*)(b + p.status);
+    w.n_active = (int32_t*)(b + p.n_active);
+    w.idx = (int32_t*)(b + p.idx);
+    w.w = (float*)(b + p.w);
+    w.sg = (float*)(b + p.sg);
+    w.logits = (float*)(b + p.logits);
+    w.gs = (float*)(b + p.gs);
+    w.cnt = (int32_t*)(b + p.cnt);
+    w.goff = (int32_t*)(b + p.goff);
+    w.active = (int32_t*)(b + p.active);
+    w.perm = (int4*)(b + p.perm);
+    w.wperm = (float*)(b + p.wperm);
+    w.inv = (int32_t*)(b + p.inv);
+    w.tgu = (float*)(b + p.tgu);
+    w.td = (float*)(b + p.td);
+    w.h = (float*)(b + p.h);
+    w.ypart = (float*)(b + p.ypart);
+    w.xn = (uint16_t*)(b + p.xn);
+    w.T = d.T;
+    w.K = d.K;
+    w.E = d.E;
+    w.H = d.H;
+    w.I = d.I;
+    w.Is = d.Is;
+    w.Imax = d.Imax;
+    w.A1 = d.A1;
+    w.C = d.C;
+    w.nb = d.nb;
+    w.J = d.J;
+    w.r = d.r;
+    return w;
+}
+
+LayerArgs args_of(const moe_layer* L) {
+    LayerArgs a;
+    memset(&a, 0, sizeof(a));
+    a.gate = L->gate;
+    a.up = L->up;
+    a.down = L->down;
+    a.s_gate = L->s_gate;
+    a.s_up = L->s_up;
+    a.s_down = L->s_down;
+    a.router = L->router;
+    a.shared_gate = L->shared_gate;
+    a.logit_bias = L->logit_bias;
+    a.H = L->hidden;
+    a.E = L->n_experts;
+    a.K = L->top_k;
+    a.I = L->inter;
+    a.Is = L->s_gate.packed ? L->shared_inter : 0;
+    a.n_adapters = L->n_adapters;
+    a.rank = L->n_adapters > 0 ? L->rank : 0;
+    a.scale = a.rank > 0 ? L->alpha / (float)a.rank : 0.0f;
+    a.has_shared = L->s_gate.packed != nullptr;
+    a.has_sgate = L->shared_gate.packed != nullptr;
+    for (int i = 0; i < L->n_adapters; ++i) a.lora[i] = L->lora[i];
+    return a;
+}
+
+moe_status ws_check(void* ws, size_t ws_bytes, size_t need) {
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < need) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+// The launch sequence shared by moe_ffn_forward and moe_block_forward.
+moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, int T,
+                       const uint16_t* residual, uint16_t* y, const Work& wk, cudaStream_t s) {
+    const LayerArgs la = args_of(L);
+    const moe_qtensor* sg = la.has_sgate ? &L->shared_gate : nullptr;
+    LAUNCH(kRouter, launch_router_logits(x, L->router, sg, L->logit_bias, T, la.H, la.E, wk.logits, wk.gs, s));
+    LAUNCH(kTopk, launch_topk(wk.logits, wk.gs, la.has_sgate, T, la.E, la.K, wk.idx, wk.w, wk.sg, s));
+    CHECK_CUDA(launch_index_build(wk, adapter_id, L->n_adapters, s));
+    // Jobs of the shared expert stay in its group even without a shared expert:
+    // their weights are zero-sized then, so they are skipped by the kernels.
+    const int max_groups = std::min(la.E, T * la.K) + 1;
+    if (la.rank > 0) LAUNCH(kLoraA, launch_lora_a(wk, la, 0, x, s));
+    LAUNCH(kGateUp, launch_gate_up(wk, la, x, max_groups, s));
+    if (la.rank > 0) LAUNCH(kLoraA, launch_lora_a(wk, la, 1, x, s));
+    LAUNCH(kDown, launch_down(wk, la, max_groups, s));
+    LAUNCH(kCombine, launch_combine(wk, residual, y, s));
+    return MOE_OK;
+}
+
+bool mixed_ok(const moe_mixed_tensor* t, int out, int in) {
+    if (!t || !t->packed || !t->scales) return false;
+    if (t->out != out || t->in != in) return false;
+    if (!(t->rho >= 0.0f && t->rho <= 1.0f)) return false;
+    return in % 64 == 0 && aligned(t->packed, 16);
+}
+
+// Super-group size floor(1/rho); the slack absorbs fp32 rounding of rho = 1/n.
+int mixed_G(float rho) { return rho > 0.0f ? (int)floor(1.0 / (double)rho + 1e-6) : 0; }
+
+}  // namespace
+
+extern "C" {
+
+int moe_version(void) { return MOEQ_VERSION; }
+
+const char* moe_status_string(moe_status st) {
+    switch (st) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case MOE_ERR_DEVICE_INDEX: return "device saw an out-of-range expert or adapter index";
+        case MOE_ERR_TIMEOUT: return "bounded device wait timed out";
+    }
+    return "unknown status";
+}
+
+int64_t moe_mixed_words(int32_t out, int32_t in, float rho) {
+    if (out <= 0 || in <= 0 || in % 16) return -1;
+    const int G = mixed_G(rho);
+    const int64_t w4 = in / 8, w2 = in / 16;
+    if (G == 0) return (int64_t)out * w2;
+    const int64_t full = out / G, rem = out % G;
+    return full * (w4 + (int64_t)(G - 1) * w2) + (rem ? w4 + (rem - 1) * w2 : 0);
+}
+
+moe_status moe_quant_pack(moe_format fmt, const float* W, int64_t rows, int32_t in, int32_t group, float rho,
+                          uint32_t* packed, uint16_t* scales, uint16_t* biases, moe_stream stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    CHECK_ARG(rows >= 0 && in > 0);
+    if (rows == 0) return MOE_OK;
+    CHECK_ARG(W && packed && scales);
+    if (fmt == MOE_FMT_AFFINE_INT4 || fmt == MOE_FMT_AFFINE_INT8) {
+        const int bits = fmt == MOE_FMT_AFFINE_INT4 ? 4 : 8;
+        CHECK_ARG(biases && group > 0 && in % group == 0 && group % 8 == 0);
+        timing_begin(s);
+        LAUNCH(kPack, launch_pack_affine(W, rows, in, group, bits, packed, scales, biases, s));
+        return MOE_OK;
+    }
+    if (fmt == MOE_FMT_MIXED_TERNARY_INT4) {
+        CHECK_ARG(biases == nullptr && in % 16 == 0 && rho >= 0.0f && rho <= 1.0f && rows <= INT32_MAX);
+        timing_begin(s);
+        LAUNCH(kPack, launch_pack_mixed(W, (int)rows, in, mixed_G(rho), packed, scales, s));
+        return MOE_OK;
+    }
+    return MOE_ERR_INVALID_ARG;
+}
+
+moe_status moe_dequant(const moe_qtensor* t, float* w_hat, moe_stream stream) {
+    CHECK_ARG(t && w_hat && t->packed && t->scales && t->biases);
+    CHECK_ARG((t->bits == 4 || t->bits == 8) && t->n >= 0 && t->out >= 0 && t->in > 0);
+    CHECK_ARG(t->group > 0 && t->in % t->group == 0 && t->group % 8 == 0);
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    LAUNCH(kDequant, launch_dequant_affine(*t, w_hat, s));
+    return MOE_OK;
+}
+
+moe_status moe_mixed_dequant(const moe_mixed_tensor* t, float* w_hat, moe_stream stream) {
+    CHECK_ARG(t && w_hat && t->packed && t->scales && t->out >= 0 && t->in > 0 && t->in % 16 == 0);
+    CHECK_ARG(t->rho >= 0.0f && t->rho <= 1.0f);
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    LAUNCH(kDequant, launch_dequant_mixed(*t, mixed_G(t->rho), w_hat, s));
+    return MOE_OK;
+}
+
+moe_status moe_router_topk(const uint16_t* x, const moe_qtensor* router, const moe_qtensor* shared_gate,
+                           const float* logit_bias, int32_t T, int32_t H, int32_t E, int32_t K, int32_t* topk_idx,
+                           float* topk_w, float* shared_scale, float* logits, moe_stream stream) {
+    CHECK_ARG(T >= 0);
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && router && topk_idx && topk_w && logits);
+    CHECK_ARG(E > 0 && K > 0 && H > 0 && H % 32 == 0);
+    if (E > MOEQ_MAX_EXPERTS || K > MOEQ_MAX_TOPK || K > E || H > MOEQ_MAX_HIDDEN) return MOE_ERR_UNSUPPORTED;
+    CHECK_ARG(qtensor_ok(*router, 1, E, H, 8));
+    const bool has_sg = shared_gate && shared_gate->packed && shared_scale;
+    if (has_sg) CHECK_ARG(qtensor_ok(*shared_gate, 1, 1, H, 8));
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    LAUNCH(kRouter, launch_router_logits(x, *router, has_sg ? shared_gate : nullptr, logit_bias, T, H, E, logits,
+                                         shared_scale, s));
+    LAUNCH(kTopk, launch_topk(logits, shared_scale, has_sg, T, E, K, topk_idx, topk_w, shared_scale, s));
+    return MOE_OK;
+}
+
+size_t moe_index_workspace_bytes(int32_t T, int32_t K, int32_t E, int32_t n_adapters) {
+    if (T < 0 || K <= 0 || E <= 0 || n_adapters < 0) return 0;
+    const size_t nb = (size_t)(E + 1) * (n_adapters + 1);
+    const size_t C = (size_t)(T + 31) / 32;
+    return kAlign + align_up(nb * C * 4 + 4);
+}
+
+moe_status moe_index_build(const int32_t* topk_idx, const int32_t* adapter_id, int32_t T, int32_t K, int32_t E,
+                           int32_t n_adapters, int32_t* counts, int32_t* offsets, int32_t* perm, void* workspace,
+                           size_t ws_bytes, moe_stream stream) {
+    CHECK_ARG(T >= 0 && K > 0 && E > 0 && n_adapters >= 0);
+    if (E > MOEQ_MAX_EXPERTS || K > MOEQ_MAX_TOPK || n_adapters > MOEQ_MAX_ADAPTERS) return MOE_ERR_UNSUPPORTED;
+    moe_status st = ws_check(workspace, ws_bytes, moe_index_workspace_bytes(T, K, E, n_adapters));
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(topk_idx && counts && offsets && perm && aligned(perm, 16));
+    Work wk;
+    memset(&wk, 0, sizeof(wk));
+    char* b = (char*)workspace;
+    wk.status = (int32_t*)b;
+    wk.cnt = (int32_t*)(b + kAlign);
+    wk.idx = const_cast<int32_t*>(topk_idx);
+    wk.goff = offsets;
+    wk.perm = (int4*)perm;
+    wk.T = T;
+    wk.K = K;
+    wk.E = E;
+    wk.A1 = n_adapters + 1;
+    wk.C = (T + 31) / 32;
+    wk.nb = (E + 1) * wk.A1;
+    wk.J = T * (K + 1);
+    timing_begin((cudaStream_t)stream);
+    CHECK_CUDA(launch_index_build_counts(wk, adapter_id, n_adapters, counts, (cudaStream_t)stream));
+    return MOE_OK;
+}
+
+moe_status lora_set_adapters(moe_layer* layer, int32_t n_adapters, int32_t rank, float alpha,
+                             const moe_lora_ptrs* sets) {
+    CHECK_ARG(layer && n_adapters >= 0 && n_adapters <= MOEQ_MAX_ADAPTERS);
+    if (n_adapters > 0) CHECK_ARG(sets && rank > 0 && rank <= MOEQ_MAX_RANK);
+    for (int a = 0; a < n_adapters; ++a) {
+        const moe_lora_ptrs& p = sets[a];
+        CHECK_ARG(lora_proj_ok(p.gate, 8) && lora_proj_ok(p.up, 8) && lora_proj_ok(p.down, 8) &&
+                  lora_proj_ok(p.s_gate, 8) && lora_proj_ok(p.s_up, 8) && lora_proj_ok(p.s_down, 8));
+    }
+    memset(layer->lora, 0, sizeof(layer->lora));
+    for (int a = 0; a < n_adapters; ++a) layer->lora[a] = sets[a];
+    layer->n_adapters = n_adapters;
+    layer->rank = n_adapters > 0 ? rank : 0;
+    layer->alpha = n_adapters > 0 ? alpha : 0.0f;
+    return MOE_OK;
+}
+
+size_t moe_ffn_workspace_bytes(const moe_layer* layer, int32_t T) {
+    if (!layer || T < 0 || validate_layer(layer) != MOE_OK) return 0;
+    return plan_of(dims_of(layer, T)).total;
+}
+
+moe_status moe_workspace_init(void* workspace, size_t ws_bytes, moe_stream stream) {
+    if (!workspace || !aligned(workspace, kAlign) || ws_bytes < kAlign) return MOE_ERR_WORKSPACE;
+    CHECK_CUDA(cudaMemsetAsync(workspace, 0, kAlign, (cudaStream_t)stream));
+    return MOE_OK;
+}
+
+moe_status moe_ffn_forward(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id, int32_t T,
+                           uint16_t* y, void* workspace, size_t ws_bytes, moe_stream stream) {
+    moe_status st = validate_layer(layer);
+    if (st != MOE_OK) return st;
+    CHECK_ARG(T >= 0);
+    const Dims d = dims_of(layer, T);
+    const WsPlan p = plan_of(d);
+    st = ws_check(workspace, ws_bytes, p.total);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && y && x != y && aligned(x, 16) && aligned(y, 2));
+    timing_begin((cudaStream_t)stream);
+    return ffn_enqueue(layer, x, adapter_id, T, nullptr, y, work_of(d, p, workspace), (cudaStream_t)stream);
+}
+
+moe_status moe_block_forward(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id, int32_t T,
+                             float eps, uint16_t* x_out, void* workspace, size_t ws_bytes, moe_stream stream) {
+    moe_status st = validate_layer(layer);
+    if (st != MOE_OK) return st;
+    CHECK_ARG(T >= 0 && eps >= 0.0f);
+    const Dims d = dims_of(layer, T);
+    const WsPlan p = plan_of(d);
+    st = ws_check(workspace, ws_bytes, p.total);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && x_out && x != x_out && aligned(x, 16) && aligned(x_out, 2));
+    const Work wk = work_of(d, p, workspace);
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    LAUNCH(kRmsnorm, launch_rmsnorm(x, T, d.H, eps, wk.xn, s));
+    return ffn_enqueue(layer, wk.xn, adapter_id, T, x, x_out, wk, s);
+}
+
+moe_status moe_rmsnorm(const uint16_t* x, int32_t T, int32_t H, float eps, uint16_t* xn, moe_stream stream) {
+    CHECK_ARG(T >= 0 && H > 0 && eps >= 0.0f);
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && xn);
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    LAUNCH(kRmsnorm, launch_rmsnorm(x, T, H, eps, xn, s));
+    return MOE_OK;
+}
+
+moe_status moe_get_device_status(void* workspace, moe_stream stream, int32_t* status) {
+    if (!workspace || !aligned(workspace, kAlign)) return MOE_ERR_WORKSPACE;
+    CHECK_ARG(status);
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t v = 0;
+    CHECK_CUDA(cudaMemcpyAsync(&v, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+    CHECK_CUDA(cudaStreamSynchronize(s));
+    CHECK_CUDA(cudaMemsetAsync(workspace, 0, sizeof(int32_t), s));
+    CHECK_CUDA(cudaStreamSynchronize(s));
+    *status = v;
+    return MOE_OK;
+}
+
+moe_status moe_mixed_linear(const moe_mixed_tensor* W, const uint16_t* x, int32_t T, float* y, moe_stream stream) {
+    CHECK_ARG(T >= 0);
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(W && x && y && mixed_ok(W, W->out, W->in) && W->out > 0);
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    LAUNCH(kMixedLinear, launch_mixed_linear(*W, mixed_G(W->rho), x, T, y, s));
+    return MOE_OK;
+}
+
+size_t moe_mixed_mlp_workspace_bytes(int32_t H, int32_t I, int32_t T) {
+    if (H <= 0 || I <= 0 || T < 0) return 0;
+    return align_up((size_t)T * I * 4) + align_up((size_t)T * H * 2) + kAlign;
+}
+
+moe_status moe_mixed_mlp_forward(const moe_mixed_tensor* gate, const moe_mixed_tensor* up,
+                                 const moe_mixed_tensor* down, const uint16_t* x, int32_t T, int32_t residual,
+                                 float eps, uint16_t* y, void* workspace, size_t ws_bytes, moe_stream stream) {
+    CHECK_ARG(T >= 0 && gate && up && down && (residual == 0 || residual == 1));
+    const int I = gate->out, H = gate->in;
+    CHECK_ARG(H > 0 && I > 0 && mixed_ok(gate, I, H) && mixed_ok(up, I, H) && mixed_ok(down, H, I));
+    CHECK_ARG(gate->rho == up->rho && gate->rho == down->rho);
+    moe_status st = ws_check(workspace, ws_bytes, moe_mixed_mlp_workspace_bytes(H, I, T));
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && y && x != y);
+    cudaStream_t s = (cudaStream_t)stream;
+    float* h = (float*)workspace;
+    uint16_t* xn = (uint16_t*)((char*)workspace + align_up((size_t)T * I * 4));
+    const int G = mixed_G(gate->rho);
+    const uint16_t* xin = x;
+    timing_begin(s);
+    if (residual) {
+        LAUNCH(kRmsnorm, launch_rmsnorm(x, T, H, eps, xn, s));
+        xin = xn;
+    }
+    LAUNCH(kMixedGateUp, launch_mixed_gate_up(*gate, *up, G, xin, T, h, s));
+    LAUNCH(kMixedDown, launch_mixed_down(*down, G, h, T, residual ? x : nullptr, y, s));
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,127 @@
+// common.cuh - device helpers and the internal launch interface of libmoeq.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moeq.h"
+
+namespace moeq {
+
+constexpr int kWarp = 32;
+
+// ------------------------------------------------------------------ bf16
+__device__ __forceinline__ float bf16f(uint16_t h) { return __uint_as_float(((uint32_t)h) << 16); }
+__device__ __forceinline__ uint16_t f2bf16(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
+
+// First error wins; later errors do not overwrite it.
+__device__ __forceinline__ void raise_status(int32_t* st, int code) {
+    if (st) atomicCAS(st, 0, code);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// q (0..2^23) as float without an integer-to-float conversion instruction.
+__device__ __forceinline__ float u2f_small(uint32_t q) { return __uint_as_float(0x4B000000u | q) - 8388608.0f; }
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// ------------------------------------------------------------ workspace
+// Device view of the forward workspace.  Offsets are fixed by ws_plan().
+struct Work {
+    int32_t* status;     // sticky error word
+    int32_t* n_active;   // number of experts with at least one job (incl. shared)
+    int32_t* idx;        // [T][K]
+    float* w;            // [T][K]
+    float* sg;           // [T]
+    float* logits;       // [T][E]
+    float* gs;           // [T]
+    int32_t* cnt;        // [nb][C] counts, scanned in place to bases
+    int32_t* goff;       // [E+2] job offset of each expert group (E = shared)
+    int32_t* active;     // [E+1] expert ids of non-empty groups, ascending
+    int4* perm;          // [J] {token, k, adapter, expert}
+    float* wperm;        // [J] combine weight of each job
+    int32_t* inv;        // [T][K+1] position of job (t, k)
+    float* tgu;          // [J][2r] LoRA A products for gate | up
+    float* td;           // [J][r]  LoRA A products for down
+    float* h;            // [J][Imax] SwiGLU activations
+    float* ypart;        // [J][H] per-job weighted outputs
+    uint16_t* xn;        // [T][H] normalised input (block mode)
+    int T, K, E, H, I, Is, Imax, A1, C, nb, J, r;
+};
+
+struct WsPlan {
+    size_t status, n_active, idx, w, sg, logits, gs, cnt, goff, active, perm, wperm, inv, tgu, td, h, ypart, xn;
+    size_t total;
+};
+
+// All the layer fields a kernel needs, passed by value.
+struct LayerArgs {
+    moe_qtensor gate, up, down, s_gate, s_up, s_down, router, shared_gate;
+    const float* logit_bias;
+    int H, E, K, I, Is, n_adapters, rank;
+    float scale;  // alpha / rank
+    bool has_shared, has_sgate;
+    moe_lora_ptrs lora[MOEQ_MAX_ADAPTERS];
+};
+
+// ------------------------------------------------------------- timing
+enum Kind {
+    kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
+    kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kKindCount
+};
+void timing_begin(cudaStream_t s);
+void timing_mark(int kind, cudaStream_t s);
+
+// ------------------------------------------------------------- launchers
+cudaError_t launch_pack_affine(const float* W, int64_t rows, int in, int group, int bits, uint32_t* packed,
+                               uint16_t* scales, uint16_t* biases, cudaStream_t s);
+cudaError_t launch_pack_mixed(const float* W, int out, int in, int G, uint32_t* packed, uint16_t* scales,
+                              cudaStream_t s);
+cudaError_t launch_dequant_affine(const moe_qtensor& t, float* out, cudaStream_t s);
+cudaError_t launch_dequant_mixed(const moe_mixed_tensor& t, int G, float* out, cudaStream_t s);
+
+cudaError_t launch_router_logits(const uint16_t* x, const moe_qtensor& router, const moe_qtensor* sgate,
+                                 const float* logit_bias, int T, int H, int E, float* logits, float* gs,
+                                 cudaStream_t s);
+cudaError_t launch_topk(const float* logits, const float* gs, bool has_sgate, int T, int E, int K, int32_t* idx,
+                        float* w, float* sg, cudaStream_t s);
+
+cudaError_t launch_index_build(const Work& wk, const int32_t* adapter_id, int n_adapters, cudaStream_t s);
+cudaError_t launch_index_build_counts(const Work& wk, const int32_t* adapter_id, int n_adapters,
+                                      int32_t* counts_out, cudaStream_t s);
+
+cudaError_t launch_lora_a(const Work& wk, const LayerArgs& L, int phase, const uint16_t* x, cudaStream_t s);
+cudaError_t launch_gate_up(const Work& wk, const LayerArgs& L, const uint16_t* x, int max_groups, cudaStream_t s);
+cudaError_t launch_down(const Work& wk, const LayerArgs& L, int max_groups, cudaStream_t s);
+cudaError_t launch_combine(const Work& wk, const uint16_t* residual, uint16_t* y, cudaStream_t s);
+
+cudaError_t launch_rmsnorm(const uint16_t* x, int T, int H, float eps, uint16_t* xn, cudaStream_t s);
+
+cudaError_t launch_mixed_linear(const moe_mixed_tensor& W, int G, const uint16_t* x, int T, float* y,
+                                cudaStream_t s);
+cudaError_t launch_mixed_gate_up(const moe_mixed_tensor& g, const moe_mixed_tensor& u, int G, const uint16_t* x,
+                                 int T, float* h, cudaStream_t s);
+cudaError_t launch_mixed_down(const moe_mixed_tensor& d, int G, const float* h, int T, const uint16_t* residual,
+                              uint16_t* y, cudaStream_t s);
+
+// Device row offset (in words) of row `o` of a mixed matrix with super-group size G.
+__host__ __device__ __forceinline__ int64_t mixed_row_offset(int o, int in, int G) {
+    const int64_t w4 = in / 8, w2 = in / 16;
+    if (G == 0) return (int64_t)o * w2;
+    const int64_t sg = o / G, pos = o % G;
+    const int64_t base = sg * (w4 + (int64_t)(G - 1) * w2);
+    return pos == 0 ? base : base + w4 + (pos - 1) * w2;
+}
+
+}  // namespace moeq

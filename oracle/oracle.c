@@ -122,6 +122,7 @@ int orc_quant_affine(const float* W, int64_t rows, int in, int bits, int group, 
                 if (wg[j] < lo) lo = wg[j];
                 if (wg[j] > hi) hi = wg[j];
             }
+            if (lo == 0.0) lo = 0.0; /* a minimum of -0 and +0 stores the bias +0 */
             uint16_t b16 = orc_bf16_round_down(lo);
             double b = orc_bf16_value(b16);
             double d = hi - b;

@@ -1,0 +1,90 @@
+"""Shared pieces of the GPU parity tests: device upload, tolerances, near-tie handling."""
+from __future__ import annotations
+
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.helpers import oracle_layer, quantize_layer, rel_l2
+
+torch = pytest.importorskip("torch")
+
+# Output tolerance of the method: relative L2 <= 5e-3 and max |diff| <= 1e-2 max |y_ref|.
+REL_L2 = 5e-3
+MAX_ABS_FRAC = 1e-2
+# Routing decisions closer than this (K-th vs (K+1)-th logit) may legitimately differ.
+TIE_GAP = 1e-4
+
+
+def need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from int4_group_affine_b200 import build
+    build.build()
+
+
+def assert_close_output(y_gpu, y_ref, what=""):
+    y_gpu = np.asarray(y_gpu, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    r = rel_l2(y_gpu, y_ref)
+    m = float(np.max(np.abs(y_gpu - y_ref))) if y_ref.size else 0.0
+    bound = MAX_ABS_FRAC * float(np.max(np.abs(y_ref))) if y_ref.size else 0.0
+    assert r <= REL_L2, "%s rel-L2 %.3e > %.1e" % (what, r, REL_L2)
+    assert m <= bound, "%s max-abs %.3e > %.3e" % (what, m, bound)
+    return r, m
+
+
+def bf16_dev_to_f64(t):
+    from int4_group_affine_b200.layer import to_host
+    return synth.bf16_to_f32(to_host(t, np.uint16)).astype(np.float64)
+
+
+def near_tie_tokens(logits: np.ndarray, K: int) -> np.ndarray:
+    """Tokens whose K-th and (K+1)-th largest oracle logits are closer than TIE_GAP."""
+    if logits.shape[1] <= K:
+        return np.zeros(logits.shape[0], bool)
+    s = -np.sort(-logits, axis=1)
+    return (s[:, K - 1] - s[:, K]) < TIE_GAP
+
+
+def alternative_sets(z: np.ndarray, K: int):
+    """Every top-K expert set consistent with the oracle logits z up to TIE_GAP ties."""
+    order = sorted(range(len(z)), key=lambda e: (-z[e], e))
+    zk = z[order[K - 1]]
+    sure = [e for e in order if z[e] > zk + TIE_GAP]
+    window = [e for e in order if abs(z[e] - zk) <= TIE_GAP]
+    need = K - len(sure)
+    out = []
+    for comb in itertools.combinations(window, need):
+        s = sure + list(comb)
+        out.append(sorted(s, key=lambda e: (-z[e], e)))
+    return out
+
+
+def check_routing(idx_gpu, idx_ref, logits_ref, K):
+    """Indices bit-exact except near ties, where the GPU's set must be a valid alternative."""
+    ties = near_tie_tokens(logits_ref, K)
+    exact = ~ties
+    assert np.array_equal(idx_gpu[exact], idx_ref[exact])
+    for t in np.nonzero(ties)[0]:
+        alts = [sorted(a) for a in alternative_sets(logits_ref[t], K)]
+        assert sorted(idx_gpu[t].tolist()) in alts
+    return ties
+
+
+def oracle_for_gpu_routing(L, x, aid, idx_gpu, logits_ref, y_ref):
+    """Oracle output per token, re-evaluated (from oracle-derived alternatives) where the
+    GPU resolved a near tie differently."""
+    K = idx_gpu.shape[1]
+    y = y_ref.copy()
+    ties = near_tie_tokens(logits_ref, K)
+    for t in np.nonzero(ties)[0]:
+        for alt in alternative_sets(logits_ref[t], K):
+            if sorted(alt) == sorted(idx_gpu[t].tolist()):
+                sel = np.array([alt], np.int32)
+                a = None if aid is None else aid[t:t + 1]
+                y[t] = L.ffn(x[t:t + 1], a, select=sel)[0][0]
+    return y

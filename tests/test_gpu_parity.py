@@ -1,0 +1,439 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same seeded inputs.
+
+Integer work (packing, codes, routing indices, job lists) must be bit-exact;
+floating-point outputs must meet rel-L2 <= 5e-3 and max-abs <= 1e-2 max|y_ref|.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from synth import workloads
+from tests.gpu_helpers import (REL_L2, assert_close_output, bf16_dev_to_f64, check_routing, need_cuda,
+                               near_tie_tokens, oracle_for_gpu_routing)
+from tests.helpers import oracle_layer, quantize_layer, rel_l2
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    need_cuda()
+
+
+def _mods():
+    import int4_group_affine_b200 as m
+    from int4_group_affine_b200 import layer as ly
+    return m, ly
+
+
+# ------------------------------------------------------------------ packing
+def _special_rows(W):
+    W = W.copy()
+    W[0, :64] = 0.0            # zero group
+    W[1, 64:128] = 0.5         # constant bf16-exact group
+    W[2, :64] = 0.0123         # constant, not bf16-exact
+    W[3, :32] = -0.0
+    W[3, 32:64] = 0.0          # signed zeros mixed
+    return W
+
+
+@pytest.mark.parametrize("bits,group", [(4, 64), (8, 64), (4, 32), (8, 32)])
+def test_pack_affine_bit_exact(bits, group):
+    m, ly = _mods()
+    W = _special_rows(synth.normal(100 + bits, "pack", (37, 512), std=0.02, outlier_prob=1e-2, outlier_factor=20.0))
+    p, s, b = oracle.quant_affine(W, bits, group)
+    Wd = ly.to_device(W)
+    pd = torch.empty((37, 512 * bits // 32), dtype=torch.int32, device="cuda")
+    sd = torch.empty((37, 512 // group), dtype=torch.int16, device="cuda")
+    bd = torch.empty_like(sd)
+    m.moe_quant_pack(m.FMT_AFFINE_INT4 if bits == 4 else m.FMT_AFFINE_INT8, Wd, 37, 512, group, 0.0, pd, sd, bd)
+    torch.cuda.synchronize()
+    assert np.array_equal(ly.to_host(pd, np.uint32), p)
+    assert np.array_equal(ly.to_host(sd, np.uint16), s)
+    assert np.array_equal(ly.to_host(bd, np.uint16), b)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_dequant_bit_exact_zero_error(bits):
+    m, ly = _mods()
+    W = synth.normal(110 + bits, "deq", (3, 5, 256), std=0.02, outlier_prob=1e-2, outlier_factor=20.0)
+    p, s, b = oracle.quant_affine(W, bits, 64)
+    ref = oracle.dequant_affine(p, s, b, 256, bits, 64)
+    t = m.QTensor()
+    pd, sd, bd = ly.to_device(p), ly.to_device(s), ly.to_device(b)
+    t.packed, t.scales, t.biases = pd.data_ptr(), sd.data_ptr(), bd.data_ptr()
+    t.n, t.out, t.in_, t.bits, t.group = 3, 5, 256, bits, 64
+    out = torch.empty((3, 5, 256), dtype=torch.float32, device="cuda")
+    m.moe_dequant(t, out)
+    torch.cuda.synchronize()
+    assert np.max(np.abs(out.cpu().numpy() - ref)) == 0.0
+
+
+@pytest.mark.parametrize("rho", [0.25, 0.5, 1 / 3, 0.0, 1.0, 0.125])
+def test_pack_mixed_bit_exact(rho):
+    m, ly = _mods()
+    W = synth.normal(120, "mpack", (37, 192), std=0.02, outlier_prob=1e-2, outlier_factor=20.0)
+    p, s = oracle.quant_mixed(W, rho)
+    dm = ly.DeviceMixed.from_fp32(ly.to_device(W), rho)
+    torch.cuda.synchronize()
+    assert np.array_equal(ly.to_host(dm.packed, np.uint32), p)
+    assert np.array_equal(ly.to_host(dm.scales, np.uint16), s)
+    out = torch.empty((37, 192), dtype=torch.float32, device="cuda")
+    m.moe_mixed_dequant(dm.T, out)
+    torch.cuda.synchronize()
+    assert np.max(np.abs(out.cpu().numpy() - oracle.dequant_mixed(p, s, 37, 192, rho))) == 0.0
+
+
+# ------------------------------------------------------------------ router
+def _router_case(shape, seed, T):
+    w = workloads.moe_weights(shape, seed=seed)
+    t = quantize_layer(w)
+    L = oracle_layer(shape, t)
+    x, aid = workloads.moe_inputs(shape, seed=seed, T=T)
+    return t, L, x, aid
+
+
+def _gpu_router(t, shape, x, T):
+    m, ly = _mods()
+    d = ly.DeviceLayer.from_host(shape, t)
+    xd = ly.to_device(x)
+    E, K = shape.E, shape.K
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, K), dtype=torch.float32, device="cuda")
+    sg = torch.empty(T, dtype=torch.float32, device="cuda")
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    lb = d.t.get("logit_bias")
+    m.moe_router_topk(xd, d.L.router, d.L.shared_gate, lb, T, shape.H, E, K, idx, w, sg, logits)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), w.cpu().numpy(), sg.cpu().numpy(), logits.cpu().numpy()
+
+
+@pytest.mark.parametrize("shape,T", [(workloads.TINY, 4), (workloads.TINY, 37),
+                                     (dataclasses.replace(workloads.TINY, K=1), 9),
+                                     (dataclasses.replace(workloads.TINY, K=8), 9),
+                                     (dataclasses.replace(workloads.TINY, logit_bias_std=1.0), 40)])
+def test_router_topk_tiny(shape, T):
+    t, L, x, _ = _router_case(shape, 200, T)
+    idx, w, sg, logits = _gpu_router(t, shape, x, T)
+    y, idx_r, w_r, sg_r, logits_r = L.ffn(x)
+    assert np.allclose(logits, logits_r, rtol=1e-5, atol=1e-5)
+    ties = check_routing(idx, idx_r, logits_r, shape.K)
+    assert np.allclose(w[~ties], w_r[~ties], rtol=1e-5, atol=1e-6)
+    assert np.allclose(sg, sg_r, rtol=1e-6, atol=1e-6)
+
+
+def test_router_equal_logits_take_lower_index():
+    m, ly = _mods()
+    shape = dataclasses.replace(workloads.TINY, K=3)
+    w = workloads.moe_weights(shape, seed=201)
+    w["router"][:] = 0.0
+    t = quantize_layer(w)
+    x, _ = workloads.moe_inputs(shape, seed=201, T=5)
+    idx, wts, _, _ = _gpu_router(t, shape, x, 5)
+    assert np.all(idx == np.array([0, 1, 2]))
+    assert np.allclose(wts, 1 / 3, rtol=1e-6)
+
+
+# ------------------------------------------------------------------ index build
+@pytest.mark.parametrize("T,K,E,na", [(1, 4, 256, 1), (5, 2, 8, 0), (37, 4, 16, 4), (100, 8, 64, 2),
+                                      (64, 4, 256, 4), (2048, 4, 256, 1)])
+def test_index_build_bit_exact(T, K, E, na):
+    m, ly = _mods()
+    z = synth.normal(300 + T, "ib/z", (T, E)).astype(np.float64)
+    idx, _ = oracle.topk(z, K)
+    aid = synth.randint(300 + T, "ib/a", (T,), -1, na - 1) if na > 1 else None
+    counts, offsets, perm = oracle.index_build(idx, aid, E, na)
+    nbytes = m.moe_index_workspace_bytes(T, K, E, na)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    c = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    o = torch.empty(E + 2, dtype=torch.int32, device="cuda")
+    p = torch.empty((T * (K + 1), 4), dtype=torch.int32, device="cuda")
+    ad = None if aid is None else ly.to_device(aid)
+    m.moe_index_build(ly.to_device(idx), ad, T, K, E, na, c, o, p, ws, nbytes)
+    torch.cuda.synchronize()
+    assert np.array_equal(c.cpu().numpy(), counts)
+    assert np.array_equal(o.cpu().numpy(), offsets)
+    assert np.array_equal(p.cpu().numpy(), perm)
+    assert m.moe_get_device_status(ws) == 0
+
+
+def test_index_build_flags_out_of_range():
+    m, ly = _mods()
+    T, K, E = 6, 2, 8
+    idx = np.array([[0, 1]] * T, np.int32)
+    idx[2, 1] = 9   # expert out of range
+    aid = np.array([0, 0, 0, 5, 0, 0], np.int32)  # adapter out of range
+    nbytes = m.moe_index_workspace_bytes(T, K, E, 1)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    c = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    o = torch.empty(E + 2, dtype=torch.int32, device="cuda")
+    p = torch.empty((T * (K + 1), 4), dtype=torch.int32, device="cuda")
+    m.moe_index_build(ly.to_device(idx), ly.to_device(aid), T, K, E, 1, c, o, p, ws, nbytes)
+    assert m.moe_get_device_status(ws) == 5
+    assert m.moe_get_device_status(ws) == 0  # read-and-clear
+    assert int(o.cpu().numpy()[-1]) == T * (K + 1)
+
+
+# ------------------------------------------------------------------ FFN tiny
+def _gpu_ffn(d, x, aid=None, block_eps=None):
+    m, ly = _mods()
+    T = x.shape[0]
+    xd = ly.to_device(x)
+    ad = None if aid is None else ly.to_device(aid)
+    ws, nb = d.workspace(T)
+    y = torch.empty_like(xd)
+    if block_eps is None:
+        m.moe_ffn_forward(d.L, xd, ad, T, y, ws, nb)
+    else:
+        m.moe_block_forward(d.L, xd, ad, T, block_eps, y, ws, nb)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status(ws) == 0
+    return y
+
+
+def _ffn_case(shape, seed, T=None, n_adapters=None, lora_zero_B=False):
+    w = workloads.moe_weights(shape, seed=seed, lora_zero_B=lora_zero_B)
+    t = quantize_layer(w)
+    x, aid = workloads.moe_inputs(shape, seed=seed, T=T)
+    return t, x, aid
+
+
+def _check_ffn(shape, t, x, aid, n_adapters=None, what=""):
+    _, ly = _mods()
+    L = oracle_layer(shape, t, n_adapters=n_adapters)
+    d = ly.DeviceLayer.from_host(shape, t, n_adapters=n_adapters)
+    y = bf16_dev_to_f64(_gpu_ffn(d, x, aid))
+    y_ref, idx_r, _, _, logits_r = L.ffn(x, aid)
+    # the GPU's routing (from moe_router_topk, same kernels) decides which oracle output applies
+    ties = near_tie_tokens(logits_r, shape.K)
+    if ties.any():
+        idx_g = _gpu_router(t, shape, x, x.shape[0])[0]
+        y_ref = oracle_for_gpu_routing(L, x, aid, idx_g, logits_r, y_ref)
+    return assert_close_output(y, y_ref, what), y, y_ref
+
+
+@pytest.mark.parametrize("T", [4, 1, 37, 70])
+def test_ffn_tiny(T):
+    shape = workloads.TINY
+    t, x, aid = _ffn_case(shape, 400, T=T)
+    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T)
+
+
+@pytest.mark.parametrize("variant", ["k1", "kE", "no_lora", "no_shared", "no_sgate", "multi_adapter", "bias",
+                                     "group32"])
+def test_ffn_tiny_variants(variant):
+    shape = workloads.TINY
+    na = None
+    if variant == "k1":
+        shape = dataclasses.replace(shape, K=1)
+    elif variant == "kE":
+        shape = dataclasses.replace(shape, K=shape.E)
+    elif variant == "multi_adapter":
+        shape = dataclasses.replace(shape, n_adapters=3, random_adapters=True)
+    elif variant == "bias":
+        shape = dataclasses.replace(shape, logit_bias_std=1.0)
+    elif variant == "group32":
+        shape = dataclasses.replace(shape, group=32)
+    t, x, aid = _ffn_case(shape, 410, T=19)
+    if variant == "group32":
+        w = workloads.moe_weights(shape, seed=410)
+        t = quantize_layer(w, group=32)
+    if variant == "no_lora":
+        na = 0
+    if variant == "no_shared":
+        for k in ("s_gate", "s_up", "s_down"):
+            for suf in ("_p", "_s", "_b"):
+                t[k + suf] = None
+    if variant == "no_sgate":
+        for suf in ("_p", "_s", "_b"):
+            t["sgate" + suf] = None
+    if variant == "multi_adapter":
+        aid = aid.copy()
+        aid[::5] = -1  # some tokens with the base only
+    _check_ffn(shape, t, x, aid, n_adapters=na, what=variant)
+
+
+def test_zero_B_equals_base_bitwise():
+    _, ly = _mods()
+    shape = workloads.TINY
+    t, x, _ = _ffn_case(shape, 420, T=9, lora_zero_B=True)
+    y0 = _gpu_ffn(ly.DeviceLayer.from_host(shape, t), x)
+    yb = _gpu_ffn(ly.DeviceLayer.from_host(shape, t, n_adapters=0), x)
+    assert torch.equal(y0, yb)
+
+
+def test_planted_swap_is_caught():
+    # The tolerance separates the method from its most likely wiring mistake:
+    # the GPU output must be far from an oracle with SiLU on the up branch.
+    _, ly = _mods()
+    shape = workloads.TINY
+    t, x, aid = _ffn_case(shape, 430, T=8)
+    d = ly.DeviceLayer.from_host(shape, t)
+    y = bf16_dev_to_f64(_gpu_ffn(d, x))
+    L = oracle_layer(shape, t)
+    oracle.set_mutation(oracle.MUTATION_SWAP_GATE_UP)
+    try:
+        ym = L.ffn(x)[0]
+    finally:
+        oracle.set_mutation(oracle.MUTATION_NONE)
+    assert rel_l2(y, ym) > 20 * REL_L2
+
+
+def test_bad_adapter_flags_status_and_falls_back_to_base():
+    m, ly = _mods()
+    shape = dataclasses.replace(workloads.TINY, n_adapters=2)
+    t, x, _ = _ffn_case(shape, 440, T=4)
+    aid = np.array([0, 7, 1, -1], np.int32)
+    d = ly.DeviceLayer.from_host(shape, t)
+    xd = ly.to_device(x)
+    ws, nb = d.workspace(4)
+    y = torch.empty_like(xd)
+    m.moe_ffn_forward(d.L, xd, ly.to_device(aid), 4, y, ws, nb)
+    assert m.moe_get_device_status(ws) == 5
+    aid_ok = aid.copy()
+    aid_ok[1] = -1
+    y2 = torch.empty_like(xd)
+    m.moe_ffn_forward(d.L, xd, ly.to_device(aid_ok), 4, y2, ws, nb)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status(ws) == 0
+    assert torch.equal(y, y2)
+
+
+def test_block_tiny():
+    _, ly = _mods()
+    shape = workloads.TINY
+    t, x, aid = _ffn_case(shape, 450, T=11)
+    L = oracle_layer(shape, t)
+    d = ly.DeviceLayer.from_host(shape, t)
+    out = bf16_dev_to_f64(_gpu_ffn(d, x, block_eps=1e-6))
+    ref = synth.bf16_to_f32(L.block(x, eps=1e-6)).astype(np.float64)
+    assert_close_block(out, ref, synth.bf16_to_f32(x).astype(np.float64))
+    # RMSNorm alone: bf16 results equal except where fp32 and fp64 round differently
+    m, _ = _mods()
+    xd = ly.to_device(x)
+    xn = torch.empty_like(xd)
+    m.moe_rmsnorm(xd, x.shape[0], shape.H, 1e-6, xn)
+    torch.cuda.synchronize()
+    got = ly.to_host(xn, np.uint16)
+    exp = oracle.rmsnorm_bf16(x, shape.H, 1e-6)
+    assert np.mean(got == exp) > 0.99
+    assert np.max(np.abs(synth.bf16_to_f32(got).astype(np.float64) - synth.bf16_to_f32(exp))) <= \
+        np.max(np.abs(synth.bf16_to_f32(exp))) * 2.0 ** -7
+
+
+def assert_close_block(out, ref, x):
+    """Block outputs are bf16(x + y): equal up to one bf16 step of the sum plus the FFN tolerance."""
+    y = ref - x
+    tol = np.abs(ref) * 2.0 ** -7 + 1e-2 * np.max(np.abs(y))
+    assert np.all(np.abs(out - ref) <= tol)
+    assert np.mean(out == ref) > 0.8
+
+
+# ------------------------------------------------------------------ full-size layers
+@pytest.fixture(scope="module")
+def full_layer():
+    """The Edge0-35B-shaped layer (seed 0) with 4 adapters and a logit bias, packed by the oracle."""
+    shape = workloads.MULTI_TENANT
+    w = workloads.moe_weights(shape, seed=0)
+    t = quantize_layer(w)
+    return shape, w, t
+
+
+def test_full_size_pack_bit_exact(full_layer):
+    m, ly = _mods()
+    shape, w, t = full_layer
+    weights = {k: ly.to_device(w[k]) for k in ("router", "sgate", "gate", "up", "down", "s_gate", "s_up", "s_down")}
+    d = ly.DeviceLayer.from_fp32(shape, weights)
+    torch.cuda.synchronize()
+    for name in ("router", "sgate", "gate", "up", "down", "s_gate", "s_up", "s_down"):
+        assert np.array_equal(ly.to_host(d.t[name + "_p"], np.uint32), t[name + "_p"]), name
+        assert np.array_equal(ly.to_host(d.t[name + "_s"], np.uint16), t[name + "_s"]), name
+        assert np.array_equal(ly.to_host(d.t[name + "_b"], np.uint16), t[name + "_b"]), name
+
+
+@pytest.mark.parametrize("K,T", [(4, 1), (8, 1), (4, 3)])
+def test_full_size_decode(full_layer, K, T):
+    shape0, w, t = full_layer
+    shape = dataclasses.replace(workloads.DECODE_K4, K=K)
+    tt = dict(t)
+    tt["logit_bias"] = None
+    x, _ = workloads.moe_inputs(shape, seed=500 + K, T=T)
+    _check_ffn(shape, tt, x, None, n_adapters=1, what="decode K=%d T=%d" % (K, T))
+
+
+def test_full_size_multi_tenant(full_layer):
+    shape, w, t = full_layer
+    x, aid = workloads.moe_inputs(shape, seed=0)
+    assert aid is not None and len(np.unique(aid)) == 4
+    _check_ffn(shape, t, x, aid, what="multi-tenant T=64")
+
+
+def test_full_size_prefill_layer_sampled(full_layer):
+    """All 2048 tokens on the GPU; the oracle recomputes a sample of them one by one."""
+    _, ly = _mods()
+    shape0, w, t = full_layer
+    shape = workloads.PREFILL
+    tt = dict(t)
+    tt["logit_bias"] = None
+    x, _ = workloads.moe_inputs(shape, seed=510)
+    d = ly.DeviceLayer.from_host(shape, tt, n_adapters=1)
+    y = bf16_dev_to_f64(_gpu_ffn(d, x))
+    L = oracle_layer(shape, tt, n_adapters=1)
+    sample = np.unique(np.concatenate([[0, 1, 31, 32, 1023, 2046, 2047],
+                                       synth.randint(510, "sample", (17,), 0, shape.T - 1)]))
+    y_ref, idx_r, _, _, logits_r = L.ffn(x[sample])
+    ties = near_tie_tokens(logits_r, shape.K)
+    if ties.any():
+        idx_g = _gpu_router(tt, shape, x[sample], len(sample))[0]
+        y_ref = oracle_for_gpu_routing(L, x[sample], None, idx_g, logits_r, y_ref)
+    assert_close_output(y[sample], y_ref, "prefill sample")
+    assert np.all(np.isfinite(y))
+
+
+# ------------------------------------------------------------------ mixed layout
+@pytest.fixture(scope="module")
+def mixed_layer():
+    s = workloads.MIXED_B1
+    W = workloads.mixed_weights(s, seed=0)
+    q = {n: oracle.quant_mixed(W[n], s.rho) for n in W}
+    return s, W, q
+
+
+@pytest.mark.parametrize("T", [1, 5, 16])
+def test_mixed_linear_full_size(mixed_layer, T):
+    m, ly = _mods()
+    s, W, q = mixed_layer
+    x = workloads.mixed_inputs(s, seed=600 + T, T=T)
+    dm = ly.DeviceMixed.from_host(s.I, s.H, s.rho, *q["gate"])
+    y = torch.empty((T, s.I), dtype=torch.float32, device="cuda")
+    m.moe_mixed_linear(dm.T, ly.to_device(x), T, y)
+    torch.cuda.synchronize()
+    ref = oracle.mixed_linear(q["gate"][0], q["gate"][1], s.I, s.H, s.rho, x)
+    assert rel_l2(y.cpu().numpy(), ref) < 1e-5
+
+
+@pytest.mark.parametrize("T,residual", [(1, 0), (16, 0), (1, 1), (16, 1), (3, 1)])
+def test_mixed_mlp_full_size(mixed_layer, T, residual):
+    m, ly = _mods()
+    s, W, q = mixed_layer
+    x = workloads.mixed_inputs(s, seed=610 + T, T=T)
+    dg = ly.DeviceMixed.from_host(s.I, s.H, s.rho, *q["gate"])
+    du = ly.DeviceMixed.from_host(s.I, s.H, s.rho, *q["up"])
+    dd = ly.DeviceMixed.from_host(s.H, s.I, s.rho, *q["down"])
+    nb = m.moe_mixed_mlp_workspace_bytes(s.H, s.I, T)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    xd = ly.to_device(x)
+    y = torch.empty_like(xd)
+    m.moe_mixed_mlp_forward(dg.T, du.T, dd.T, xd, T, residual, 1e-6, y, ws, nb)
+    torch.cuda.synchronize()
+    out = bf16_dev_to_f64(y)
+    if residual:
+        ref = synth.bf16_to_f32(oracle.mixed_block(q["gate"], q["up"], q["down"], s.H, s.I, s.rho, x)).astype(np.float64)
+        assert_close_block(out, ref, synth.bf16_to_f32(x).astype(np.float64))
+    else:
+        ref = oracle.mixed_mlp(q["gate"], q["up"], q["down"], s.H, s.I, s.rho, x)
+        assert_close_output(out, ref, "mixed mlp")
