@@ -172,6 +172,7 @@ def step_accounting(shape, idx, aid):
     weights = router_bytes(H, E) + U * (gu + d) + sgu + sd + P * sum(lb.values()) + SP * sum(slb.values())
     flops = 2 * T * H * (E + 1) + 2 * T * K * 3 * H * I + 2 * T * 3 * H * Is
     flops += 2 * (T * K) * r * (3 * H + 3 * I) + 2 * T * r * (3 * H + 3 * Is) if r else 0
+    b["lora_a"] /= 2  # two launches per call (gate/up A, then down A)
     return {"kernel_bytes": b, "weight_bytes": weights, "act_bytes": 2 * T * H * 2, "flops": flops, "experts": U}
 
 
@@ -206,6 +207,53 @@ def max_over_ranks(v, world):
     t = torch.tensor([v], dtype=torch.float64, device="cuda")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def capture_steps(step, first, count):
+    """A CUDA graph of `count` consecutive steps (step(i) enqueues on the current stream)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=side):
+        for i in range(count):
+            step(first + i)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    return g
+
+
+def timed_replay(g, world, clocks=None):
+    """Device time (ms) of one replay, bracketed by barrier + synchronize; max over ranks."""
+    import torch
+    g.replay()  # untimed warm-up replay
+    barrier(world)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    t0 = time.time()
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    e1.synchronize()
+    t1 = time.time()
+    barrier(world)
+    return max_over_ranks(e0.elapsed_time(e1), world), t0, t1
+
+
+def kernel_times(moeq, step, first, count):
+    """Per-kernel device time from event nodes recorded inside one graph replay."""
+    import torch
+    moeq.moe_timing_enable(True)
+    try:
+        g = capture_steps(step, first, count)
+        g.replay()
+        torch.cuda.synchronize()
+        kt = moeq.moe_timing_collect()
+    finally:
+        moeq.moe_timing_enable(False)
+    del g
+    return kt
 
 
 # ----------------------------------------------------------------- workload construction
@@ -318,42 +366,28 @@ def run_moe(args, world, rank, local):
             src = xs[0]
             for l, lay in enumerate(layers):
                 dst = xa if l % 2 == 0 else xb
-                moeq.moe_block_forward(lay.L, src, None, T, 1e-6, dst, ws, nbytes, stream)
+                moeq.moe_block_forward(lay.L, src, None, T, 1e-6, dst, ws, nbytes)
                 src = dst
         else:
             i = s % n_inputs
             moeq.moe_ffn_forward(layers[s % copies].L, xs[i], None if aids is None else aids[i], T, ys[s % 2],
-                                 ws, nbytes, stream)
+                                 ws, nbytes)
 
     for s in range(W):
         step(s)
-    barrier(world)
+    torch.cuda.synchronize()
+    g = capture_steps(step, W, K)
     clocks = ClockSampler(local)
-    time.sleep(0.25)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    t_wall0 = time.time()
-    e0.record(stream)
-    for s in range(K):
-        step(W + s)
-    e1.record(stream)
-    e1.synchronize()
-    t_wall1 = time.time()
-    barrier(world)
-    ms = e0.elapsed_time(e1)
-    time.sleep(0.25)
+    time.sleep(0.5)
+    ms, t_wall0, t_wall1 = timed_replay(g, world)
+    time.sleep(0.5)
     clocks.stop()
-    ms = max_over_ranks(ms, world)
+    del g
     ms_step = ms / K
     tokens_per_step = T * (copies if stack else 1)
 
-    # per-kernel durations: the same steps again with library event timing on
-    moeq.moe_timing_enable(True)
-    barrier(world)
-    for s in range(K):
-        step(W + s)
-    kt = moeq.moe_timing_collect()
-    moeq.moe_timing_enable(False)
+    # per-kernel durations: the same steps captured again with library event timing on
+    kt = kernel_times(moeq, step, W, K)
     launches_per_step = sum(c for _, c in kt.values()) / K
 
     # routing of each timed step (for byte accounting), recomputed outside the timed region
@@ -371,7 +405,7 @@ def run_moe(args, world, rank, local):
     roof = None
     if dom is not None:
         dur_ms = kt[dom][0] / kt[dom][1]
-        per_launch = acc["kernel_bytes"].get(dom)
+        per_launch = acc["kernel_bytes"].get({"router_logits": "router"}.get(dom, dom))
         if per_launch is not None:
             gbs = per_launch / (dur_ms * 1e-3) / 1e9
             roof = {"kernel": dom, "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
@@ -463,23 +497,19 @@ def run_e2e(moeq, shape, layers, xs_host, aids_host, K, W, copies, n_inputs, sta
             src = dx
             for l, lay in enumerate(layers):
                 dst = xa if l % 2 == 0 else xb
-                moeq.moe_block_forward(lay.L, src, None, T, 1e-6, dst, ws, nbytes, stream)
+                moeq.moe_block_forward(lay.L, src, None, T, 1e-6, dst, ws, nbytes)
                 src = dst
             hy.copy_(src, non_blocking=True)
         else:
-            moeq.moe_ffn_forward(layers[s % copies].L, dx, da, T, dy, ws, nbytes, stream)
+            moeq.moe_ffn_forward(layers[s % copies].L, dx, da, T, dy, ws, nbytes)
             hy.copy_(dy, non_blocking=True)
 
     for s in range(W):
         step(s)
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for s in range(K):
-        step(W + s)
-    e1.record(stream)
-    e1.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    torch.cuda.synchronize()
+    g = capture_steps(step, W, K)
+    ms, _, _ = timed_replay(g, world)
+    del g
     toks = T * (len(layers) if stack else 1)
     h2d = T * H * 2 + (0 if ha is None else T * 4)
     return {"value": round(toks * K * world / (ms * 1e-3), 2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -521,31 +551,21 @@ def run_mixed(args, world, rank, local):
         for l in range(L):
             m = mats[base + l]
             dst = bufs[l % 2]
-            moeq.moe_mixed_mlp_forward(m["gate"].T, m["up"].T, m["down"].T, src, T, 1, 1e-6, dst, ws, nb, stream)
+            moeq.moe_mixed_mlp_forward(m["gate"].T, m["up"].T, m["down"].T, src, T, 1, 1e-6, dst, ws, nb)
             src = dst
 
     for s in range(W):
         step(s)
-    barrier(world)
+    torch.cuda.synchronize()
+    g = capture_steps(step, W, K)
     clocks = ClockSampler(local)
-    time.sleep(0.25)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0 = time.time()
-    e0.record(stream)
-    for s in range(K):
-        step(W + s)
-    e1.record(stream)
-    e1.synchronize()
-    t1 = time.time()
-    time.sleep(0.25)
+    time.sleep(0.5)
+    ms, t0, t1 = timed_replay(g, world)
+    time.sleep(0.5)
     clocks.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    del g
     ms_step = ms / K
-    moeq.moe_timing_enable(True)
-    for s in range(K):
-        step(W + s)
-    kt = moeq.moe_timing_collect()
-    moeq.moe_timing_enable(False)
+    kt = kernel_times(moeq, step, W, K)
     layer_bytes = sum(m.nbytes() for m in mats[0].values())
     peaks, src = measured_peaks()
     hbm = float(peaks["hbm_gbs"])

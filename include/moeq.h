@@ -16,9 +16,10 @@
  *  - Every function returns a moe_status.  Argument errors are detected on the
  *    host before anything is enqueued and return MOE_ERR_INVALID_ARG or
  *    MOE_ERR_UNSUPPORTED; a failed launch returns MOE_ERR_CUDA.  Problems that
- *    only the device can see (an expert or adapter index out of range in
- *    caller-supplied routing) set a sticky status word inside the workspace
- *    (read with moe_get_device_status); the offending job contributes zero.
+ *    only the device can see set a sticky status word inside the workspace
+ *    (read with moe_get_device_status): an expert index out of range in
+ *    caller-supplied routing makes that job contribute zero; an adapter id out
+ *    of range runs that token on the base weights alone.
  *
  * Storage formats:
  *  - Affine (int4 or int8), groups of `group` consecutive input elements
@@ -265,8 +266,9 @@ MOEQ_API moe_status moe_mixed_mlp_forward(const moe_mixed_tensor* gate, const mo
  * kernel after it).  moe_timing_collect synchronises on the recorded events,
  * adds each kind's time (ms) and launch count into the host arrays (n_kinds
  * entries, indexed by kind) and clears the record.  At most 1 << 16 launches
- * are recorded between collects; later ones are not timed.  Enabling is not
- * thread-safe and must not overlap stream capture. */
+ * are recorded between collects; later ones are not timed.  Under stream
+ * capture the records become event nodes of the graph; collect after exactly
+ * one replay of that graph.  Enabling is not thread-safe. */
 MOEQ_API int moe_timing_kinds(void);
 MOEQ_API const char* moe_timing_kind_name(int kind);
 MOEQ_API moe_status moe_timing_enable(int enable);

@@ -75,6 +75,17 @@ struct LayerArgs {
     moe_lora_ptrs lora[MOEQ_MAX_ADAPTERS];
 };
 
+// Raise a kernel's dynamic shared-memory limit to at least `bytes`, calling the
+// runtime only when the cached limit is too small (so repeated launches, and
+// launches during stream capture, do not call it again).  The cache assumes one
+// device per process.
+inline cudaError_t ensure_smem(const void* fn, size_t bytes, int& cached) {
+    if (bytes <= 48 * 1024 || (int)bytes <= cached) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) cached = (int)bytes;
+    return e;
+}
+
 // ------------------------------------------------------------- timing
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,

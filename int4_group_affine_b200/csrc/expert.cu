@@ -341,7 +341,8 @@ cudaError_t launch_gate_up(const Work& wk, const LayerArgs& L, const uint16_t* x
     const int64_t items = (int64_t)max_groups * ntiles;
     const int grid = (int)(items < num_sms() * 4 ? items : num_sms() * 4);
     const size_t smem = (size_t)kTok * L.H * sizeof(float) + (size_t)kTok * (L.H / 32) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int cached = 0;
+    cudaError_t e = ensure_smem((const void*)gate_up_kernel, smem, cached);
     if (e != cudaSuccess) return e;
     gate_up_kernel<<<grid, kGUWarps * 32, smem, s>>>(wk, L, x);
     return cudaGetLastError();
@@ -353,7 +354,8 @@ cudaError_t launch_down(const Work& wk, const LayerArgs& L, int max_groups, cuda
     const int64_t items = (int64_t)max_groups * ntiles;
     const int grid = (int)(items < num_sms() * 8 ? items : num_sms() * 8);
     const size_t smem = (size_t)kTok * wk.Imax * sizeof(float) + (size_t)kTok * (wk.Imax / 32) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int cached = 0;
+    cudaError_t e = ensure_smem((const void*)down_kernel, smem, cached);
     if (e != cudaSuccess) return e;
     down_kernel<<<grid, kDWarps * 32, smem, s>>>(wk, L);
     return cudaGetLastError();

@@ -16,18 +16,20 @@ namespace {
 
 struct JobKey {
     int expert, adapter, bucket;
-    bool bad;
+    bool bad;         // some index was out of range (flags the status)
+    bool bad_expert;  // the job cannot run: its weight becomes 0
 };
 
 // Same mapping in count and scatter: an out-of-range expert becomes expert 0
-// with weight 0, an out-of-range adapter becomes "none"; both flag the status.
+// with weight 0; an out-of-range adapter becomes "none" (the token runs on the
+// base weights); both flag the status.
 __device__ __forceinline__ JobKey job_key(const Work& wk, const int32_t* adapter_id, int n_adapters, int t, int k) {
     JobKey j;
-    j.bad = false;
+    j.bad = j.bad_expert = false;
     int e = k < wk.K ? wk.idx[(int64_t)t * wk.K + k] : wk.E;
     if (k < wk.K && (e < 0 || e >= wk.E)) {
         e = 0;
-        j.bad = true;
+        j.bad = j.bad_expert = true;
     }
     int a = adapter_id ? adapter_id[t] : (n_adapters > 0 ? 0 : -1);
     if (a < -1 || a >= n_adapters) {
@@ -140,7 +142,7 @@ __global__ void index_scatter_kernel(Work wk, const int32_t* __restrict__ adapte
         wk.perm[pos] = make_int4(t, k, j.adapter, j.expert);
         if (wk.wperm) {
             float wt = k < wk.K ? wk.w[(int64_t)t * wk.K + k] : wk.sg[t];
-            wk.wperm[pos] = j.bad ? 0.0f : wt;
+            wk.wperm[pos] = j.bad_expert ? 0.0f : wt;
         }
         if (wk.inv) wk.inv[(int64_t)t * (wk.K + 1) + k] = pos;
     }

@@ -177,8 +177,9 @@ mixed_down_kernel(moe_mixed_tensor Wd, int G, const float* __restrict__ h, int T
 }
 
 cudaError_t set_smem(const void* fn, size_t smem) {
-    if (smem <= 48 * 1024) return cudaSuccess;
-    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int c_lin = 0, c_gu = 0, c_down = 0;
+    int& c = fn == (const void*)mixed_linear_kernel ? c_lin : fn == (const void*)mixed_gate_up_kernel ? c_gu : c_down;
+    return ensure_smem(fn, smem, c);
 }
 
 size_t stage_bytes(int n) { return (size_t)kMT * n * sizeof(float) + (size_t)kMT * (n / 32) * sizeof(float); }

@@ -162,14 +162,14 @@ cudaError_t launch_router_logits(const uint16_t* x, const moe_qtensor& router, c
     dim3 grid((R + kRouterRows - 1) / kRouterRows, (T + tok - 1) / tok);
     const size_t smem = (size_t)tok * H * sizeof(float);
     if (tok == kRouterTokMax) {
-        cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<kRouterTokMax>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        static int cached = 0;
+        cudaError_t e = ensure_smem((const void*)router_logits_kernel<kRouterTokMax>, smem, cached);
         if (e != cudaSuccess) return e;
         router_logits_kernel<kRouterTokMax>
             <<<grid, kRouterWarps * 32, smem, s>>>(x, router, sg, has, logit_bias, T, H, E, logits, gs);
     } else {
-        cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<kRouterTokMax / 2>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        static int cached = 0;
+        cudaError_t e = ensure_smem((const void*)router_logits_kernel<kRouterTokMax / 2>, smem, cached);
         if (e != cudaSuccess) return e;
         router_logits_kernel<kRouterTokMax / 2>
             <<<grid, kRouterWarps * 32, smem, s>>>(x, router, sg, has, logit_bias, T, H, E, logits, gs);

@@ -29,13 +29,26 @@ void record(int kind, cudaStream_t s) {
         if (cudaEventCreate(&ev) != cudaSuccess) return;
         g_pool.push_back(ev);
     }
-    if (cudaEventRecord(g_pool[i], s) != cudaSuccess) return;
+    // Under stream capture the record becomes an event node of the graph, so the
+    // times come from the graph's replay.
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return;
+    const cudaError_t e = cap == cudaStreamCaptureStatusActive
+                              ? cudaEventRecordWithFlags(g_pool[i], s, cudaEventRecordExternal)
+                              : cudaEventRecord(g_pool[i], s);
+    if (e != cudaSuccess) return;
     g_recs.push_back(Rec{kind});
 }
 
 }  // namespace
 
-void timing_begin(cudaStream_t s) { record(-1, s); }
+// Start of an entry point's launch sequence.  Also drops a stale, non-sticky
+// error left by an earlier runtime call, so that the launch checks that follow
+// report this call's launches only (sticky device errors persist regardless).
+void timing_begin(cudaStream_t s) {
+    (void)cudaGetLastError();
+    record(-1, s);
+}
 void timing_mark(int kind, cudaStream_t s) { record(kind, s); }
 
 }  // namespace moeq
@@ -60,15 +73,20 @@ moe_status moe_timing_collect(float* total_ms, int32_t* launches, int32_t n_kind
         g_recs.clear();
         return MOE_ERR_CUDA;
     }
+    bool missing = false;
     for (size_t i = 1; i < g_recs.size(); ++i) {
         const int k = g_recs[i].kind;
         if (k < 0 || k >= n_kinds) continue;
         float ms = 0.0f;
-        if (cudaEventElapsedTime(&ms, g_pool[i - 1], g_pool[i]) != cudaSuccess) continue;
+        if (cudaEventElapsedTime(&ms, g_pool[i - 1], g_pool[i]) != cudaSuccess) {
+            missing = true;  // e.g. events of a captured graph that was not replayed
+            continue;
+        }
         total_ms[k] += ms;
         launches[k] += 1;
     }
     g_recs.clear();
+    if (missing) (void)cudaGetLastError();  // do not leave the query's error for the next launch check
     return MOE_OK;
 }
 

@@ -350,9 +350,10 @@ def test_full_size_pack_bit_exact(full_layer):
     d = ly.DeviceLayer.from_fp32(shape, weights)
     torch.cuda.synchronize()
     for name in ("router", "sgate", "gate", "up", "down", "s_gate", "s_up", "s_down"):
-        assert np.array_equal(ly.to_host(d.t[name + "_p"], np.uint32), t[name + "_p"]), name
-        assert np.array_equal(ly.to_host(d.t[name + "_s"], np.uint16), t[name + "_s"]), name
-        assert np.array_equal(ly.to_host(d.t[name + "_b"], np.uint16), t[name + "_b"]), name
+        for suf, dt in (("_p", np.uint32), ("_s", np.uint16), ("_b", np.uint16)):
+            got = ly.to_host(d.t[name + suf], dt)
+            assert got.size == t[name + suf].size, name + suf
+            assert np.array_equal(got.ravel(), t[name + suf].ravel()), name + suf
 
 
 @pytest.mark.parametrize("K,T", [(4, 1), (8, 1), (4, 3)])
