@@ -227,6 +227,31 @@ MOEQ_API moe_status moe_workspace_init(void* workspace, size_t ws_bytes, moe_str
 MOEQ_API moe_status moe_ffn_forward(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id, int32_t T,
                            uint16_t* y, void* workspace, size_t ws_bytes, moe_stream stream);
 
+/* ------------------------------------------ forward without device allocation
+ * No counterpart on the pages: this entry point exists for callers that cannot
+ * allocate device memory at the point where they run the layer (an engine's
+ * enqueue hook or plugin that must not allocate, a serving runtime that has
+ * reserved all device memory up front, or code that cannot afford the implicit
+ * synchronisation an allocation may cause).  It computes exactly what
+ * moe_ffn_forward computes, on the same kernels, but takes its workspace from
+ * a fixed array of MOEQ_STATIC_WS_BYTES compiled into the library; every device
+ * that loads the library holds that array until the process exits.  The caller
+ * still passes x, adapter_id and y (device pointers, as for moe_ffn_forward).
+ *  - Returns MOE_ERR_WORKSPACE, enqueuing nothing, when
+ *    moe_ffn_workspace_bytes(layer, T) exceeds MOEQ_STATIC_WS_BYTES (16 MiB:
+ *    e.g. up to about 300 tokens of the 2048-hidden, 256-expert, top-4 layer).
+ *  - The first call on a device looks up the array's device address there
+ *    (once per device, with that device current); make that first call before
+ *    any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents: each
+ *    call clears the status header it needs zeroed, and calls that overlap on
+ *    the GPU (on different streams, or from several host threads) race on it.
+ *    Order them on one stream.
+ *  - No device memory is allocated or freed. */
+#define MOEQ_STATIC_WS_BYTES (16u * 1024u * 1024u)
+MOEQ_API moe_status moe_ffn_forward_static(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id,
+                                           int32_t T, uint16_t* y, moe_stream stream);
+
 /* Pre-norm residual block for stacked layers:
  *   x_out = bf16(x + FFN(bf16(RMSNorm(x)))), RMSNorm with unit weight and eps.
  * x_out may not alias x.  Same workspace rules as moe_ffn_forward. */

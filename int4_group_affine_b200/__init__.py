@@ -164,3 +164,10 @@ def moe_timing_collect() -> dict:
     cnt = (ctypes.c_int32 * n)()
     _check("moe_timing_collect", L.moe_timing_collect(ms, cnt, n))
     return {L.moe_timing_kind_name(k).decode(): (float(ms[k]), int(cnt[k])) for k in range(n) if cnt[k]}
+
+
+def moe_ffn_forward_static(layer: Layer, x, adapter_id, T, y, stream=None):
+    """moe_ffn_forward with the library's built-in device workspace (no allocation anywhere)."""
+    _check("moe_ffn_forward_static", _lib.lib().moe_ffn_forward_static(ctypes.byref(layer), _ptr(x),
+                                                                       _ptr(adapter_id), T, _ptr(y),
+                                                                       _stream(stream)))

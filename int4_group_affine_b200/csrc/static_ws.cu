@@ -1,0 +1,59 @@
+// static_ws.cu - moe_ffn_forward_static: the MoE FFN forward with its scratch in
+// a fixed device array compiled into the library, for callers that cannot
+// allocate device memory.
+//
+// Who needs it: code that runs where a device allocation is not allowed or not
+// safe, for example an inference engine's enqueue hook or plugin that must not
+// allocate, a serving runtime that reserves all device memory up front, or a
+// caller that cannot afford the implicit device synchronisation an allocation
+// may cause.  Those callers still pass the inputs and the output; only the
+// workspace comes from here.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace {
+
+// The scratch of every moe_ffn_forward_static call, on every device that loads
+// the library, held until the process exits.  In host code this name is only a
+// stand-in for the symbol; kernels receive the device address obtained below.
+static __device__ __align__(256) unsigned char g_static_ws[MOEQ_STATIC_WS_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_dev_ptr[kMaxDevices] = {};
+
+// Device address of g_static_ws on the current device, looked up once per device.
+moe_status static_ws_address(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_dev_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) {
+            (void)cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        g_dev_ptr[dev] = p;
+    }
+    *out = g_dev_ptr[dev];
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_ffn_forward_static(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id,
+                                             int32_t T, uint16_t* y, moe_stream stream) {
+    if (T < 0) return MOE_ERR_INVALID_ARG;
+    const size_t need = moe_ffn_workspace_bytes(layer, T);
+    if (need == 0) return MOE_ERR_INVALID_ARG;  // the layer itself was rejected
+    if (need > (size_t)MOEQ_STATIC_WS_BYTES) return MOE_ERR_WORKSPACE;
+    void* ws = nullptr;
+    moe_status st = static_ws_address(&ws);
+    if (st != MOE_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    // The array keeps the previous call's contents: the status header must
+    // start at zero (everything else is written before it is read).
+    if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return moe_ffn_forward(layer, x, adapter_id, T, y, ws, need, stream);
+}
