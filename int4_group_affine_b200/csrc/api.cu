@@ -111,8 +111,9 @@ WsPlan plan_of(const Dims& d) {
         o = align_up(o + bytes);
         return at;
     };
-    p.status = take(8);  // status word + n_active share the first 256 bytes
+    p.status = take(16);  // status word, n_active and the decode barrier share the first 256 bytes
     p.n_active = p.status + 4;
+    p.bar = p.status + 8;
     p.idx = take((size_t)d.T * d.K * 4);
     p.w = take((size_t)d.T * d.K * 4);
     p.sg = take((size_t)d.T * 4);
@@ -129,6 +130,11 @@ WsPlan plan_of(const Dims& d) {
     p.h = take((size_t)d.J * d.Imax * 4);
     p.ypart = take((size_t)d.J * d.H * 4);
     p.xn = take((size_t)d.T * d.H * 2);
+    const bool dec = d.T <= MOEQ_DECODE_MAX_TOKENS && d.J <= MOEQ_DECODE_MAX_JOBS;
+    p.dts = take(dec ? (size_t)d.T * 2 * d.r * 4 : 0);
+    p.dtg = take(dec ? (size_t)d.T * d.K * 2 * d.r * 4 : 0);
+    p.dgus = take(dec ? (size_t)d.T * std::max(d.Is, 1) * 2 * 4 : 0);
+    p.dtdp = take(dec ? (size_t)MOEQ_DECODE_MAX_CTAS * d.J * d.r * 4 : 0);
     p.total = o;
     return p;
 }
@@ -217,6 +223,35 @@ moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* ada
     LAUNCH(kDown, launch_down(wk, la, max_groups, s));
     LAUNCH(kCombine, launch_combine(wk, residual, y, s));
     return MOE_OK;
+}
+
+// The single fused kernel for a few tokens (csrc/decode.cu).  Returns false when
+// it does not apply (too many tokens or jobs, shapes outside its limits), so the
+// caller runs the multi-kernel path instead; otherwise *st is the launch result.
+bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, int T, int block, float eps,
+                uint16_t* y, const Dims& d, const WsPlan& p, void* ws, cudaStream_t s, moe_status* st) {
+    if (d.T > MOEQ_DECODE_MAX_TOKENS || d.J > MOEQ_DECODE_MAX_JOBS) return false;
+    const LayerArgs la = args_of(L);
+    if (!decode_supported(la, T, nullptr)) return false;
+    char* b = (char*)ws;
+    DecodeScratch sc;
+    sc.logits = (float*)(b + p.logits);
+    sc.gsl = (float*)(b + p.gs);
+    sc.ts = (float*)(b + p.dts);
+    sc.tg = (float*)(b + p.dtg);
+    sc.gus = (float*)(b + p.dgus);
+    sc.h = (float*)(b + p.h);
+    sc.tdp = (float*)(b + p.dtdp);
+    sc.bar = (unsigned long long*)(b + p.bar);
+    sc.status = (int32_t*)(b + p.status);
+    const cudaError_t e = launch_decode(la, x, adapter_id, y, T, block, eps, sc, s);
+    if (e == cudaErrorNotSupported || e == cudaErrorCooperativeLaunchTooLarge) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    *st = e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (e == cudaSuccess) timing_mark(kDecode, s);
+    return true;
 }
 
 bool mixed_ok(const moe_mixed_tensor* t, int out, int in) {
@@ -392,8 +427,10 @@ moe_status moe_ffn_forward(const moe_layer* layer, const uint16_t* x, const int3
     if (st != MOE_OK) return st;
     if (T == 0) return MOE_OK;
     CHECK_ARG(x && y && x != y && aligned(x, 16) && aligned(y, 2));
-    timing_begin((cudaStream_t)stream);
-    return ffn_enqueue(layer, x, adapter_id, T, nullptr, y, work_of(d, p, workspace), (cudaStream_t)stream);
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    if (try_decode(layer, x, adapter_id, T, 0, 0.0f, y, d, p, workspace, s, &st)) return st;
+    return ffn_enqueue(layer, x, adapter_id, T, nullptr, y, work_of(d, p, workspace), s);
 }
 
 moe_status moe_block_forward(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id, int32_t T,
@@ -410,6 +447,7 @@ moe_status moe_block_forward(const moe_layer* layer, const uint16_t* x, const in
     const Work wk = work_of(d, p, workspace);
     cudaStream_t s = (cudaStream_t)stream;
     timing_begin(s);
+    if (try_decode(layer, x, adapter_id, T, 1, eps, x_out, d, p, workspace, s, &st)) return st;
     LAUNCH(kRmsnorm, launch_rmsnorm(x, T, d.H, eps, wk.xn, s));
     return ffn_enqueue(layer, wk.xn, adapter_id, T, x, x_out, wk, s);
 }

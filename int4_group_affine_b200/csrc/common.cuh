@@ -62,6 +62,7 @@ struct Work {
 
 struct WsPlan {
     size_t status, n_active, idx, w, sg, logits, gs, cnt, goff, active, perm, wperm, inv, tgu, td, h, ypart, xn;
+    size_t bar, dts, dtg, dgus, dtdp;  // fused decode scratch (sizes zero when T is too large for it)
     size_t total;
 };
 
@@ -86,10 +87,22 @@ inline cudaError_t ensure_smem(const void* fn, size_t bytes, int& cached) {
     return e;
 }
 
+// ------------------------------------------------------------- fused decode
+#define MOEQ_DECODE_MAX_TOKENS 8
+#define MOEQ_DECODE_MAX_JOBS 32
+#define MOEQ_DECODE_MAX_CTAS 256
+
+// Scratch of the fused decode kernel (all inside the forward workspace).
+struct DecodeScratch {
+    float *logits, *gsl, *ts, *tg, *gus, *h, *tdp;
+    unsigned long long* bar;  // monotonic arrival counter: starts zeroed (workspace header)
+    int32_t* status;
+};
+
 // ------------------------------------------------------------- timing
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
-    kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kKindCount
+    kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kKindCount
 };
 void timing_begin(cudaStream_t s);
 void timing_mark(int kind, cudaStream_t s);
@@ -118,6 +131,10 @@ cudaError_t launch_down(const Work& wk, const LayerArgs& L, int max_groups, cuda
 cudaError_t launch_combine(const Work& wk, const uint16_t* residual, uint16_t* y, cudaStream_t s);
 
 cudaError_t launch_rmsnorm(const uint16_t* x, int T, int H, float eps, uint16_t* xn, cudaStream_t s);
+
+bool decode_supported(const LayerArgs& L, int T, size_t* smem_out);
+cudaError_t launch_decode(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, uint16_t* y, int T,
+                          int block, float eps, const DecodeScratch& sc, cudaStream_t s);
 
 cudaError_t launch_mixed_linear(const moe_mixed_tensor& W, int G, const uint16_t* x, int T, float* y,
                                 cudaStream_t s);
