@@ -16,6 +16,7 @@ using namespace moeq;
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr int kTcMinTokens = 16;  // from this many tokens on, the expert GEMMs use the tensor cores
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
@@ -217,6 +218,17 @@ moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* ada
     // Jobs of the shared expert stay in its group even without a shared expert:
     // their weights are zero-sized then, so they are skipped by the kernels.
     const int max_groups = std::min(la.E, T * la.K) + 1;
+    if (T >= kTcMinTokens && tc_supported(la)) {
+        // many tokens: expert-grouped GEMMs on the tcgen05 tensor cores; the SwiGLU
+        // activations go to the workspace's h region as bf16 (the down GEMM's operand)
+        uint16_t* hb = reinterpret_cast<uint16_t*>(wk.h);
+        if (la.rank > 0) LAUNCH(kTcLoraGUKind, launch_tc_gemm(la, kTcLoraGU, x, la.H, wk, nullptr, wk.Imax, s));
+        LAUNCH(kTcGUKind, launch_tc_gemm(la, kTcGU, x, la.H, wk, hb, wk.Imax, s));
+        if (la.rank > 0) LAUNCH(kTcLoraDownKind, launch_tc_gemm(la, kTcLoraDown, hb, wk.Imax, wk, nullptr, wk.Imax, s));
+        LAUNCH(kTcDownKind, launch_tc_gemm(la, kTcDown, hb, wk.Imax, wk, nullptr, wk.Imax, s));
+        LAUNCH(kCombine, launch_combine(wk, residual, y, s));
+        return MOE_OK;
+    }
     if (la.rank > 0) LAUNCH(kLoraA, launch_lora_a(wk, la, 0, x, s));
     LAUNCH(kGateUp, launch_gate_up(wk, la, x, max_groups, s));
     if (la.rank > 0) LAUNCH(kLoraA, launch_lora_a(wk, la, 1, x, s));

@@ -102,7 +102,8 @@ struct DecodeScratch {
 // ------------------------------------------------------------- timing
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
-    kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kKindCount
+    kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kTcLoraGUKind, kTcGUKind,
+    kTcLoraDownKind, kTcDownKind, kKindCount
 };
 void timing_begin(cudaStream_t s);
 void timing_mark(int kind, cudaStream_t s);
@@ -131,6 +132,12 @@ cudaError_t launch_down(const Work& wk, const LayerArgs& L, int max_groups, cuda
 cudaError_t launch_combine(const Work& wk, const uint16_t* residual, uint16_t* y, cudaStream_t s);
 
 cudaError_t launch_rmsnorm(const uint16_t* x, int T, int H, float eps, uint16_t* xn, cudaStream_t s);
+
+// tcgen05 grouped GEMM modes (csrc/prefill.cu)
+enum TcMode { kTcGU = 0, kTcDown = 1, kTcLoraGU = 2, kTcLoraDown = 3 };
+bool tc_supported(const LayerArgs& L);
+cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, int ld_act, const Work& wk,
+                           const uint16_t* hb_out, int ldh, cudaStream_t s);
 
 bool decode_supported(const LayerArgs& L, int T, size_t* smem_out);
 cudaError_t launch_decode(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, uint16_t* y, int T,
