@@ -155,25 +155,74 @@ def routing_stats(idx, aid, K, n_adapters):
 
 
 def step_accounting(shape, idx, aid):
-    """Algorithmic bytes (touched weights + activations) and flops of one layer call."""
+    """Algorithmic bytes and flops of one layer call, per kernel unit and in total.
+
+    Bytes: the weights a unit must touch (distinct experts, distinct expert-adapter
+    pairs for LoRA) plus its activation inputs and outputs in the path's formats
+    (x bf16, h bf16, per-job outputs fp32).  Flops: 2 per multiply-add the method
+    defines (LoRA-A of the adapter each job uses only)."""
     H, E, K, I, Is, r, T = shape.H, shape.E, shape.K, shape.I, shape.Is, shape.rank, idx.shape[0]
     gu, d = expert_bytes(H, I)
     sgu, sd = expert_bytes(H, Is)
     lb = lora_bytes(H, I, r)
     slb = lora_bytes(H, Is, r)
     U, P, SP = routing_stats(idx, aid, K, shape.n_adapters)
+    TK = T * K
     J = T * (K + 1)
+    h_bytes = (TK * I + T * Is) * 2
     b = {
-        "router": router_bytes(H, E) + T * H * 2,
-        "gate_up": U * gu + sgu + P * lb["B_gu"] + SP * slb["B_gu"] + T * H * 2,
-        "down": U * d + sd + P * lb["B_d"] + SP * slb["B_d"] + J * (I * 4 + H * 4),
-        "lora_a": P * (lb["A_gu"] + lb["A_d"]) + SP * (slb["A_gu"] + slb["A_d"]),
+        "router": router_bytes(H, E) + T * H * 2 + T * E * 4,
+        "gate_up": U * gu + sgu + P * lb["B_gu"] + SP * slb["B_gu"] + T * H * 2 + h_bytes,
+        "down": U * d + sd + P * lb["B_d"] + SP * slb["B_d"] + h_bytes + J * H * 4,
+        "lora_gu": P * lb["A_gu"] + SP * slb["A_gu"] + T * H * 2,
+        "lora_down": P * lb["A_d"] + SP * slb["A_d"] + h_bytes,
+    }
+    f = {
+        "router": 2 * T * H * (E + 1),
+        "gate_up": 2 * TK * 2 * H * I + 2 * T * 2 * H * Is + (2 * TK * 2 * I * r + 2 * T * 2 * Is * r if r else 0),
+        "down": 2 * TK * H * I + 2 * T * H * Is + (2 * TK * H * r + 2 * T * H * r if r else 0),
+        "lora_gu": 2 * TK * 2 * r * H + 2 * T * 2 * r * H if r else 0,
+        "lora_down": 2 * TK * r * I + 2 * T * r * Is if r else 0,
     }
     weights = router_bytes(H, E) + U * (gu + d) + sgu + sd + P * sum(lb.values()) + SP * sum(slb.values())
-    flops = 2 * T * H * (E + 1) + 2 * T * K * 3 * H * I + 2 * T * 3 * H * Is
-    flops += 2 * (T * K) * r * (3 * H + 3 * I) + 2 * T * r * (3 * H + 3 * Is) if r else 0
-    b["lora_a"] /= 2  # two launches per call (gate/up A, then down A)
-    return {"kernel_bytes": b, "weight_bytes": weights, "act_bytes": 2 * T * H * 2, "flops": flops, "experts": U}
+    act = 2 * T * H * 2
+    b["layer"] = weights + act
+    f["layer"] = sum(f.values())
+    b["lora_a"] = (b["lora_gu"] + b["lora_down"]) / 2  # the CUDA-core LoRA-A kernel runs twice per call
+    f["lora_a"] = (f["lora_gu"] + f["lora_down"]) / 2
+    return {"kernel_bytes": b, "kernel_flops": f, "weight_bytes": weights, "act_bytes": act, "flops": f["layer"],
+            "experts": U}
+
+
+# library timing kind -> accounting unit
+KIND_UNIT = {"router_logits": "router", "tc_router": "router", "gate_up": "gate_up", "tc_gate_up": "gate_up",
+             "down": "down", "tc_down": "down", "lora_a": "lora_a", "tc_lora_gate_up": "lora_gu",
+             "tc_lora_down": "lora_down", "decode_fused": "layer"}
+
+
+def kernel_roofline(kind, dur_ms, nbytes, nflops, peaks, src, timed_s):
+    """Roofline entry of one kernel: the bound is whichever of HBM time and bf16
+    tensor time is larger for its algorithmic bytes and flops; the tensor peak is
+    the burst figure for a timed region under a second, else the sustained one."""
+    hbm = float(peaks["hbm_gbs"])
+    tpeak_key = "bf16_tflops" if timed_s < 1.0 else "bf16_tflops_sustained"
+    tpk = float(peaks[tpeak_key])
+    t_mem = nbytes / (hbm * 1e9)
+    t_tc = nflops / (tpk * 1e12)
+    sec = dur_ms * 1e-3
+    gbs = nbytes / sec / 1e9
+    tfs = nflops / sec / 1e12
+    tensor = {"achieved": round(tfs, 2), "peak": tpk, "unit": "TFLOP/s", "frac": round(tfs / tpk, 4),
+              "peak_source": "%s %s" % (src, tpeak_key)}
+    if t_tc > t_mem:
+        roof = {"kernel": kind, "bound": "tensor", "achieved": round(tfs, 2), "peak": tpk, "unit": "TFLOP/s",
+                "frac": round(tfs / tpk, 4), "peak_source": "%s %s" % (src, tpeak_key)}
+    else:
+        roof = {"kernel": kind, "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(gbs / hbm, 4), "peak_source": "%s hbm_gbs" % src, "tensor": tensor}
+    roof.update({"traffic": None, "launch_us": round(dur_ms * 1e3, 3), "bytes_per_launch": int(nbytes),
+                 "flops_per_launch": int(nflops)})
+    return roof
 
 
 # ----------------------------------------------------------------- distributed plumbing
@@ -403,14 +452,10 @@ def run_moe(args, world, rank, local):
     hbm = float(peaks["hbm_gbs"])
     dom = max(kt.items(), key=lambda kv: kv[1][0])[0] if kt else None
     roof = None
-    if dom is not None:
-        dur_ms = kt[dom][0] / kt[dom][1]
-        per_launch = acc["kernel_bytes"].get({"router_logits": "router"}.get(dom, dom))
-        if per_launch is not None:
-            gbs = per_launch / (dur_ms * 1e-3) / 1e9
-            roof = {"kernel": dom, "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(gbs / hbm, 4), "traffic": None, "peak_source": src,
-                    "launch_us": round(dur_ms * 1e3, 3), "bytes_per_launch": int(per_launch)}
+    if dom is not None and dom in KIND_UNIT:
+        unit = KIND_UNIT[dom]
+        roof = kernel_roofline(dom, kt[dom][0] / kt[dom][1], acc["kernel_bytes"][unit], acc["kernel_flops"][unit],
+                               peaks, src, ms * 1e-3)
     step_bytes = acc["weight_bytes"] + acc["act_bytes"]
     step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
     value = tokens_per_step * K * world / (ms * 1e-3)
@@ -457,15 +502,17 @@ def accounting_for_steps(moeq, shape, layers, xs, xs_host, aids_host, K, W, copi
                              idx, w, sg, logits)
         a = step_accounting(shape, idx.cpu().numpy(), aids_host[i])
         if tot is None:
-            tot = {"kernel_bytes": dict(a["kernel_bytes"]), "weight_bytes": a["weight_bytes"],
-                   "act_bytes": a["act_bytes"], "flops": a["flops"]}
+            tot = {"kernel_bytes": dict(a["kernel_bytes"]), "kernel_flops": dict(a["kernel_flops"]),
+                   "weight_bytes": a["weight_bytes"], "act_bytes": a["act_bytes"], "flops": a["flops"]}
         else:
-            for k in tot["kernel_bytes"]:
-                tot["kernel_bytes"][k] += a["kernel_bytes"][k]
+            for kk in ("kernel_bytes", "kernel_flops"):
+                for k in tot[kk]:
+                    tot[kk][k] += a[kk][k]
             for k in ("weight_bytes", "act_bytes", "flops"):
                 tot[k] += a[k]
-    for k in tot["kernel_bytes"]:
-        tot["kernel_bytes"][k] /= nsteps
+    for kk in ("kernel_bytes", "kernel_flops"):
+        for k in tot[kk]:
+            tot[kk][k] /= nsteps
     for k in ("weight_bytes", "act_bytes", "flops"):
         tot[k] /= nsteps
     if stack:  # the whole stack per step; each layer's routing approximated by copy 0's

@@ -207,12 +207,26 @@ moe_status ws_check(void* ws, size_t ws_bytes, size_t need) {
     return MOE_OK;
 }
 
+// Router logits (and the shared-expert gate logit in gs): on the tensor cores from
+// kTcMinTokens tokens on, the gate row then by the CUDA-core kernel alone.
+moe_status router_enqueue(const uint16_t* x, const moe_qtensor& router, const moe_qtensor* sg, const float* lb,
+                          int T, int H, int E, float* logits, float* gs, int32_t* status, cudaStream_t s) {
+    if (T >= kTcMinTokens && tc_router_supported(router, H, E)) {
+        LAUNCH(kTcRouterKind, launch_tc_router(router, lb, x, T, H, E, logits, status, s));
+        if (sg) LAUNCH(kRouter, launch_router_logits(x, router, sg, nullptr, T, H, 0, logits, gs, s));
+        return MOE_OK;
+    }
+    LAUNCH(kRouter, launch_router_logits(x, router, sg, lb, T, H, E, logits, gs, s));
+    return MOE_OK;
+}
+
 // The launch sequence shared by moe_ffn_forward and moe_block_forward.
 moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, int T,
                        const uint16_t* residual, uint16_t* y, const Work& wk, cudaStream_t s) {
     const LayerArgs la = args_of(L);
     const moe_qtensor* sg = la.has_sgate ? &L->shared_gate : nullptr;
-    LAUNCH(kRouter, launch_router_logits(x, L->router, sg, L->logit_bias, T, la.H, la.E, wk.logits, wk.gs, s));
+    moe_status rst = router_enqueue(x, L->router, sg, L->logit_bias, T, la.H, la.E, wk.logits, wk.gs, wk.status, s);
+    if (rst != MOE_OK) return rst;
     LAUNCH(kTopk, launch_topk(wk.logits, wk.gs, la.has_sgate, T, la.E, la.K, wk.idx, wk.w, wk.sg, s));
     CHECK_CUDA(launch_index_build(wk, adapter_id, L->n_adapters, s));
     // Jobs of the shared expert stay in its group even without a shared expert:
@@ -358,8 +372,10 @@ moe_status moe_router_topk(const uint16_t* x, const moe_qtensor* router, const m
     if (has_sg) CHECK_ARG(qtensor_ok(*shared_gate, 1, 1, H, 8));
     cudaStream_t s = (cudaStream_t)stream;
     timing_begin(s);
-    LAUNCH(kRouter, launch_router_logits(x, *router, has_sg ? shared_gate : nullptr, logit_bias, T, H, E, logits,
-                                         shared_scale, s));
+    // no workspace here: a tensor-core wait that ran out has no status word to report to
+    moe_status rst = router_enqueue(x, *router, has_sg ? shared_gate : nullptr, logit_bias, T, H, E, logits,
+                                    shared_scale, nullptr, s);
+    if (rst != MOE_OK) return rst;
     LAUNCH(kTopk, launch_topk(logits, shared_scale, has_sg, T, E, K, topk_idx, topk_w, shared_scale, s));
     return MOE_OK;
 }

@@ -103,7 +103,7 @@ struct DecodeScratch {
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
     kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kTcLoraGUKind, kTcGUKind,
-    kTcLoraDownKind, kTcDownKind, kKindCount
+    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKindCount
 };
 void timing_begin(cudaStream_t s);
 void timing_mark(int kind, cudaStream_t s);
@@ -138,6 +138,10 @@ enum TcMode { kTcGU = 0, kTcDown = 1, kTcLoraGU = 2, kTcLoraDown = 3 };
 bool tc_supported(const LayerArgs& L);
 cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, int ld_act, const Work& wk,
                            const uint16_t* hb_out, int ldh, cudaStream_t s);
+// router logits [T][E] on the tensor cores (the shared-expert gate row is not included)
+bool tc_router_supported(const moe_qtensor& router, int H, int E);
+cudaError_t launch_tc_router(const moe_qtensor& router, const float* logit_bias, const uint16_t* x, int T, int H,
+                             int E, float* logits, int32_t* status, cudaStream_t s);
 
 bool decode_supported(const LayerArgs& L, int T, size_t* smem_out);
 cudaError_t launch_decode(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, uint16_t* y, int T,

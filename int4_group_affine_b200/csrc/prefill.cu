@@ -1,53 +1,85 @@
 // prefill.cu - expert-grouped GEMMs on the tcgen05 tensor cores (sm_100a) for
-// the many-token case: gate/up with fused SwiGLU, down with the routing weight,
-// and the two LoRA-A products.
+// the many-token case: the 8-bit router, gate/up with fused SwiGLU, down with
+// the routing weight, and the two LoRA-A products.
 //
-// Swap-AB: a tile is 128 weight rows (M, one TMEM lane each) by up to 64 jobs of
-// one expert group (N), over K in steps of 64 (= one quantisation group of 64).
-// Tiles live in shared memory K-major with the 128-byte swizzle.  Per K-step of
-// 64 every thread of the CTA
-//   - issues cp.async for later tiles: raw int4 words + scales/biases (or bf16
-//     LoRA-A rows) 6 tiles ahead, gathered activation rows 2 tiles ahead;
-//   - dequantises its share of this tile's int4 words into bf16 (one 32-bit word
-//     = 8 weights = one 16-byte chunk, w = fma(q, s, b) rounded once to bf16);
-// then one elected thread issues the tcgen05.mma instructions (4 per 64 of K and
-// matrix) into TMEM and commits them to an mbarrier.  After the last K-step of
-// a tile the CTA reads the accumulators back with tcgen05.ld and runs the
-// mode's epilogue.  Persistent grid: CTA c takes items c, c + grid, ...
+// Swap-AB: a tile is weight rows (M, one TMEM lane each) by up to 64 jobs of one
+// expert group (N), over K in steps of 64.  Operand tiles live in shared memory
+// K-major with the 128-byte swizzle, the layout the MMA descriptors name.
+//
+// Weights stream through the tensor memory accelerator: for each span of 128
+// bytes of packed words per row (K = 256 for int4, 128 for int8) one elected
+// thread loads a 128-row box per block with cp.async.bulk.tensor into a ring of
+// three slots, two spans ahead, so DRAM sees whole 128-byte lines.  Each thread
+// owns one weight row (half of one for int8): it prefetches that row's scales
+// and biases into registers one span ahead and dequantises its 64 weights of
+// each K-step into bf16 (w = fma(q, s, b), one rounding).  Activations (rows
+// gathered by token, or the h rows of the jobs) come in with cp.async four
+// K-steps ahead.  One thread issues the MMAs (4 x K=16 per block) and commits
+// them to an mbarrier.
+//
+// The unmerged LoRA-B term (alpha/r) B (A x) is one more MMA K-step per item
+// (per 64 columns of K' = adapters x r per matrix): operand A holds the LoRA-B
+// rows of every adapter side by side along K', operand B holds each job's scaled
+// LoRA-A products in its own adapter's columns (zero elsewhere), so the product
+// adds exactly each job's own adapter term into the accumulator.  Operand A is a
+// pseudo-span of the weight ring that the producer warp's lanes fill with
+// cp.async (zero where a column belongs to another matrix); operand B is staged
+// by the dequantisation warps from registers fetched a step ahead.
+//
+//   gate/up: block 0 = gate rows, block 1 = up rows, two accumulators; epilogue
+//            SiLU(g) * u -> h (bf16).
+//   down:    blocks = two consecutive 128-row blocks of down_proj; epilogue
+//            scales by the job's combine weight -> ypart.
+//   router:  int8 rows; block 0 = bf16(w), block 1 = bf16(w - bf16(w)), both
+//            into one accumulator, so the logits carry ~16 bits of each weight;
+//            epilogue adds the logit bias -> logits.
+//   LoRA-A:  bf16 A rows of every adapter (cp.async), 64 real rows per tile.
+//
+// Warp roles: 8 dequantisation warps (loads of activations and scales, dequant,
+// epilogue) and one producer warp whose lane 0 issues the TMA spans and the MMAs;
+// they hand stages over through mbarriers, so no CTA-wide barrier sits in the
+// K loop.  Persistent grid: CTA c takes items c, c + grid, ...
+#include <cudaTypedefs.h>
+
 #include "tc.cuh"
 
 namespace moeq {
 namespace {
 
-constexpr int kTcThreads = 256;
-constexpr int kBM = 128;   // rows per MMA tile
-constexpr int kNT = 64;    // jobs per tile (MMA N <= 64)
-constexpr int kRA = 8;     // raw A ring slots
-constexpr int kLA = 6;     // raw A lookahead (tiles)
-constexpr int kRB = 4;     // activation ring slots
-constexpr int kLB = 2;     // activation lookahead
-constexpr int kRawBytes = 10 * 1024;      // int4: 2 x 128 x 32 B words + 2 x 2 x 128 x 4 B scale/bias pairs
+constexpr int kDeqWarps = 8;                     // dequantisation warps
+constexpr int kTcThreads = (kDeqWarps + 1) * 32;  // + the producer warp (TMA and MMA issue)
+constexpr int kBM = 128;                  // rows per MMA block
+constexpr int kNT = 64;                   // jobs per tile (MMA N <= 64)
+constexpr int kLB = 4;                    // activation lookahead (K-steps)
+constexpr int kRB = kLB + 2;              // activation ring: a slot is free once the MMAs of its step are done
+constexpr int kRS = 3;                    // weight span ring (two spans in flight)
+constexpr int kSpanBytes = kBM * 128;     // one block of one span: 128 rows x 128 B
+constexpr int kRawSlot = 2 * kSpanBytes;  // two blocks
 constexpr int kBBytes = kNT * 128;        // 64 rows x 128 B
-constexpr int kAStage = 2 * kBM * 128;    // gate + up bf16 tiles (32 KB)
+constexpr int kAStage = 2 * kBM * 128;    // two bf16 blocks of 128 x 64 (32 KB)
 constexpr int kLoraRows = 64;             // real LoRA-A rows per M tile
+constexpr int kLoraSlot = kLoraRows * 128;
 constexpr int kMaxGroups = MOEQ_MAX_EXPERTS + 1;
-constexpr int kTBuf = kNT * 64;           // staged LoRA products (floats): 64 jobs x up to 2r = 64
+static_assert(kRB * kLoraSlot <= kRS * kRawSlot, "LoRA-A ring must fit in the weight ring");
 
-enum Mode { kGU = 0, kDown = 1, kLoraGU = 2, kLoraDown = 3 };
+enum Mode { kGU = 0, kDown = 1, kLoraGU = 2, kLoraDown = 3, kRouterMode = 4 };
 
 struct TcArgs {
+    CUtensorMap tm[4];    // weight words: gate/up {gate, up, s_gate, s_up}; down {down, s_down}; router {router}
     LayerArgs L;
     int mode;
-    const uint16_t* act;  // bf16 activation rows: x (GU, LoraGU: row = token) or h (Down, LoraDown: row = job)
+    const uint16_t* act;  // bf16 activation rows: x (by token) or h (by job)
     int ld_act;           // elements per activation row
     const int4* perm;     // [J] jobs {token, k, adapter, expert}
     const float* wperm;   // [J] combine weights
     const int32_t* goff;  // [E+2] job offsets of the expert groups (group E = shared expert)
-    uint16_t* h_out;      // GU: [J][ldh] bf16
+    uint16_t* h_out;      // gate/up: [J][ldh] bf16
     int ldh;
-    float* ypart;         // Down: [J][H]
-    float* t_out;         // LoraGU: [J][2r], LoraDown: [J][r]
-    const float* t_in;    // GU: [J][2r], Down: [J][r]
+    float* ypart;         // down: [J][H]
+    float* t_out;         // LoRA-A gate/up: [J][2r], LoRA-A down: [J][r]
+    const float* t_in;    // gate/up: [J][2r], down: [J][r]
+    float* logits;        // router: [T][E]
+    int T;                // router: tokens
     int32_t* status;
 };
 
@@ -56,10 +88,14 @@ struct Geo {  // one expert group's geometry in the current mode
     bool shared, skip;
 };
 
+__device__ __forceinline__ int rows_per_item(int mode) {
+    return mode == kDown ? 2 * kBM : (mode == kLoraGU || mode == kLoraDown) ? kLoraRows : kBM;
+}
+
 __device__ __forceinline__ Geo geo_of(const TcArgs& a, int g, int count) {
     const LayerArgs& L = a.L;
     Geo q;
-    q.shared = g == L.E;
+    q.shared = a.mode != kRouterMode && g == L.E;
     q.skip = count == 0 || (q.shared && !L.has_shared);
     q.mat = q.shared ? 0 : g;
     const int I = q.shared ? L.Is : L.I;
@@ -68,26 +104,30 @@ __device__ __forceinline__ Geo geo_of(const TcArgs& a, int g, int count) {
         case kGU: q.M = I; q.K = L.H; break;
         case kDown: q.M = L.H; q.K = I; break;
         case kLoraGU: q.M = L.n_adapters * 2 * r; q.K = L.H; break;
-        default: q.M = L.n_adapters * r; q.K = I; break;
+        case kLoraDown: q.M = L.n_adapters * r; q.K = I; break;
+        default: q.M = L.E; q.K = L.H; q.mat = 0; break;
     }
     if (q.M <= 0) q.skip = true;
-    const int rows_per_tile = (a.mode == kGU || a.mode == kDown) ? kBM : kLoraRows;
-    q.mtiles = q.skip ? 0 : (q.M + rows_per_tile - 1) / rows_per_tile;
+    const int rpi = rows_per_item(a.mode);
+    q.mtiles = q.skip ? 0 : (q.M + rpi - 1) / rpi;
     q.ntiles = q.skip ? 0 : (count + kNT - 1) / kNT;
     return q;
+}
+
+// LoRA-B K-steps appended to each gate/up or down item (K' = adapters x r per matrix)
+__device__ __forceinline__ int lora_steps(const TcArgs& a) {
+    const LayerArgs& L = a.L;
+    if ((a.mode != kGU && a.mode != kDown) || L.rank <= 0 || L.n_adapters <= 0) return 0;
+    const int kp = (a.mode == kGU ? 2 : 1) * L.n_adapters * L.rank;
+    return (kp + 63) / 64;
 }
 
 // Position in this CTA's stream of (item, k-step) tiles.
 struct Pos {
     int item;  // global item index (>= nitems: past the end)
-    int kt;    // k-step inside the item
-    int g, mt, nt, KT;
+    int kt;    // k-step inside the item: [0, KW) weight steps, [KW, KT) LoRA-B steps
+    int g, mt, nt, KW, KT;
 };
-
-__device__ __forceinline__ const moe_qtensor& wmat(const LayerArgs& L, int mode, bool shared, int which) {
-    if (mode == kGU) return which == 0 ? (shared ? L.s_gate : L.gate) : (shared ? L.s_up : L.up);
-    return shared ? L.s_down : L.down;
-}
 
 __device__ __forceinline__ const moe_lora_proj* tlora(const LayerArgs& L, int a, bool shared, int which) {
     if (a < 0 || a >= L.n_adapters) return nullptr;
@@ -117,6 +157,46 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bf
     return o;
 }
 
+// Two int8 words (8 codes) -> hi = bf16(w) and lo = bf16(w - hi) for w = s*q + b in fp32.
+__device__ __forceinline__ void dequant8_hilo(uint32_t w0, uint32_t w1, float s, float b, uint4& hi, uint4& lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint32_t w = p < 2 ? w0 : w1;
+        const int sh = 16 * (p & 1);
+        const float v0 = fmaf(s, u2f_small((w >> sh) & 0xFFu), b);
+        const float v1 = fmaf(s, u2f_small((w >> (sh + 8)) & 0xFFu), b);
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
+        const float2 hf = __bfloat1622float2(hv);
+        const __nv_bfloat162 lv = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+        h[p] = *reinterpret_cast<const uint32_t*>(&hv);
+        l[p] = *reinterpret_cast<const uint32_t*>(&lv);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ uint32_t pick4(const uint32_t (&v)[4], int i) {
+    return i == 0 ? v[0] : i == 1 ? v[1] : i == 2 ? v[2] : v[3];
+}
+
+__device__ __forceinline__ __nv_bfloat162 bf16x2_of(uint32_t half_word) {
+    return __bfloat162bfloat162(__ushort_as_bfloat16((unsigned short)(half_word & 0xFFFFu)));
+}
+
+// This thread's activation chunk (and LoRA-A chunk) of one item.
+struct BCtx {
+    const uint16_t* src[2];
+    const uint16_t* la[2];  // LoRA-A modes: bf16 A chunks (NULL: zero fill)
+    bool live[2];
+};
+
+// Registers of one LoRA-B step, fetched a step ahead.
+struct LoraRegs {
+    float4 t[2][2];  // LoRA-A products of this thread's two (job, chunk) pairs, unscaled
+    bool t_live[2];
+};
+
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ __align__(1024) unsigned char tsm_raw[];
     // 128-byte-swizzled tiles need 1024-byte aligned bases: align by hand (the
@@ -125,45 +205,59 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     const LayerArgs& L = a.L;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int mode = a.mode;
+    const bool lora_mode = mode == kLoraGU || mode == kLoraDown;
+    const bool int8_mode = mode == kRouterMode;
     const bool int4_mode = mode == kGU || mode == kDown;
-    const int nmat = mode == kGU ? 2 : 1;
+    const int SP = int8_mode ? 2 : 4;  // K-steps per weight span (128 B of words per row)
     const int r = L.rank;
+    const int NL = lora_steps(a);
 
-    // shared memory: [A stages 2 x 32 KB][activation ring 4 x 8 KB][raw ring 8 x 10 KB]
+    // shared memory: [A stages 2 x 32 KB][activation ring kRB x 8 KB][weight ring kRS x 32 KB]
     unsigned char* sA = tsm;
     unsigned char* sB = sA + 2 * kAStage;
     unsigned char* sR = sB + kRB * kBBytes;
-    __shared__ uint64_t bar_tile[4];
-    __shared__ uint64_t bar_acc;
+    __shared__ uint64_t bar_full[2];      // A stage (and its activation slot) written: one arrival per dequant warp
+    __shared__ uint64_t bar_tile[4];      // MMAs of a step done (tcgen05.commit)
+    __shared__ uint64_t bar_acc;          // MMAs of an item done
+    __shared__ uint64_t bar_raw[kRS];     // span landed: 32 producer-lane arrivals (+ TMA transaction count)
+    __shared__ uint64_t bar_rawfree[kRS]; // span consumed: one arrival per dequant warp + the producer's commit
     __shared__ uint32_t s_tmem;
     __shared__ int s_items[kMaxGroups + 1];
     __shared__ int s_goff[kMaxGroups + 1];
-    __shared__ int4 s_job[3][kNT];      // job entries of the three most recent loader items
-    __shared__ float s_wt[3][kNT];
-    __shared__ float s_t[kTBuf];        // staged LoRA products for the epilogue
-    __shared__ int s_ok;
+    __shared__ volatile int s_ok;
 
     // ---------------------------------------------------------- set-up
-    const int ngroups = L.E + 1;
-    for (int g = tid; g <= ngroups; g += kTcThreads) s_goff[g] = a.goff[g];
-    if (warp == 0) {
+    const int ngroups = int8_mode ? 1 : L.E + 1;
+    if (int8_mode) {
+        if (tid == 0) {
+            s_goff[0] = 0;
+            s_goff[1] = a.T;
+        }
+    } else {
+        for (int g = tid; g <= ngroups; g += kTcThreads) s_goff[g] = a.goff[g];
+    }
+    if (warp == kDeqWarps) {
         tc::tmem_alloc(&s_tmem, 512);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
+        for (int i = 0; i < 2; ++i) tc::mbar_init(&bar_full[i], kDeqWarps);
         for (int i = 0; i < 4; ++i) tc::mbar_init(&bar_tile[i], 1);
+        for (int i = 0; i < kRS; ++i) {
+            tc::mbar_init(&bar_raw[i], 32);
+            tc::mbar_init(&bar_rawfree[i], kDeqWarps + 1);
+        }
         tc::mbar_init(&bar_acc, 1);
         tc::mbar_init_fence();
         s_ok = 1;
     }
-    // zero both A stages once (LoRA modes never write rows 64..127)
+    // zero both A stages once (LoRA-A modes never write rows 64..127)
     for (int i = tid; i < 2 * kAStage / 16; i += kTcThreads) reinterpret_cast<uint4*>(sA)[i] = make_uint4(0, 0, 0, 0);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = s_tmem;
-    // item prefix over groups (every CTA computes the same table)
-    if (tid == 0) {
+    if (tid == 0) {  // item prefix over groups (every CTA computes the same table)
         int acc = 0;
         for (int g = 0; g < ngroups; ++g) {
             s_items[g] = acc;
@@ -181,7 +275,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         p.kt = 0;
         if (item >= nitems) {
             p.g = p.mt = p.nt = 0;
-            p.KT = 1;
+            p.KW = p.KT = 1;
             return;
         }
         int lo = 0, hi = ngroups - 1;  // last group with s_items[g] <= item
@@ -195,320 +289,547 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         p.g = lo;
         p.mt = rem / q.ntiles;
         p.nt = rem % q.ntiles;
-        p.KT = q.K / 64;
+        p.KW = q.K / 64;
+        p.KT = p.KW + NL;
     };
-    auto advance = [&](Pos& p) {
-        if (p.item >= nitems) return;
-        if (++p.kt == p.KT) decode(p.item + NB, p);
-    };
+    auto tile_jobs = [&](const Pos& p) { return min(kNT, s_goff[p.g + 1] - s_goff[p.g] - p.nt * kNT); };
 
-    // ---------------------------------------------------------- loaders
-    // raw A of tile position p into raw slot `slot`
-    auto load_raw = [&](const Pos& p, int slot) {
-        if (p.item >= nitems) return;
-        unsigned char* raw = sR + slot * kRawBytes;
-        const Geo q = geo_of(a, p.g, s_goff[p.g + 1] - s_goff[p.g]);
-        if (int4_mode) {
-            const int ng = q.K / wmat(L, mode, q.shared, 0).group;
-            const int group = wmat(L, mode, q.shared, 0).group;
-            const int gidx = (p.kt * 64) / group;
-            const int pair = gidx & ~1;
-            for (int u = tid; u < nmat * kBM * 4; u += kTcThreads) {  // 2 x 16 B of words, s pair, b pair
-                const int mat = u / (kBM * 4), row = (u / 4) % kBM, part = u % 4;
-                const moe_qtensor& W = wmat(L, mode, q.shared, mat);
-                const int R = p.mt * kBM + row;
-                const bool live = R < q.M;
-                const int64_t grow = (int64_t)q.mat * q.M + (live ? R : 0);
-                if (part < 2) {
-                    const uint32_t* src = W.packed + grow * (q.K / 8) + p.kt * 8 + part * 4;
-                    tc::cp16(tc::smem_u32(raw + (mat * kBM + row) * 32 + part * 16), src, live ? 16u : 0u);
-                } else {
-                    const uint16_t* base = part == 2 ? W.scales : W.biases;
-                    unsigned char* dst = raw + 8192 + ((part - 2) * 2 * kBM + mat * kBM + row) * 4;
-                    if (live) tc::cp4(tc::smem_u32(dst), base + grow * ng + pair);
-                    else *reinterpret_cast<uint32_t*>(dst) = 0u;
-                }
-            }
-        } else {
-            // LoRA-A rows (bf16): tile rows 0..63 of M tile mt
-            const int rpa = mode == kLoraGU ? 2 * r : r;
-            for (int u = tid; u < kLoraRows * 8; u += kTcThreads) {
-                const int row = u / 8, c = u % 8;
-                const int R = p.mt * kLoraRows + row;
-                const int ad = R / rpa, d = R % rpa;
-                const uint16_t* src = nullptr;
-                if (R < q.M) {
-                    const int which = mode == kLoraGU ? (d < r ? 0 : 1) : 2;
-                    const moe_lora_proj* lp = tlora(L, ad, q.shared, which);
-                    if (lp) src = lp->A + ((int64_t)q.mat * r + (mode == kLoraGU ? d % r : d)) * q.K + p.kt * 64 + c * 8;
-                }
-                tc::cp16(tc::smem_u32(raw + row * 128 + c * 16), src ? src : a.act, src ? 16u : 0u);
-            }
-        }
-    };
-    // activation rows of tile position p into activation slot `slot`; `tab` is the
-    // job table of p's item (filled when the loader enters the item)
-    auto load_b = [&](const Pos& p, int slot, int tab) {
-        if (p.item >= nitems) return;
-        unsigned char* dst = sB + slot * kBBytes;
-        const int base = s_goff[p.g] + p.nt * kNT, end = s_goff[p.g + 1];
-        const bool by_token = mode == kGU || mode == kLoraGU;
-        for (int u = tid; u < kNT * 8; u += kTcThreads) {
-            const int n = u / 8, c = u % 8;
-            const int job = base + n;
-            const bool live = job < end;
-            const int64_t rowi = live ? (by_token ? s_job[tab][n].x : job) : 0;
-            const uint16_t* src = a.act + rowi * a.ld_act + p.kt * 64 + c * 8;
-            tc::cp16(tc::smem_u32(dst + tc::sw128_off(n, c)), src, live ? 16u : 0u);
-        }
-    };
-    auto fill_table = [&](const Pos& p, int tab) {
-        if (p.item >= nitems) return;
-        const int base = s_goff[p.g] + p.nt * kNT, end = s_goff[p.g + 1];
-        if (tid < kNT) {
-            const int job = base + tid;
-            s_job[tab][tid] = job < end ? a.perm[job] : make_int4(0, 0, -1, 0);
-            s_wt[tab][tid] = (job < end && a.wperm) ? a.wperm[job] : 0.0f;
-        }
-    };
-
-    // ---------------------------------------------------------- stream
-    Pos pc, pa, pb;  // consumer, raw-A loader, activation loader
-    decode(blockIdx.x, pc);
-    pa = pc;
-    pb = pc;
-    int tab_b = 0;  // job-table slot of the activation loader's item (items cycle through 3 slots)
-    int seq_b = 0;  // items entered by the activation loader
-    int seq_c = 0;  // items entered by the consumer
-    // prologue: raw tiles 0..kLA-1 and activation tiles 0..kLB-1
-    fill_table(pb, 0);
-    __syncthreads();
-    for (int i = 0; i < kLA; ++i) {
-        load_raw(pa, i % kRA);
-        if (i < kLB) {
-            load_b(pb, i % kRB, tab_b);
-            const int prev = pb.item;
-            advance(pb);
-            if (pb.item != prev) {
-                ++seq_b;
-                tab_b = seq_b % 3;
-                __syncthreads();
-                fill_table(pb, tab_b);
-                __syncthreads();
-            }
-        }
-        tc::cp_commit();
-        advance(pa);
-    }
-
-    uint32_t t = 0;        // tiles consumed by this CTA
-    uint32_t n_items = 0;  // items finished by this CTA
-    while (pc.item < nitems) {
-        // the MMAs of tile t-2 must be done before stage t%2 and activation slot (t+2)%4 are rewritten
-        if (t >= 2) {
-            const uint32_t tp = t - 2;
-            if (!tc::mbar_wait(&bar_tile[tp % 4], (tp / 4) & 1u, a.status)) s_ok = 0;
-        }
-        // issue loads for raw tile t+kLA and activation tile t+kLB
-        load_raw(pa, (t + kLA) % kRA);
-        advance(pa);
-        load_b(pb, (t + kLB) % kRB, tab_b);
-        tc::cp_commit();
-        {
-            const int prev = pb.item;
-            advance(pb);
-            if (pb.item != prev) {
-                ++seq_b;
-                tab_b = seq_b % 3;
-                fill_table(pb, tab_b);
-            }
-        }
-        tc::cp_wait<2>();  // this tile's group (issued kLB steps ago) has landed
-        __syncthreads();
-
-        const Geo q = geo_of(a, pc.g, s_goff[pc.g + 1] - s_goff[pc.g]);
-        const int n_here = min(kNT, s_goff[pc.g + 1] - s_goff[pc.g] - pc.nt * kNT);
-        const int Nmma = (n_here + 15) / 16 * 16;
-        unsigned char* stA = sA + (t % 2) * kAStage;
-        const unsigned char* raw = sR + (t % kRA) * kRawBytes;
-        if (int4_mode) {
-            const int group = wmat(L, mode, q.shared, 0).group;
-            const int gidx0 = (pc.kt * 64) / group, pair = gidx0 & ~1;
-            for (int u = tid; u < nmat * kBM * 8; u += kTcThreads) {
-                const int mat = u / (kBM * 8), row = (u / 8) % kBM, c = u % 8;
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(raw + (mat * kBM + row) * 32 + c * 4);
-                const int gsel = (pc.kt * 64 + c * 8) / group - pair;  // 0 or 1 inside the loaded pair
-                const __nv_bfloat16* sp =
-                    reinterpret_cast<const __nv_bfloat16*>(raw + 8192 + (0 * 2 * kBM + mat * kBM + row) * 4);
-                const __nv_bfloat16* bp =
-                    reinterpret_cast<const __nv_bfloat16*>(raw + 8192 + (1 * 2 * kBM + mat * kBM + row) * 4);
-                const __nv_bfloat162 s2 = __bfloat162bfloat162(sp[gsel]);
-                const __nv_bfloat162 b2 = __bfloat162bfloat162(bp[gsel]);
-                *reinterpret_cast<uint4*>(stA + mat * (kBM * 128) + tc::sw128_off(row, c)) = dequant8(w, s2, b2);
-            }
-        } else {
-            for (int u = tid; u < kLoraRows * 8; u += kTcThreads) {
-                const int row = u / 8, c = u % 8;
-                *reinterpret_cast<uint4*>(stA + tc::sw128_off(row, c)) =
-                    *reinterpret_cast<const uint4*>(raw + row * 128 + c * 16);
-            }
-        }
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-        if (!s_ok) break;
-        tc::tc_fence_after();
-        if (tid == 0) {
-            const uint32_t idesc = tc::idesc_bf16(kBM, Nmma);
-            const uint32_t bbase = tc::smem_u32(sB + (t % kRB) * kBBytes);
-            for (int mat = 0; mat < nmat; ++mat) {
-                const uint32_t abase = tc::smem_u32(stA + mat * (kBM * 128));
-                const uint64_t ad = tc::sdesc_k_sw128(abase), bd = tc::sdesc_k_sw128(bbase);
-                for (int k = 0; k < 4; ++k)  // 4 x K=16 inside the 128-byte swizzle atom: +32 B each
-                    tc::mma_bf16(tmem + mat * 256, ad + 2 * k, bd + 2 * k, idesc, (pc.kt > 0 || k > 0) ? 1u : 0u);
-            }
-            tc::mma_commit(&bar_tile[t % 4]);
-            if (pc.kt == pc.KT - 1) tc::mma_commit(&bar_acc);
-        }
-        ++t;
-
-        if (pc.kt == pc.KT - 1) {
-            // ---------------------------------------------------- epilogue
-            if (!tc::mbar_wait(&bar_acc, n_items & 1u, a.status)) s_ok = 0;
-            ++n_items;
-            tc::tc_fence_after();
-            const int tab_c = seq_c % 3;
-            const int base = s_goff[pc.g] + pc.nt * kNT;
-            // LoRA products of this tile's jobs into shared memory
-            const int tw = mode == kGU ? 2 * r : (mode == kDown ? r : 0);
-            if (tw > 0)
-                for (int u = tid; u < kNT * tw; u += kTcThreads) {
-                    const int n = u / tw, k = u % tw;
-                    s_t[u] = n < n_here ? a.t_in[(int64_t)(base + n) * tw + k] : 0.0f;
-                }
-            __syncthreads();
-            const int quarter = warp % 4, half = warp / 4;
-            const int row = quarter * 32 + lane;  // TMEM lane of this thread
-            for (int ch = half; ch * 16 < Nmma; ch += 2) {
-                uint32_t d0[16], d1[16];
-                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ch * 16;
-                tc::tmem_ld16(taddr, d0);
-                if (mode == kGU) tc::tmem_ld16(taddr + 256, d1);
-                tc::tmem_wait_ld();
+    const int nar = L.n_adapters * r;
+    // spans of an item in the weight ring: its weight spans, then one per LoRA-B step
+    auto wspans = [&](const Pos& p) { return (p.KW + SP - 1) / SP; };
+    if (warp == kDeqWarps) {
+        // ====================================================== producer warp: TMA, LoRA-B rows, MMA issue
+        Pos pc;
+        decode(blockIdx.x, pc);
+        Pos pt = pc;  // item of the next span to load
+        int pt_span = 0;
+        uint32_t issued = 0;  // spans issued
+        bool ok = true;
+        // LoRA-B rows of step s into slot: lane -> chunk lane % 8 of rows lane / 8 + 4 i
+        auto lora_span = [&](const Pos& p, int s, int slot) {
+            const Geo q = geo_of(a, p.g, s_goff[p.g + 1] - s_goff[p.g]);
+            const uint32_t dst0 = tc::smem_u32(sR + slot * kRawSlot);
+            const int c = lane % 8, cp = 64 * s + 8 * c;
+            for (int blk = 0; blk < 2; ++blk) {
+                int part = 0, cc = cp;
                 if (mode == kGU) {
-                    const int i = pc.mt * kBM + row;
-                    if (i < q.M) {
-                        const moe_lora_proj* lg = nullptr;
-                        const moe_lora_proj* lu = nullptr;
-                        int cur = -2;
-                        float bgv[MOEQ_MAX_RANK / 2], buv[MOEQ_MAX_RANK / 2];
-                        for (int c = 0; c < 16; ++c) {
-                            const int n = ch * 16 + c;
-                            if (n >= n_here) break;
-                            const int4 job = s_job[tab_c][n];
-                            float g = __uint_as_float(d0[c]), u = __uint_as_float(d1[c]);
-                            if (job.z != cur) {  // jobs are sorted by adapter: reload B rows per run
-                                cur = job.z;
-                                lg = tlora(L, cur, q.shared, 0);
-                                lu = tlora(L, cur, q.shared, 1);
-                                for (int k = 0; k < r && k < MOEQ_MAX_RANK / 2; ++k) {
-                                    bgv[k] = lg ? bf16f(lg->B[((int64_t)q.mat * q.M + i) * r + k]) : 0.0f;
-                                    buv[k] = lu ? bf16f(lu->B[((int64_t)q.mat * q.M + i) * r + k]) : 0.0f;
-                                }
-                            }
-                            if (lg || lu) {
-                                float dg = 0.0f, du = 0.0f;
-                                for (int k = 0; k < r && k < MOEQ_MAX_RANK / 2; ++k) {
-                                    dg = fmaf(bgv[k], s_t[n * tw + k], dg);
-                                    du = fmaf(buv[k], s_t[n * tw + r + k], du);
-                                }
-                                g += L.scale * dg;
-                                u += L.scale * du;
-                            }
-                            a.h_out[(int64_t)(base + n) * a.ldh + i] = f2bf16(silu(g) * u);
-                        }
-                    }
-                } else if (mode == kDown) {
-                    const int o = pc.mt * kBM + row;
-                    if (o < q.M) {
-                        const moe_lora_proj* ld = nullptr;
-                        int cur = -2;
-                        float bdv[MOEQ_MAX_RANK / 2];
-                        for (int c = 0; c < 16; ++c) {
-                            const int n = ch * 16 + c;
-                            if (n >= n_here) break;
-                            const int4 job = s_job[tab_c][n];
-                            float v = __uint_as_float(d0[c]);
-                            if (job.z != cur) {
-                                cur = job.z;
-                                ld = tlora(L, cur, q.shared, 2);
-                                for (int k = 0; k < r && k < MOEQ_MAX_RANK / 2; ++k)
-                                    bdv[k] = ld ? bf16f(ld->B[((int64_t)q.mat * L.H + o) * r + k]) : 0.0f;
-                            }
-                            if (ld) {
-                                float dd = 0.0f;
-                                for (int k = 0; k < r && k < MOEQ_MAX_RANK / 2; ++k) dd = fmaf(bdv[k], s_t[n * tw + k], dd);
-                                v += L.scale * dd;
-                            }
-                            a.ypart[(int64_t)(base + n) * L.H + o] = s_wt[tab_c][n] * v;
-                        }
+                    part = cp < nar ? 0 : 1;
+                    cc = cp - part * nar;
+                }
+                const bool mine = mode == kGU ? part == blk : true;  // gate rows take gate columns only
+                const moe_lora_proj* lp = (mine && cc < nar) ? tlora(L, cc / r, q.shared, mode == kGU ? part : 2) : nullptr;
+                const int row0 = mode == kGU ? p.mt * kBM : p.mt * 2 * kBM + blk * kBM;
+                const uint16_t* src = lp ? lp->B + ((int64_t)q.mat * q.M + row0) * r + cc % r : a.act;
+                for (int i = 0; i < kBM / 4; ++i) {
+                    const int row = lane / 8 + 4 * i;
+                    const bool live = lp && row0 + row < q.M;
+                    tc::cp16(dst0 + blk * kSpanBytes + tc::sw128_off(row, c), live ? src + (int64_t)row * r : a.act,
+                             live ? 16u : 0u);
+                }
+            }
+            tc::cp_commit();  // (so that the final drain's wait covers these copies)
+            tc::cp_arrive_noinc(&bar_raw[slot]);
+        };
+        // the next span into slot issued % kRS, once the span kRS before it is consumed
+        auto span_next = [&]() {
+            if (pt.item >= nitems || !ok) return;
+            const uint32_t seq = issued;
+            const int slot = seq % kRS;
+            if (seq >= (uint32_t)kRS && !tc::mbar_wait_ok(&bar_rawfree[slot], ((seq / kRS) - 1) & 1u, a.status, &s_ok)) {
+                ok = false;
+                return;
+            }
+            const int nw = wspans(pt);
+            if (pt_span < nw) {
+                uint64_t* bar = &bar_raw[slot];
+                if (lane == 0) {
+                    const Geo q = geo_of(a, pt.g, s_goff[pt.g + 1] - s_goff[pt.g]);
+                    const uint32_t dst = tc::smem_u32(sR + slot * kRawSlot);
+                    const int x = pt_span * 32;  // 32 words = 128 B per row
+                    if (mode == kGU) {
+                        const int y = q.mat * q.M + pt.mt * kBM;
+                        tc::mbar_arrive_expect_tx(bar, 2 * kSpanBytes);
+                        tc::tma_load_2d(dst, &a.tm[q.shared ? 2 : 0], x, y, bar);
+                        tc::tma_load_2d(dst + kSpanBytes, &a.tm[q.shared ? 3 : 1], x, y, bar);
+                    } else if (mode == kDown) {
+                        const int y = q.mat * q.M + pt.mt * 2 * kBM;
+                        tc::mbar_arrive_expect_tx(bar, 2 * kSpanBytes);
+                        tc::tma_load_2d(dst, &a.tm[q.shared ? 1 : 0], x, y, bar);
+                        tc::tma_load_2d(dst + kSpanBytes, &a.tm[q.shared ? 1 : 0], x, y + kBM, bar);
+                    } else {
+                        tc::mbar_arrive_expect_tx(bar, kSpanBytes);
+                        tc::tma_load_2d(dst, &a.tm[0], x, pt.mt * kBM, bar);
                     }
                 } else {
+                    tc::mbar_arrive(bar);
+                }
+            } else {
+                lora_span(pt, pt_span - nw, slot);
+            }
+            ++issued;
+            if (++pt_span >= nw + NL) {
+                decode(pt.item + NB, pt);
+                pt_span = 0;
+            }
+        };
+        if (!lora_mode) {
+            span_next();
+            span_next();
+        }
+        uint32_t t = 0, cs = 0;  // steps and spans consumed
+        while (pc.item < nitems && ok) {
+            const bool wstep = pc.kt < pc.KW;
+            const bool opens = !lora_mode && (!wstep || pc.kt % SP == 0);
+            if (opens) span_next();  // keep two spans ahead
+            if (!ok || !tc::mbar_wait_ok(&bar_full[t % 2], (t / 2) & 1u, a.status, &s_ok)) {
+                ok = false;
+                break;
+            }
+            // LoRA-B step: its operand A (this warp's own copies) must have landed
+            if (!wstep && !tc::mbar_wait_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok)) {
+                ok = false;
+                break;
+            }
+            tc::tc_fence_after();
+            if (lane == 0) {
+                const int Nmma = (tile_jobs(pc) + 15) / 16 * 16;
+                const uint32_t idesc = tc::idesc_bf16(kBM, Nmma);
+                const uint32_t bbase = tc::smem_u32(sB + (t % kRB) * kBBytes);
+                const uint32_t sbase = wstep ? tc::smem_u32(sA + (t % 2) * kAStage) : tc::smem_u32(sR + (cs % kRS) * kRawSlot);
+                const int nblk = lora_mode ? 1 : 2;
+                for (int blk = 0; blk < nblk; ++blk) {
+                    const uint32_t boff = wstep ? blk * (kBM * 128) : blk * kSpanBytes;
+                    const uint64_t ad = tc::sdesc_k_sw128(sbase + boff), bd = tc::sdesc_k_sw128(bbase);
+                    // router: hi and lo parts into one accumulator; otherwise one accumulator per block
+                    const uint32_t d = tmem + (int8_mode ? 0u : (uint32_t)blk * 256u);
+                    for (int k = 0; k < 4; ++k) {  // 4 x K=16 inside the 128-byte swizzle atom: +32 B each
+                        const bool first = pc.kt == 0 && k == 0 && (!int8_mode || blk == 0);
+                        tc::mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, first ? 0u : 1u);
+                    }
+                }
+                tc::mma_commit(&bar_tile[t % 4]);
+                // the span's slot is free once these MMAs are done (they read it directly for LoRA-B)
+                if (!lora_mode && (!wstep || pc.kt % SP == SP - 1 || pc.kt == pc.KW - 1))
+                    tc::mma_commit(&bar_rawfree[cs % kRS]);
+                if (pc.kt == pc.KT - 1) tc::mma_commit(&bar_acc);
+            }
+            __syncwarp();
+            ++t;
+            if (++pc.kt == pc.KT) decode(pc.item + NB, pc);
+            if (!lora_mode && pc.item < nitems && (pc.kt >= pc.KW || pc.kt % SP == 0)) ++cs;
+        }
+        // drain (bounded): this warp's copies, the last MMAs, the latest span issued into each slot
+        tc::cp_wait<0>();
+        if (lane == 0) {
+            if (t > 0) tc::mbar_wait(&bar_tile[(t - 1) % 4], ((t - 1) / 4) & 1u, a.status);
+            for (uint32_t sq = issued > (uint32_t)kRS ? issued - kRS : 0; sq < issued; ++sq)
+                tc::mbar_wait(&bar_raw[sq % kRS], (sq / kRS) & 1u, a.status);
+            if (!ok) s_ok = 0;
+        }
+        __syncwarp();
+    } else {
+        // ====================================================== dequantisation warps
+        // ---- weight rows.  int4: thread -> (block, row), the K-step's 8 words of the row;
+        //      int8: thread -> (row, half of the K-step's 16 words)
+        const int wrow = tid % kBM;
+        const int wblk = int8_mode ? 0 : tid / kBM;
+        const int wh = tid / kBM;  // int8: half
+        const int group = int8_mode ? L.router.group : L.gate.group;
+        const int gshift = group == 64 ? 6 : 5;
+        // scale/bias words (pairs of bf16) of one span of this thread's row
+        const int span_groups = (SP * 64) >> gshift;  // 2, 4 or 8
+        const int span_words = span_groups / 2;       // 1, 2 or 4
+        auto fetch_sb = [&](const Pos& p, int span, uint32_t (&sv)[4], uint32_t (&bv)[4]) {
+            const Geo q = geo_of(a, p.g, s_goff[p.g + 1] - s_goff[p.g]);
+            int row;
+            const moe_qtensor* W;
+            if (mode == kGU) {
+                row = p.mt * kBM + wrow;
+                W = wblk == 0 ? (q.shared ? &L.s_gate : &L.gate) : (q.shared ? &L.s_up : &L.up);
+            } else if (mode == kDown) {
+                row = p.mt * 2 * kBM + wblk * kBM + wrow;
+                W = q.shared ? &L.s_down : &L.down;
+            } else {
+                row = p.mt * kBM + wrow;
+                W = &L.router;
+            }
+            const bool ok = row < q.M;
+            const int ng = q.K >> gshift;
+            const int64_t off = ((int64_t)q.mat * q.M + (ok ? row : 0)) * ng + span * span_groups;
+            const int g0 = span * span_groups;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const bool in = ok && j < span_words && g0 + 2 * j < ng;
+                sv[j] = in ? __ldg(reinterpret_cast<const unsigned int*>(W->scales + off + 2 * j)) : 0u;
+                bv[j] = in ? __ldg(reinterpret_cast<const unsigned int*>(W->biases + off + 2 * j)) : 0u;
+            }
+        };
+
+        // ---- activation rows (and LoRA-A rows): rows brow, brow + 32, 16-byte chunk bch
+        const int brow = tid / 8, bch = tid % 8;
+        auto make_b = [&](const Pos& p, BCtx& c) {
+            const bool by_token = mode == kGU || mode == kLoraGU;
+            const bool live_item = p.item < nitems;
+            const int base = live_item ? s_goff[p.g] + p.nt * kNT : 0;
+            const int end = live_item ? s_goff[p.g + 1] : 0;
+            const Geo q = geo_of(a, p.g, end - base + p.nt * kNT);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int job = base + brow + 32 * j;
+                c.live[j] = job < end;
+                const int64_t rowi = c.live[j] ? (by_token ? a.perm[job].x : job) : 0;
+                c.src[j] = a.act + rowi * a.ld_act + bch * 8;
+                c.la[j] = nullptr;
+                if (lora_mode && live_item) {
                     const int rpa = mode == kLoraGU ? 2 * r : r;
-                    const int R = pc.mt * kLoraRows + row;
-                    if (row < kLoraRows && R < q.M) {
+                    const int R = p.mt * kLoraRows + brow + 32 * j;
+                    if (R < q.M) {
                         const int ad = R / rpa, d = R % rpa;
-                        for (int c = 0; c < 16; ++c) {
-                            const int n = ch * 16 + c;
-                            if (n >= n_here) break;
-                            if (s_job[tab_c][n].z == ad) a.t_out[(int64_t)(base + n) * rpa + d] = __uint_as_float(d0[c]);
-                        }
+                        const int which = mode == kLoraGU ? (d < r ? 0 : 1) : 2;
+                        const moe_lora_proj* lp = tlora(L, ad, q.shared, which);
+                        if (lp) c.la[j] = lp->A + ((int64_t)q.mat * r + (mode == kLoraGU ? d % r : d)) * q.K + bch * 8;
                     }
                 }
             }
+        };
+        auto issue_b = [&](const BCtx& c, int kt, int slot) {
+            const uint32_t base = tc::smem_u32(sB + slot * kBBytes);
+            const uint32_t rb = tc::smem_u32(sR + slot * kLoraSlot);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int row = brow + 32 * j;
+                tc::cp16(base + tc::sw128_off(row, bch), c.src[j] + (c.live[j] ? kt * 64 : 0), c.live[j] ? 16u : 0u);
+                if (lora_mode)  // this thread's own LoRA-A chunks; it copies them into the A stage itself
+                    tc::cp16(rb + (uint32_t)(row * 128 + bch * 16), c.la[j] ? c.la[j] + kt * 64 : a.act,
+                             c.la[j] ? 16u : 0u);
+            }
+        };
+
+        // ---- LoRA-B operand B: thread holds (job row, chunk) = (brow, bch) and (brow + 32, bch).
+        // K' column c' of step s is 64 s + 8 chunk + e; gate/up: [gate adapters | up adapters].
+        auto fetch_lora = [&](const Pos& p, int s, LoraRegs& R) {
+            const Geo q = geo_of(a, p.g, s_goff[p.g + 1] - s_goff[p.g]);
+            const int base = s_goff[p.g] + p.nt * kNT, end = s_goff[p.g + 1];
+            const int cp = 64 * s + 8 * bch;
+            const int part = (mode == kGU && cp >= nar) ? 1 : 0;
+            const int cc = cp - part * nar;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int job = base + brow + 32 * j;
+                R.t_live[j] = false;
+                if (job < end && cc < nar) {
+                    const int ad = a.perm[job].z;
+                    if (ad == cc / r && tlora(L, ad, q.shared, mode == kGU ? part : 2)) {
+                        const int tw = mode == kGU ? 2 * r : r;
+                        const float4* tp =
+                            reinterpret_cast<const float4*>(a.t_in + (int64_t)job * tw + part * r + cc % r);
+                        R.t[j][0] = tp[0];
+                        R.t[j][1] = tp[1];
+                        R.t_live[j] = true;
+                    }
+                }
+            }
+        };
+        auto stage_lora = [&](const LoraRegs& R, unsigned char* sBslot) {
+            const float sc = L.scale;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                uint4 o = make_uint4(0, 0, 0, 0);
+                if (R.t_live[j]) {
+                    const __nv_bfloat162 p0 = __floats2bfloat162_rn(sc * R.t[j][0].x, sc * R.t[j][0].y);
+                    const __nv_bfloat162 p1 = __floats2bfloat162_rn(sc * R.t[j][0].z, sc * R.t[j][0].w);
+                    const __nv_bfloat162 p2 = __floats2bfloat162_rn(sc * R.t[j][1].x, sc * R.t[j][1].y);
+                    const __nv_bfloat162 p3 = __floats2bfloat162_rn(sc * R.t[j][1].z, sc * R.t[j][1].w);
+                    o = make_uint4(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1),
+                                   *reinterpret_cast<const uint32_t*>(&p2), *reinterpret_cast<const uint32_t*>(&p3));
+                }
+                *reinterpret_cast<uint4*>(sBslot + tc::sw128_off(brow + 32 * j, bch)) = o;
+            }
+        };
+
+        // ------------------------------------------------------ stream
+        Pos pc, pb;  // consumer, activation loader (kLB steps ahead)
+        decode(blockIdx.x, pc);
+        pb = pc;
+        BCtx cb;
+        make_b(pb, cb);
+        auto issue_step = [&](uint32_t seq) {  // loads of the activation loader's step, then advance it
+            if (pb.item < nitems) {
+                if (pb.kt < pb.KW) issue_b(cb, pb.kt, seq % kRB);  // LoRA-B steps are staged by the consumer
+                if (++pb.kt == pb.KT) {
+                    decode(pb.item + NB, pb);
+                    make_b(pb, cb);
+                }
+            }
+            tc::cp_commit();
+        };
+        for (int i = 0; i < kLB; ++i) issue_step(i);
+        // scale/bias registers: current span and the next one
+        uint32_t s_cur[4] = {0, 0, 0, 0}, b_cur[4] = {0, 0, 0, 0}, s_nxt[4] = {0, 0, 0, 0}, b_nxt[4] = {0, 0, 0, 0};
+        Pos pn = pc;  // item of the next span whose scales are fetched
+        int pn_span = 0;
+        auto sb_next = [&]() {
+            if (pn.item >= nitems) return;
+            fetch_sb(pn, pn_span, s_nxt, b_nxt);
+            if (++pn_span * SP >= pn.KW) {
+                decode(pn.item + NB, pn);
+                pn_span = 0;
+            }
+        };
+        if (!lora_mode) sb_next();
+        LoraRegs lr;
+
+        uint32_t t = 0;        // steps consumed by this CTA
+        uint32_t sseq = 0;     // weight spans consumed by this CTA
+        uint32_t n_items = 0;  // items finished by this CTA
+        while (pc.item < nitems) {
+            const bool wstep = pc.kt < pc.KW;
+            const bool span_start = !lora_mode && wstep && pc.kt % SP == 0;
+            // the MMAs of step t-2 must be done before A stage t%2 and activation slot (t+kLB)%kRB are rewritten
+            if (t >= 2 && !tc::mbar_wait_ok(&bar_tile[(t - 2) % 4], ((t - 2) / 4) & 1u, a.status, &s_ok)) break;
+            if (span_start) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    s_cur[j] = s_nxt[j];
+                    b_cur[j] = b_nxt[j];
+                }
+                sb_next();
+            }
+            // inputs of the first LoRA-B step, fetched during the last weight step so their latency
+            // overlaps it (later LoRA-B steps fetch theirs right after staging the previous one)
+            if (NL > 0 && pc.kt + 1 == pc.KW) fetch_lora(pc, 0, lr);
+            issue_step(t + kLB);
+            tc::cp_wait<kLB>();  // this step's group (issued kLB steps ago) has landed
+            if (span_start && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) break;
+
+            unsigned char* stA = sA + (t % 2) * kAStage;
+            const int kk = pc.kt % SP;  // K-step inside the span
+            if (int4_mode && wstep) {
+                // words 8kk .. 8kk+7 = 16-byte chunks 2kk, 2kk+1 of the swizzled 128-byte row
+                const unsigned char* rowp = sR + (sseq % kRS) * kRawSlot + wblk * kSpanBytes + wrow * 128;
+                const uint4 wa = *reinterpret_cast<const uint4*>(rowp + (((2 * kk) ^ (wrow & 7)) << 4));
+                const uint4 wb = *reinterpret_cast<const uint4*>(rowp + (((2 * kk + 1) ^ (wrow & 7)) << 4));
+                const int ga = (kk * 64) >> gshift, gb = (kk * 64 + 32) >> gshift;  // groups of words 0-3, 4-7
+                const __nv_bfloat162 sa = bf16x2_of(pick4(s_cur, ga >> 1) >> (16 * (ga & 1)));
+                const __nv_bfloat162 ba = bf16x2_of(pick4(b_cur, ga >> 1) >> (16 * (ga & 1)));
+                const __nv_bfloat162 sb = bf16x2_of(pick4(s_cur, gb >> 1) >> (16 * (gb & 1)));
+                const __nv_bfloat162 bb = bf16x2_of(pick4(b_cur, gb >> 1) >> (16 * (gb & 1)));
+                unsigned char* arow = stA + wblk * (kBM * 128);
+                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 0)) = dequant8(wa.x, sa, ba);
+                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 1)) = dequant8(wa.y, sa, ba);
+                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 2)) = dequant8(wa.z, sa, ba);
+                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 3)) = dequant8(wa.w, sa, ba);
+                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 4)) = dequant8(wb.x, sb, bb);
+                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 5)) = dequant8(wb.y, sb, bb);
+                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 6)) = dequant8(wb.z, sb, bb);
+                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 7)) = dequant8(wb.w, sb, bb);
+            } else if (int4_mode) {
+                stage_lora(lr, sB + (t % kRB) * kBBytes);
+                if (pc.kt + 1 < pc.KT) fetch_lora(pc, pc.kt + 1 - pc.KW, lr);
+            } else if (int8_mode) {
+                // half wh of this K-step's 16 words: chunks 4kk + 2wh, 4kk + 2wh + 1 of the row
+                const unsigned char* rowp = sR + (sseq % kRS) * kRawSlot + wrow * 128;
+                const int gg = (kk * 64 + wh * 32) >> gshift;
+                const float s = bf16f((uint16_t)(pick4(s_cur, gg >> 1) >> (16 * (gg & 1))));
+                const float b = bf16f((uint16_t)(pick4(b_cur, gg >> 1) >> (16 * (gg & 1))));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + (((4 * kk + 2 * wh + h) ^ (wrow & 7)) << 4));
+                    uint4 hi, lo;
+                    dequant8_hilo(w4.x, w4.y, s, b, hi, lo);  // output chunk 4 wh + 2h
+                    uint32_t off = tc::sw128_off(wrow, 4 * wh + 2 * h);
+                    *reinterpret_cast<uint4*>(stA + off) = hi;
+                    *reinterpret_cast<uint4*>(stA + kBM * 128 + off) = lo;
+                    dequant8_hilo(w4.z, w4.w, s, b, hi, lo);  // output chunk 4 wh + 2h + 1
+                    off = tc::sw128_off(wrow, 4 * wh + 2 * h + 1);
+                    *reinterpret_cast<uint4*>(stA + off) = hi;
+                    *reinterpret_cast<uint4*>(stA + kBM * 128 + off) = lo;
+                }
+            } else {
+                const unsigned char* raw = sR + (t % kRB) * kLoraSlot;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int row = brow + 32 * j;
+                    *reinterpret_cast<uint4*>(stA + tc::sw128_off(row, bch)) =
+                        *reinterpret_cast<const uint4*>(raw + row * 128 + bch * 16);
+                }
+            }
+            // hand the stage to the MMA warp: generic writes (and this thread's landed
+            // cp.async data) made visible to the tensor core, then one arrival per warp
+            tc::fence_async_smem();
             tc::tc_fence_before();
-            __syncthreads();
-            ++seq_c;
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(&bar_full[t % 2]);
+                if (!lora_mode && (!wstep || kk == SP - 1 || pc.kt == pc.KW - 1)) tc::mbar_arrive(&bar_rawfree[sseq % kRS]);
+            }
+            ++t;
+
+            if (pc.kt == pc.KT - 1) {
+                // ---------------------------------------------------- epilogue
+                if (!tc::mbar_wait_ok(&bar_acc, n_items & 1u, a.status, &s_ok)) break;
+                ++n_items;
+                tc::tc_fence_after();
+                const Geo q = geo_of(a, pc.g, s_goff[pc.g + 1] - s_goff[pc.g]);
+                const int n_here = tile_jobs(pc);
+                const int base = s_goff[pc.g] + pc.nt * kNT;
+                const int quarter = warp % 4;         // TMEM lane quarter of this warp
+                const int row = quarter * 32 + lane;  // TMEM lane of this thread
+                for (int ch = warp / 4; ch * 16 < n_here; ch += 2) {  // 16-column chunks
+                    uint32_t d0[16], d1[16];
+                    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ch * 16;
+                    tc::tmem_ld16(taddr, d0);
+                    if (int4_mode) tc::tmem_ld16(taddr + 256, d1);
+                    tc::tmem_wait_ld();
+                    if (mode == kGU) {
+                        const int i = pc.mt * kBM + row;
+                        if (i < q.M) {
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) {
+                                const int n = ch * 16 + c;
+                                if (n < n_here)
+                                    a.h_out[(int64_t)(base + n) * a.ldh + i] =
+                                        f2bf16(silu(__uint_as_float(d0[c])) * __uint_as_float(d1[c]));
+                            }
+                        }
+                    } else if (mode == kDown) {
+                        const int o0 = pc.mt * 2 * kBM + row;
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const int n = ch * 16 + c;
+                            if (n < n_here) {
+                                const float wj = a.wperm ? __ldg(a.wperm + base + n) : 0.0f;
+                                float* yp = a.ypart + (int64_t)(base + n) * L.H;
+                                if (o0 < q.M) yp[o0] = wj * __uint_as_float(d0[c]);
+                                if (o0 + kBM < q.M) yp[o0 + kBM] = wj * __uint_as_float(d1[c]);
+                            }
+                        }
+                    } else if (int8_mode) {
+                        const int e = pc.mt * kBM + row;
+                        if (e < q.M) {
+                            const float lb = L.logit_bias ? L.logit_bias[e] : 0.0f;
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) {
+                                const int n = ch * 16 + c;
+                                if (n < n_here) a.logits[(int64_t)(base + n) * L.E + e] = __uint_as_float(d0[c]) + lb;
+                            }
+                        }
+                    } else {
+                        const int rpa = mode == kLoraGU ? 2 * r : r;
+                        const int R = pc.mt * kLoraRows + row;
+                        if (row < kLoraRows && R < q.M) {
+                            const int ad = R / rpa, d = R % rpa;
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) {
+                                const int n = ch * 16 + c;
+                                if (n < n_here && __ldg(&a.perm[base + n].z) == ad)
+                                    a.t_out[(int64_t)(base + n) * rpa + d] = __uint_as_float(d0[c]);
+                            }
+                        }
+                    }
+                }
+                // the next item's first MMA overwrites the accumulators: its stage arrival
+                // (after these reads) orders them
+                tc::tc_fence_before();
+            }
+            // advance the consumer
+            if (++pc.kt == pc.KT) decode(pc.item + NB, pc);
+            if (!lora_mode && pc.item < nitems && (pc.kt >= pc.KW || pc.kt % SP == 0)) ++sseq;  // next step opens a span
         }
-        advance(pc);
+        // no cp.async may still target this CTA's shared memory at exit
+        tc::cp_wait<0>();
+        if (pc.item < nitems) s_ok = 0;  // left early: let the producer stop waiting
     }
-    // drain: no cp.async may still target this CTA's shared memory at exit
-    tc::cp_wait<0>();
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+    if (warp == kDeqWarps) tc::tmem_dealloc(tmem, 512);
 }
 
-}  // namespace
-
-// Host-side conditions of the tensor-core path.
-bool tc_supported(const LayerArgs& L) {
-    if (L.H % 128 || L.I % 128 || L.H < 128 || L.I < 128) return false;
-    if (L.has_shared && (L.Is % 128 || L.Is < 128)) return false;
-    if (L.gate.group != 64 && L.gate.group != 32) return false;
-    if (L.down.group != L.gate.group || (L.has_shared && (L.s_gate.group != L.gate.group || L.s_down.group != L.gate.group)))
-        return false;
-    if (L.rank > MOEQ_MAX_RANK / 2) return false;
-    if (L.E + 1 > kMaxGroups) return false;
-    // scale/bias pairs are fetched as 4-byte words
-    const moe_qtensor* ts[] = {&L.gate, &L.up, &L.down, &L.s_gate, &L.s_up, &L.s_down};
-    for (const moe_qtensor* q : ts)
-        if (q->packed && (((uintptr_t)q->scales & 3) || ((uintptr_t)q->biases & 3))) return false;
-    return true;
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
 }
 
-size_t tc_smem_bytes() { return 2 * kAStage + kRB * kBBytes + kRA * kRawBytes + 1024; }
+// Tensor map over packed words [rows][words_per_row] (uint32), boxes of 32 words x
+// 128 rows with the 128-byte swizzle; out-of-range rows and words read as zero.
+cudaError_t encode_words(CUtensorMap* m, const void* base, int64_t rows, int64_t words_per_row) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)words_per_row, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)words_per_row * 4};
+    const cuuint32_t box[2] = {32, (cuuint32_t)kBM};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 
-cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, int ld_act, const Work& wk,
-                           const uint16_t* hb_out, int ldh, cudaStream_t s) {
+bool words_tma_ok(const moe_qtensor& q) {
+    const int wpr = q.in * q.bits / 32;
+    return q.packed && ((uintptr_t)q.packed & 15) == 0 && (wpr * 4) % 16 == 0 && ((uintptr_t)q.scales & 3) == 0 &&
+           ((uintptr_t)q.biases & 3) == 0;
+}
+
+cudaError_t launch_kernel(TcArgs& a, cudaStream_t s) {
     static int cached = 0;
-    const size_t smem = tc_smem_bytes();
+    const size_t smem = 2 * kAStage + kRB * kBBytes + kRS * kRawSlot + 1024;
     cudaError_t e = ensure_smem((const void*)tc_gemm_kernel, smem, cached);
     if (e != cudaSuccess) return e;
     int nsm = 0, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    tc_gemm_kernel<<<nsm, kTcThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Host-side conditions of the tensor-core expert path.
+bool tc_supported(const LayerArgs& L) {
+    if (L.H % 128 || L.I % 128 || L.H < 128 || L.I < 128) return false;
+    if (L.has_shared && (L.Is % 128 || L.Is < 128)) return false;
+    if (L.gate.group != 64 && L.gate.group != 32) return false;
+    if (L.gate.bits != 4 || L.up.bits != 4 || L.down.bits != 4) return false;
+    if (L.up.group != L.gate.group || L.down.group != L.gate.group) return false;
+    if (L.has_shared && (L.s_gate.group != L.gate.group || L.s_up.group != L.gate.group ||
+                         L.s_down.group != L.gate.group || L.s_gate.bits != 4 || L.s_up.bits != 4 ||
+                         L.s_down.bits != 4))
+        return false;
+    if (L.E + 1 > kMaxGroups) return false;
+    // LoRA-B rows and LoRA-A products are moved in 8-element chunks that never
+    // straddle two adapters: rank a multiple of 8, B rows 16-byte aligned
+    if (L.n_adapters > 0 && L.rank > 0) {
+        if (L.rank % 8) return false;
+        for (int ad = 0; ad < L.n_adapters; ++ad) {
+            const moe_lora_proj* ps[] = {&L.lora[ad].gate, &L.lora[ad].up, &L.lora[ad].down,
+                                         &L.lora[ad].s_gate, &L.lora[ad].s_up, &L.lora[ad].s_down};
+            for (const moe_lora_proj* p : ps)
+                if (p->B && ((uintptr_t)p->B & 15)) return false;
+        }
+    }
+    if (!words_tma_ok(L.gate) || !words_tma_ok(L.up) || !words_tma_ok(L.down)) return false;
+    if (L.has_shared && (!words_tma_ok(L.s_gate) || !words_tma_ok(L.s_up) || !words_tma_ok(L.s_down))) return false;
+    return encode_fn() != nullptr;
+}
+
+bool tc_router_supported(const moe_qtensor& router, int H, int E) {
+    return H % 128 == 0 && H >= 128 && E >= 1 && router.bits == 8 && (router.group == 64 || router.group == 32) &&
+           router.in == H && words_tma_ok(router) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, int ld_act, const Work& wk,
+                           const uint16_t* hb_out, int ldh, cudaStream_t s) {
     TcArgs a;
+    memset(&a, 0, sizeof(a));
     a.L = L;
     a.mode = mode;
     a.act = act;
@@ -519,11 +840,41 @@ cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, in
     a.h_out = const_cast<uint16_t*>(hb_out);
     a.ldh = ldh;
     a.ypart = wk.ypart;
-    a.t_out = mode == kLoraGU ? wk.tgu : wk.td;
-    a.t_in = mode == kGU ? wk.tgu : wk.td;
+    a.t_out = mode == kTcLoraGU ? wk.tgu : wk.td;
+    a.t_in = mode == kTcGU ? wk.tgu : wk.td;
     a.status = wk.status;
-    tc_gemm_kernel<<<nsm, kTcThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = cudaSuccess;
+    if (mode == kTcGU) {
+        e = encode_words(&a.tm[0], L.gate.packed, (int64_t)L.E * L.I, L.H / 8);
+        if (e == cudaSuccess) e = encode_words(&a.tm[1], L.up.packed, (int64_t)L.E * L.I, L.H / 8);
+        if (e == cudaSuccess && L.has_shared) e = encode_words(&a.tm[2], L.s_gate.packed, L.Is, L.H / 8);
+        if (e == cudaSuccess && L.has_shared) e = encode_words(&a.tm[3], L.s_up.packed, L.Is, L.H / 8);
+    } else if (mode == kTcDown) {
+        e = encode_words(&a.tm[0], L.down.packed, (int64_t)L.E * L.H, L.I / 8);
+        if (e == cudaSuccess && L.has_shared) e = encode_words(&a.tm[1], L.s_down.packed, L.H, L.Is / 8);
+    }
+    if (e != cudaSuccess) return e;
+    return launch_kernel(a, s);
+}
+
+cudaError_t launch_tc_router(const moe_qtensor& router, const float* logit_bias, const uint16_t* x, int T, int H,
+                             int E, float* logits, int32_t* status, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    TcArgs a;
+    memset(&a, 0, sizeof(a));
+    a.L.router = router;
+    a.L.logit_bias = logit_bias;
+    a.L.H = H;
+    a.L.E = E;
+    a.mode = kRouterMode;
+    a.act = x;
+    a.ld_act = H;
+    a.logits = logits;
+    a.T = T;
+    a.status = status;
+    cudaError_t e = encode_words(&a.tm[0], router.packed, E, H / 4);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(a, s);
 }
 
 }  // namespace moeq
