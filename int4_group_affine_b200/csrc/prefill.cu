@@ -2,20 +2,25 @@
 // the many-token case: the 8-bit router, gate/up with fused SwiGLU, down with
 // the routing weight, and the two LoRA-A products.
 //
-// Swap-AB: a tile is weight rows (M, one TMEM lane each) by up to 64 jobs of one
-// expert group (N), over K in steps of 64.  Operand tiles live in shared memory
-// K-major with the 128-byte swizzle, the layout the MMA descriptors name.
+// Swap-AB: a tile is weight rows (M = 128, one TMEM lane each) by up to 64 jobs
+// of one expert group (N), over K in steps of 64.
 //
 // Weights stream through the tensor memory accelerator: for each span of 128
-// bytes of packed words per row (K = 256 for int4, 128 for int8) one elected
-// thread loads a 128-row box per block with cp.async.bulk.tensor into a ring of
-// three slots, two spans ahead, so DRAM sees whole 128-byte lines.  Each thread
-// owns one weight row (half of one for int8): it prefetches that row's scales
-// and biases into registers one span ahead and dequantises its 64 weights of
-// each K-step into bf16 (w = fma(q, s, b), one rounding).  Activations (rows
-// gathered by token, or the h rows of the jobs) come in with cp.async four
-// K-steps ahead.  One thread issues the MMAs (4 x K=16 per block) and commits
-// them to an mbarrier.
+// bytes of packed words per row (K = 256 for int4, 128 for int8) the producer
+// warp loads a 128-row box per block with cp.async.bulk.tensor (128-byte
+// swizzle) into a ring of four slots, three spans ahead, so DRAM sees whole
+// 128-byte lines.  Each dequantisation thread owns one weight row (half of one
+// for int8) and thus one TMEM lane: it prefetches the row's scales and biases
+// into registers one span ahead, dequantises the row's 64 weights of each K-step
+// into bf16 (w = fma(q, s, b), one rounding) and writes them with tcgen05.st
+// into one of four TMEM stages, the MMA's A operand; the dequantised tile never
+// touches shared memory, whose bandwidth then serves the MMA's B reads.
+// Activations (rows gathered by token, or the h rows of the jobs) come in with
+// cp.async four K-steps ahead into a K-major 128-byte-swizzled ring (operand B).
+// One producer lane issues the MMAs (4 x K=16 per block) and commits them to
+// mbarriers; accumulators are double-buffered in TMEM and each item's epilogue
+// runs a few steps after its last MMA, so the dequantisation never waits on the
+// tensor core at item boundaries.
 //
 // The unmerged LoRA-B term (alpha/r) B (A x) is one more MMA K-step per item
 // (per 64 columns of K' = adapters x r per matrix): operand A holds the LoRA-B
@@ -33,12 +38,13 @@
 //   router:  int8 rows; block 0 = bf16(w), block 1 = bf16(w - bf16(w)), both
 //            into one accumulator, so the logits carry ~16 bits of each weight;
 //            epilogue adds the logit bias -> logits.
-//   LoRA-A:  bf16 A rows of every adapter (cp.async), 64 real rows per tile.
+//   LoRA-A:  bf16 A rows of every adapter, copied by cp.async straight into the
+//            swizzled operand layout, 64 real rows per tile.
 //
 // Warp roles: 8 dequantisation warps (loads of activations and scales, dequant,
-// epilogue) and one producer warp whose lane 0 issues the TMA spans and the MMAs;
-// they hand stages over through mbarriers, so no CTA-wide barrier sits in the
-// K loop.  Persistent grid: CTA c takes items c, c + grid, ...
+// epilogue) and one producer warp (TMA spans, LoRA-B rows, MMA issue); they hand
+// steps over through mbarriers, so no CTA-wide barrier sits in the K loop.
+// Persistent grid: CTA c takes items c, c + grid, ...
 #include <cudaTypedefs.h>
 
 #include "tc.cuh"
@@ -46,21 +52,25 @@
 namespace moeq {
 namespace {
 
-constexpr int kDeqWarps = 8;                     // dequantisation warps
-constexpr int kTcThreads = (kDeqWarps + 1) * 32;  // + the producer warp (TMA and MMA issue)
-constexpr int kBM = 128;                  // rows per MMA block
-constexpr int kNT = 64;                   // jobs per tile (MMA N <= 64)
-constexpr int kLB = 4;                    // activation lookahead (K-steps)
-constexpr int kRB = kLB + 2;              // activation ring: a slot is free once the MMAs of its step are done
-constexpr int kRS = 3;                    // weight span ring (two spans in flight)
-constexpr int kSpanBytes = kBM * 128;     // one block of one span: 128 rows x 128 B
-constexpr int kRawSlot = 2 * kSpanBytes;  // two blocks
-constexpr int kBBytes = kNT * 128;        // 64 rows x 128 B
-constexpr int kAStage = 2 * kBM * 128;    // two bf16 blocks of 128 x 64 (32 KB)
-constexpr int kLoraRows = 64;             // real LoRA-A rows per M tile
+constexpr int kDeqWarps = 8;                      // dequantisation warps
+constexpr int kTcThreads = (kDeqWarps + 1) * 32;  // + the producer warp (TMA, LoRA-B rows, MMA issue)
+constexpr int kBM = 128;                          // rows per MMA block
+constexpr int kNT = 64;                           // jobs per tile (MMA N <= 64)
+constexpr int kAS = 4;                            // A stages in TMEM (dequantisation runs up to kAS steps ahead)
+constexpr int kLB = 4;                            // activation lookahead (K-steps)
+constexpr int kRB = kLB + kAS;                    // activation ring: slot of step t - kAS is free at step t
+constexpr int kRS = 4;                            // weight span ring (three spans in flight)
+constexpr int kTiles = 8;                         // per-step MMA completion barriers
+constexpr int kSpanBytes = kBM * 128;             // one block of one span: 128 rows x 128 B
+constexpr int kRawSlot = 2 * kSpanBytes;          // two blocks
+constexpr int kBBytes = kNT * 128;                // 64 rows x 128 B
+constexpr int kLoraRows = 64;                     // real LoRA-A rows per M tile
 constexpr int kLoraSlot = kLoraRows * 128;
 constexpr int kMaxGroups = MOEQ_MAX_EXPERTS + 1;
+// TMEM columns: accumulator D(buffer b, block k) at 128 b + 64 k; A stage s, block k at 256 + 64 s + 32 k
+constexpr uint32_t kTmemA = 256;
 static_assert(kRB * kLoraSlot <= kRS * kRawSlot, "LoRA-A ring must fit in the weight ring");
+static_assert(kTmemA + kAS * 64 <= 512, "TMEM columns");
 
 enum Mode { kGU = 0, kDown = 1, kLoraGU = 2, kLoraDown = 3, kRouterMode = 4 };
 
@@ -138,7 +148,7 @@ __device__ __forceinline__ const moe_lora_proj* tlora(const LayerArgs& L, int a,
     return (q->A && q->B) ? q : nullptr;
 }
 
-// 8 nibbles of one word -> 8 bf16 (s*q + b, one rounding), in element order.
+// 8 nibbles of one word -> 8 bf16 (s*q + b, one rounding), as 4 pairs in element order.
 __device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
     const __nv_bfloat162 k128 = __float2bfloat162_rn(128.0f);
     uint32_t r[4];
@@ -158,8 +168,7 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bf
 }
 
 // Two int8 words (8 codes) -> hi = bf16(w) and lo = bf16(w - hi) for w = s*q + b in fp32.
-__device__ __forceinline__ void dequant8_hilo(uint32_t w0, uint32_t w1, float s, float b, uint4& hi, uint4& lo) {
-    uint32_t h[4], l[4];
+__device__ __forceinline__ void dequant8_hilo(uint32_t w0, uint32_t w1, float s, float b, uint32_t* hi, uint32_t* lo) {
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         const uint32_t w = p < 2 ? w0 : w1;
@@ -169,11 +178,9 @@ __device__ __forceinline__ void dequant8_hilo(uint32_t w0, uint32_t w1, float s,
         const __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
         const float2 hf = __bfloat1622float2(hv);
         const __nv_bfloat162 lv = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
-        h[p] = *reinterpret_cast<const uint32_t*>(&hv);
-        l[p] = *reinterpret_cast<const uint32_t*>(&lv);
+        hi[p] = *reinterpret_cast<const uint32_t*>(&hv);
+        lo[p] = *reinterpret_cast<const uint32_t*>(&lv);
     }
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 __device__ __forceinline__ uint32_t pick4(const uint32_t (&v)[4], int i) {
@@ -184,19 +191,22 @@ __device__ __forceinline__ __nv_bfloat162 bf16x2_of(uint32_t half_word) {
     return __bfloat162bfloat162(__ushort_as_bfloat16((unsigned short)(half_word & 0xFFFFu)));
 }
 
-// This thread's activation chunk (and LoRA-A chunk) of one item.
+// This thread's activation chunks (and LoRA-A chunks) of one item.
 struct BCtx {
     const uint16_t* src[2];
     const uint16_t* la[2];  // LoRA-A modes: bf16 A chunks (NULL: zero fill)
     bool live[2];
 };
 
-// Registers of one LoRA-B step, fetched a step ahead.
+// LoRA-B operand B of one step, fetched a step ahead.
 struct LoraRegs {
     float4 t[2][2];  // LoRA-A products of this thread's two (job, chunk) pairs, unscaled
     bool t_live[2];
 };
 
+// One instantiation per mode, so that each kernel holds only its own path (a
+// loop body small enough for the instruction caches).
+template <int kMode>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ __align__(1024) unsigned char tsm_raw[];
     // 128-byte-swizzled tiles need 1024-byte aligned bases: align by hand (the
@@ -204,21 +214,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     unsigned char* tsm = tsm_raw + ((1024u - (tc::smem_u32(tsm_raw) & 1023u)) & 1023u);
     const LayerArgs& L = a.L;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int mode = a.mode;
-    const bool lora_mode = mode == kLoraGU || mode == kLoraDown;
-    const bool int8_mode = mode == kRouterMode;
-    const bool int4_mode = mode == kGU || mode == kDown;
-    const int SP = int8_mode ? 2 : 4;  // K-steps per weight span (128 B of words per row)
+    constexpr int mode = kMode;
+    constexpr bool lora_mode = mode == kLoraGU || mode == kLoraDown;
+    constexpr bool int8_mode = mode == kRouterMode;
+    constexpr bool int4_mode = mode == kGU || mode == kDown;
+    constexpr int SP = int8_mode ? 2 : 4;  // K-steps per weight span (128 B of words per row)
     const int r = L.rank;
     const int NL = lora_steps(a);
 
-    // shared memory: [A stages 2 x 32 KB][activation ring kRB x 8 KB][weight ring kRS x 32 KB]
-    unsigned char* sA = tsm;
-    unsigned char* sB = sA + 2 * kAStage;
+    // shared memory: [activation ring kRB x 8 KB][weight ring kRS x 32 KB]
+    unsigned char* sB = tsm;
     unsigned char* sR = sB + kRB * kBBytes;
-    __shared__ uint64_t bar_full[2];      // A stage (and its activation slot) written: one arrival per dequant warp
-    __shared__ uint64_t bar_tile[4];      // MMAs of a step done (tcgen05.commit)
-    __shared__ uint64_t bar_acc;          // MMAs of an item done
+    __shared__ uint64_t bar_full[kAS];    // step's operands written: one arrival per dequant warp
+    __shared__ uint64_t bar_tile[kTiles]; // MMAs of a step done (tcgen05.commit)
+    __shared__ uint64_t bar_acc[2];       // MMAs of an item done, per accumulator buffer
     __shared__ uint64_t bar_raw[kRS];     // span landed: 32 producer-lane arrivals (+ TMA transaction count)
     __shared__ uint64_t bar_rawfree[kRS]; // span consumed: one arrival per dequant warp + the producer's commit
     __shared__ uint32_t s_tmem;
@@ -241,18 +250,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) tc::mbar_init(&bar_full[i], kDeqWarps);
-        for (int i = 0; i < 4; ++i) tc::mbar_init(&bar_tile[i], 1);
+        for (int i = 0; i < kAS; ++i) tc::mbar_init(&bar_full[i], kDeqWarps);
+        for (int i = 0; i < kTiles; ++i) tc::mbar_init(&bar_tile[i], 1);
         for (int i = 0; i < kRS; ++i) {
             tc::mbar_init(&bar_raw[i], 32);
             tc::mbar_init(&bar_rawfree[i], kDeqWarps + 1);
         }
-        tc::mbar_init(&bar_acc, 1);
+        tc::mbar_init(&bar_acc[0], 1);
+        tc::mbar_init(&bar_acc[1], 1);
         tc::mbar_init_fence();
         s_ok = 1;
     }
-    // zero both A stages once (LoRA-A modes never write rows 64..127)
-    for (int i = tid; i < 2 * kAStage / 16; i += kTcThreads) reinterpret_cast<uint4*>(sA)[i] = make_uint4(0, 0, 0, 0);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -293,10 +301,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         p.KT = p.KW + NL;
     };
     auto tile_jobs = [&](const Pos& p) { return min(kNT, s_goff[p.g + 1] - s_goff[p.g] - p.nt * kNT); };
-
     const int nar = L.n_adapters * r;
     // spans of an item in the weight ring: its weight spans, then one per LoRA-B step
     auto wspans = [&](const Pos& p) { return (p.KW + SP - 1) / SP; };
+
     if (warp == kDeqWarps) {
         // ====================================================== producer warp: TMA, LoRA-B rows, MMA issue
         Pos pc;
@@ -372,21 +380,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 pt_span = 0;
             }
         };
-        if (!lora_mode) {
-            span_next();
-            span_next();
-        }
-        uint32_t t = 0, cs = 0;  // steps and spans consumed
+        if (!lora_mode)
+            for (int i = 0; i < kRS - 1; ++i) span_next();
+        uint32_t t = 0, cs = 0, ib = 0;  // steps, spans and items consumed
         while (pc.item < nitems && ok) {
             const bool wstep = pc.kt < pc.KW;
             const bool opens = !lora_mode && (!wstep || pc.kt % SP == 0);
-            if (opens) span_next();  // keep two spans ahead
-            if (!ok || !tc::mbar_wait_ok(&bar_full[t % 2], (t / 2) & 1u, a.status, &s_ok)) {
+            if (opens) span_next();  // keep kRS - 1 spans ahead
+            if (!ok || !tc::mbar_wait_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok)) {
                 ok = false;
                 break;
             }
             // LoRA-B step: its operand A (this warp's own copies) must have landed
-            if (!wstep && !tc::mbar_wait_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok)) {
+            if (!lora_mode && !wstep && !tc::mbar_wait_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok)) {
                 ok = false;
                 break;
             }
@@ -394,34 +400,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (lane == 0) {
                 const int Nmma = (tile_jobs(pc) + 15) / 16 * 16;
                 const uint32_t idesc = tc::idesc_bf16(kBM, Nmma);
-                const uint32_t bbase = tc::smem_u32(sB + (t % kRB) * kBBytes);
-                const uint32_t sbase = wstep ? tc::smem_u32(sA + (t % 2) * kAStage) : tc::smem_u32(sR + (cs % kRS) * kRawSlot);
-                const int nblk = lora_mode ? 1 : 2;
-                for (int blk = 0; blk < nblk; ++blk) {
-                    const uint32_t boff = wstep ? blk * (kBM * 128) : blk * kSpanBytes;
-                    const uint64_t ad = tc::sdesc_k_sw128(sbase + boff), bd = tc::sdesc_k_sw128(bbase);
-                    // router: hi and lo parts into one accumulator; otherwise one accumulator per block
-                    const uint32_t d = tmem + (int8_mode ? 0u : (uint32_t)blk * 256u);
-                    for (int k = 0; k < 4; ++k) {  // 4 x K=16 inside the 128-byte swizzle atom: +32 B each
-                        const bool first = pc.kt == 0 && k == 0 && (!int8_mode || blk == 0);
-                        tc::mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, first ? 0u : 1u);
+                const uint64_t bd = tc::sdesc_k_sw128(tc::smem_u32(sB + (t % kRB) * kBBytes));
+                const uint32_t dacc = tmem + (ib & 1u) * 128u;
+                if (lora_mode) {  // A: the LoRA-A rows, copied swizzled into the ring
+                    const uint64_t ad = tc::sdesc_k_sw128(tc::smem_u32(sR + (t % kRB) * kLoraSlot));
+                    for (int k = 0; k < 4; ++k) tc::mma_bf16(dacc, ad + 2 * k, bd + 2 * k, idesc, (pc.kt > 0 || k > 0) ? 1u : 0u);
+                } else if (!wstep) {  // LoRA-B step: A = LoRA-B rows of the pseudo-span, one accumulator per block
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const uint64_t ad = tc::sdesc_k_sw128(tc::smem_u32(sR + (cs % kRS) * kRawSlot + blk * kSpanBytes));
+                        for (int k = 0; k < 4; ++k) tc::mma_bf16(dacc + blk * 64, ad + 2 * k, bd + 2 * k, idesc, 1u);
+                    }
+                } else {  // weight step: A = the dequantised tile in TMEM
+                    const uint32_t astage = tmem + kTmemA + (t % kAS) * 64;
+                    for (int blk = 0; blk < 2; ++blk) {
+                        // router: hi and lo parts into one accumulator; otherwise one accumulator per block
+                        const uint32_t d = dacc + (int8_mode ? 0u : (uint32_t)blk * 64u);
+                        for (int k = 0; k < 4; ++k) {  // K=16 per MMA: 8 TMEM columns, +32 B in the swizzled B tile
+                            const bool first = pc.kt == 0 && k == 0 && (!int8_mode || blk == 0);
+                            tc::mma_bf16_ts(d, astage + blk * 32 + 8 * k, bd + 2 * k, idesc, first ? 0u : 1u);
+                        }
                     }
                 }
-                tc::mma_commit(&bar_tile[t % 4]);
+                tc::mma_commit(&bar_tile[t % kTiles]);
                 // the span's slot is free once these MMAs are done (they read it directly for LoRA-B)
                 if (!lora_mode && (!wstep || pc.kt % SP == SP - 1 || pc.kt == pc.KW - 1))
                     tc::mma_commit(&bar_rawfree[cs % kRS]);
-                if (pc.kt == pc.KT - 1) tc::mma_commit(&bar_acc);
+                if (pc.kt == pc.KT - 1) tc::mma_commit(&bar_acc[ib & 1u]);
             }
             __syncwarp();
             ++t;
+            if (pc.kt == pc.KT - 1) ++ib;
             if (++pc.kt == pc.KT) decode(pc.item + NB, pc);
             if (!lora_mode && pc.item < nitems && (pc.kt >= pc.KW || pc.kt % SP == 0)) ++cs;
         }
         // drain (bounded): this warp's copies, the last MMAs, the latest span issued into each slot
         tc::cp_wait<0>();
         if (lane == 0) {
-            if (t > 0) tc::mbar_wait(&bar_tile[(t - 1) % 4], ((t - 1) / 4) & 1u, a.status);
+            if (t > 0) tc::mbar_wait(&bar_tile[(t - 1) % kTiles], ((t - 1) / kTiles) & 1u, a.status);
             for (uint32_t sq = issued > (uint32_t)kRS ? issued - kRS : 0; sq < issued; ++sq)
                 tc::mbar_wait(&bar_raw[sq % kRS], (sq / kRS) & 1u, a.status);
             if (!ok) s_ok = 0;
@@ -430,10 +445,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     } else {
         // ====================================================== dequantisation warps
         // ---- weight rows.  int4: thread -> (block, row), the K-step's 8 words of the row;
-        //      int8: thread -> (row, half of the K-step's 16 words)
+        //      int8: thread -> (row, half of the K-step's 16 words).  Warp w writes TMEM
+        //      lanes 32 (w % 4) .. +31, which are its rows.
         const int wrow = tid % kBM;
         const int wblk = int8_mode ? 0 : tid / kBM;
         const int wh = tid / kBM;  // int8: half
+        const uint32_t tlane = (uint32_t)((warp % 4) * 32) << 16;
         const int group = int8_mode ? L.router.group : L.gate.group;
         const int gshift = group == 64 ? 6 : 5;
         // scale/bias words (pairs of bf16) of one span of this thread's row
@@ -499,9 +516,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             for (int j = 0; j < 2; ++j) {
                 const int row = brow + 32 * j;
                 tc::cp16(base + tc::sw128_off(row, bch), c.src[j] + (c.live[j] ? kt * 64 : 0), c.live[j] ? 16u : 0u);
-                if (lora_mode)  // this thread's own LoRA-A chunks; it copies them into the A stage itself
-                    tc::cp16(rb + (uint32_t)(row * 128 + bch * 16), c.la[j] ? c.la[j] + kt * 64 : a.act,
-                             c.la[j] ? 16u : 0u);
+                if (lora_mode)  // LoRA-A rows straight into the MMA's swizzled operand layout
+                    tc::cp16(rb + tc::sw128_off(row, bch), c.la[j] ? c.la[j] + kt * 64 : a.act, c.la[j] ? 16u : 0u);
             }
         };
 
@@ -547,6 +563,72 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
         };
 
+        // ---- epilogue of a finished item (accumulator buffer seq % 2)
+        auto epilogue = [&](const Pos& p, uint32_t seq) -> bool {
+            if (!tc::mbar_wait_ok(&bar_acc[seq & 1u], (seq >> 1) & 1u, a.status, &s_ok)) return false;
+            tc::tc_fence_after();
+            const Geo q = geo_of(a, p.g, s_goff[p.g + 1] - s_goff[p.g]);
+            const int n_here = tile_jobs(p);
+            const int base = s_goff[p.g] + p.nt * kNT;
+            const uint32_t dacc = tmem + tlane + (seq & 1u) * 128u;
+            const int row = (warp % 4) * 32 + lane;  // TMEM lane of this thread
+            for (int ch = warp / 4; ch * 16 < n_here; ch += 2) {  // 16-column chunks
+                uint32_t d0[16], d1[16];
+                tc::tmem_ld16(dacc + ch * 16, d0);
+                if (int4_mode) tc::tmem_ld16(dacc + 64 + ch * 16, d1);
+                tc::tmem_wait_ld();
+                if (mode == kGU) {
+                    const int i = p.mt * kBM + row;
+                    if (i < q.M) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const int n = ch * 16 + c;
+                            if (n < n_here)
+                                a.h_out[(int64_t)(base + n) * a.ldh + i] =
+                                    f2bf16(silu(__uint_as_float(d0[c])) * __uint_as_float(d1[c]));
+                        }
+                    }
+                } else if (mode == kDown) {
+                    const int o0 = p.mt * 2 * kBM + row;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int n = ch * 16 + c;
+                        if (n < n_here) {
+                            const float wj = a.wperm ? __ldg(a.wperm + base + n) : 0.0f;
+                            float* yp = a.ypart + (int64_t)(base + n) * L.H;
+                            if (o0 < q.M) yp[o0] = wj * __uint_as_float(d0[c]);
+                            if (o0 + kBM < q.M) yp[o0 + kBM] = wj * __uint_as_float(d1[c]);
+                        }
+                    }
+                } else if (int8_mode) {
+                    const int e = p.mt * kBM + row;
+                    if (e < q.M) {
+                        const float lb = L.logit_bias ? L.logit_bias[e] : 0.0f;
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const int n = ch * 16 + c;
+                            if (n < n_here) a.logits[(int64_t)(base + n) * L.E + e] = __uint_as_float(d0[c]) + lb;
+                        }
+                    }
+                } else {
+                    const int rpa = mode == kLoraGU ? 2 * r : r;
+                    const int R = p.mt * kLoraRows + row;
+                    if (row < kLoraRows && R < q.M) {
+                        const int ad = R / rpa, d = R % rpa;
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const int n = ch * 16 + c;
+                            if (n < n_here && __ldg(&a.perm[base + n].z) == ad)
+                                a.t_out[(int64_t)(base + n) * rpa + d] = __uint_as_float(d0[c]);
+                        }
+                    }
+                }
+            }
+            // the item two later writes this buffer; its first arrival (after these reads) orders them
+            tc::tc_fence_before();
+            return true;
+        };
+
         // ------------------------------------------------------ stream
         Pos pc, pb;  // consumer, activation loader (kLB steps ahead)
         decode(blockIdx.x, pc);
@@ -578,15 +660,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         };
         if (!lora_mode) sb_next();
         LoraRegs lr;
+        // the epilogue of an item runs kAS steps after its last step, when its MMAs are done
+        bool ep_pend = false;
+        Pos ep_pos = pc;
+        uint32_t ep_seq = 0, ep_t = 0;
 
         uint32_t t = 0;        // steps consumed by this CTA
         uint32_t sseq = 0;     // weight spans consumed by this CTA
         uint32_t n_items = 0;  // items finished by this CTA
+        bool good = true;
         while (pc.item < nitems) {
             const bool wstep = pc.kt < pc.KW;
             const bool span_start = !lora_mode && wstep && pc.kt % SP == 0;
-            // the MMAs of step t-2 must be done before A stage t%2 and activation slot (t+kLB)%kRB are rewritten
-            if (t >= 2 && !tc::mbar_wait_ok(&bar_tile[(t - 2) % 4], ((t - 2) / 4) & 1u, a.status, &s_ok)) break;
+            // the MMAs of step t - kAS must be done before TMEM stage t % kAS and activation slot
+            // (t + kLB) % kRB are rewritten
+            if (t >= (uint32_t)kAS &&
+                !tc::mbar_wait_ok(&bar_tile[(t - kAS) % kTiles], ((t - kAS) / kTiles) & 1u, a.status, &s_ok)) {
+                good = false;
+                break;
+            }
             if (span_start) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -600,10 +692,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (NL > 0 && pc.kt + 1 == pc.KW) fetch_lora(pc, 0, lr);
             issue_step(t + kLB);
             tc::cp_wait<kLB>();  // this step's group (issued kLB steps ago) has landed
-            if (span_start && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) break;
+            if (span_start && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) {
+                good = false;
+                break;
+            }
 
-            unsigned char* stA = sA + (t % 2) * kAStage;
             const int kk = pc.kt % SP;  // K-step inside the span
+            const uint32_t astage = tmem + tlane + kTmemA + (t % kAS) * 64;
             if (int4_mode && wstep) {
                 // words 8kk .. 8kk+7 = 16-byte chunks 2kk, 2kk+1 of the swizzled 128-byte row
                 const unsigned char* rowp = sR + (sseq % kRS) * kRawSlot + wblk * kSpanBytes + wrow * 128;
@@ -614,131 +709,74 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const __nv_bfloat162 ba = bf16x2_of(pick4(b_cur, ga >> 1) >> (16 * (ga & 1)));
                 const __nv_bfloat162 sb = bf16x2_of(pick4(s_cur, gb >> 1) >> (16 * (gb & 1)));
                 const __nv_bfloat162 bb = bf16x2_of(pick4(b_cur, gb >> 1) >> (16 * (gb & 1)));
-                unsigned char* arow = stA + wblk * (kBM * 128);
-                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 0)) = dequant8(wa.x, sa, ba);
-                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 1)) = dequant8(wa.y, sa, ba);
-                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 2)) = dequant8(wa.z, sa, ba);
-                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 3)) = dequant8(wa.w, sa, ba);
-                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 4)) = dequant8(wb.x, sb, bb);
-                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 5)) = dequant8(wb.y, sb, bb);
-                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 6)) = dequant8(wb.z, sb, bb);
-                *reinterpret_cast<uint4*>(arow + tc::sw128_off(wrow, 7)) = dequant8(wb.w, sb, bb);
+                // word j = K elements 8j .. 8j+7 = TMEM columns 4j .. 4j+3 of this block
+                const uint32_t ta = astage + wblk * 32;
+                uint4 o0 = dequant8(wa.x, sa, ba), o1 = dequant8(wa.y, sa, ba);
+                tc::tmem_st8(ta + 0, o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w);
+                o0 = dequant8(wa.z, sa, ba), o1 = dequant8(wa.w, sa, ba);
+                tc::tmem_st8(ta + 8, o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w);
+                o0 = dequant8(wb.x, sb, bb), o1 = dequant8(wb.y, sb, bb);
+                tc::tmem_st8(ta + 16, o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w);
+                o0 = dequant8(wb.z, sb, bb), o1 = dequant8(wb.w, sb, bb);
+                tc::tmem_st8(ta + 24, o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w);
+                tc::tmem_wait_st();
             } else if (int4_mode) {
                 stage_lora(lr, sB + (t % kRB) * kBBytes);
                 if (pc.kt + 1 < pc.KT) fetch_lora(pc, pc.kt + 1 - pc.KW, lr);
             } else if (int8_mode) {
-                // half wh of this K-step's 16 words: chunks 4kk + 2wh, 4kk + 2wh + 1 of the row
+                // half wh of this K-step's 16 words: chunks 4kk + 2wh, 4kk + 2wh + 1 of the row;
+                // K elements 32 wh .. +31 = TMEM columns 16 wh .. +15 of the hi and lo blocks
                 const unsigned char* rowp = sR + (sseq % kRS) * kRawSlot + wrow * 128;
                 const int gg = (kk * 64 + wh * 32) >> gshift;
                 const float s = bf16f((uint16_t)(pick4(s_cur, gg >> 1) >> (16 * (gg & 1))));
                 const float b = bf16f((uint16_t)(pick4(b_cur, gg >> 1) >> (16 * (gg & 1))));
+                uint32_t hv[16], lv[16];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + (((4 * kk + 2 * wh + h) ^ (wrow & 7)) << 4));
-                    uint4 hi, lo;
-                    dequant8_hilo(w4.x, w4.y, s, b, hi, lo);  // output chunk 4 wh + 2h
-                    uint32_t off = tc::sw128_off(wrow, 4 * wh + 2 * h);
-                    *reinterpret_cast<uint4*>(stA + off) = hi;
-                    *reinterpret_cast<uint4*>(stA + kBM * 128 + off) = lo;
-                    dequant8_hilo(w4.z, w4.w, s, b, hi, lo);  // output chunk 4 wh + 2h + 1
-                    off = tc::sw128_off(wrow, 4 * wh + 2 * h + 1);
-                    *reinterpret_cast<uint4*>(stA + off) = hi;
-                    *reinterpret_cast<uint4*>(stA + kBM * 128 + off) = lo;
+                    dequant8_hilo(w4.x, w4.y, s, b, hv + 8 * h, lv + 8 * h);
+                    dequant8_hilo(w4.z, w4.w, s, b, hv + 8 * h + 4, lv + 8 * h + 4);
                 }
-            } else {
-                const unsigned char* raw = sR + (t % kRB) * kLoraSlot;
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int row = brow + 32 * j;
-                    *reinterpret_cast<uint4*>(stA + tc::sw128_off(row, bch)) =
-                        *reinterpret_cast<const uint4*>(raw + row * 128 + bch * 16);
-                }
+                tc::tmem_st16(astage + 16 * wh, hv);
+                tc::tmem_st16(astage + 32 + 16 * wh, lv);
+                tc::tmem_wait_st();
             }
-            // hand the stage to the MMA warp: generic writes (and this thread's landed
-            // cp.async data) made visible to the tensor core, then one arrival per warp
+            // hand the step to the MMA warp: shared-memory operands (this thread's landed
+            // cp.async data and generic writes) made visible to the tensor core, TMEM stores
+            // complete, then one arrival per warp
             tc::fence_async_smem();
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                tc::mbar_arrive(&bar_full[t % 2]);
+                tc::mbar_arrive(&bar_full[t % kAS]);
                 if (!lora_mode && (!wstep || kk == SP - 1 || pc.kt == pc.KW - 1)) tc::mbar_arrive(&bar_rawfree[sseq % kRS]);
             }
             ++t;
 
-            if (pc.kt == pc.KT - 1) {
-                // ---------------------------------------------------- epilogue
-                if (!tc::mbar_wait_ok(&bar_acc, n_items & 1u, a.status, &s_ok)) break;
-                ++n_items;
-                tc::tc_fence_after();
-                const Geo q = geo_of(a, pc.g, s_goff[pc.g + 1] - s_goff[pc.g]);
-                const int n_here = tile_jobs(pc);
-                const int base = s_goff[pc.g] + pc.nt * kNT;
-                const int quarter = warp % 4;         // TMEM lane quarter of this warp
-                const int row = quarter * 32 + lane;  // TMEM lane of this thread
-                for (int ch = warp / 4; ch * 16 < n_here; ch += 2) {  // 16-column chunks
-                    uint32_t d0[16], d1[16];
-                    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ch * 16;
-                    tc::tmem_ld16(taddr, d0);
-                    if (int4_mode) tc::tmem_ld16(taddr + 256, d1);
-                    tc::tmem_wait_ld();
-                    if (mode == kGU) {
-                        const int i = pc.mt * kBM + row;
-                        if (i < q.M) {
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                const int n = ch * 16 + c;
-                                if (n < n_here)
-                                    a.h_out[(int64_t)(base + n) * a.ldh + i] =
-                                        f2bf16(silu(__uint_as_float(d0[c])) * __uint_as_float(d1[c]));
-                            }
-                        }
-                    } else if (mode == kDown) {
-                        const int o0 = pc.mt * 2 * kBM + row;
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const int n = ch * 16 + c;
-                            if (n < n_here) {
-                                const float wj = a.wperm ? __ldg(a.wperm + base + n) : 0.0f;
-                                float* yp = a.ypart + (int64_t)(base + n) * L.H;
-                                if (o0 < q.M) yp[o0] = wj * __uint_as_float(d0[c]);
-                                if (o0 + kBM < q.M) yp[o0 + kBM] = wj * __uint_as_float(d1[c]);
-                            }
-                        }
-                    } else if (int8_mode) {
-                        const int e = pc.mt * kBM + row;
-                        if (e < q.M) {
-                            const float lb = L.logit_bias ? L.logit_bias[e] : 0.0f;
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                const int n = ch * 16 + c;
-                                if (n < n_here) a.logits[(int64_t)(base + n) * L.E + e] = __uint_as_float(d0[c]) + lb;
-                            }
-                        }
-                    } else {
-                        const int rpa = mode == kLoraGU ? 2 * r : r;
-                        const int R = pc.mt * kLoraRows + row;
-                        if (row < kLoraRows && R < q.M) {
-                            const int ad = R / rpa, d = R % rpa;
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                const int n = ch * 16 + c;
-                                if (n < n_here && __ldg(&a.perm[base + n].z) == ad)
-                                    a.t_out[(int64_t)(base + n) * rpa + d] = __uint_as_float(d0[c]);
-                            }
-                        }
-                    }
+            if (pc.kt == pc.KT - 1) {  // this step ends an item: its epilogue is deferred
+                if (ep_pend && !epilogue(ep_pos, ep_seq)) {
+                    good = false;
+                    break;
                 }
-                // the next item's first MMA overwrites the accumulators: its stage arrival
-                // (after these reads) orders them
-                tc::tc_fence_before();
+                ep_pend = true;
+                ep_pos = pc;
+                ep_seq = n_items++;
+                ep_t = t;
+            } else if (ep_pend && t >= ep_t + kAS) {
+                ep_pend = false;
+                if (!epilogue(ep_pos, ep_seq)) {
+                    good = false;
+                    break;
+                }
             }
             // advance the consumer
             if (++pc.kt == pc.KT) decode(pc.item + NB, pc);
             if (!lora_mode && pc.item < nitems && (pc.kt >= pc.KW || pc.kt % SP == 0)) ++sseq;  // next step opens a span
         }
+        if (good && ep_pend && !epilogue(ep_pos, ep_seq)) good = false;
         // no cp.async may still target this CTA's shared memory at exit
         tc::cp_wait<0>();
-        if (pc.item < nitems) s_ok = 0;  // left early: let the producer stop waiting
+        if (!good) s_ok = 0;  // left early: let the producer stop waiting
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -779,16 +817,27 @@ bool words_tma_ok(const moe_qtensor& q) {
            ((uintptr_t)q.biases & 3) == 0;
 }
 
-cudaError_t launch_kernel(TcArgs& a, cudaStream_t s) {
+template <int kMode>
+cudaError_t launch_mode(TcArgs& a, int nsm, cudaStream_t s) {
     static int cached = 0;
-    const size_t smem = 2 * kAStage + kRB * kBBytes + kRS * kRawSlot + 1024;
-    cudaError_t e = ensure_smem((const void*)tc_gemm_kernel, smem, cached);
+    const size_t smem = kRB * kBBytes + kRS * kRawSlot + 1024;
+    cudaError_t e = ensure_smem((const void*)tc_gemm_kernel<kMode>, smem, cached);
     if (e != cudaSuccess) return e;
+    tc_gemm_kernel<kMode><<<nsm, kTcThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kernel(TcArgs& a, cudaStream_t s) {
     int nsm = 0, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    tc_gemm_kernel<<<nsm, kTcThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    switch (a.mode) {
+        case kGU: return launch_mode<kGU>(a, nsm, s);
+        case kDown: return launch_mode<kDown>(a, nsm, s);
+        case kLoraGU: return launch_mode<kLoraGU>(a, nsm, s);
+        case kLoraDown: return launch_mode<kLoraDown>(a, nsm, s);
+        default: return launch_mode<kRouterMode>(a, nsm, s);
+    }
 }
 
 }  // namespace
