@@ -56,21 +56,23 @@ constexpr int kDeqWarps = 8;                      // dequantisation warps
 constexpr int kTcThreads = (kDeqWarps + 1) * 32;  // + the producer warp (TMA, LoRA-B rows, MMA issue)
 constexpr int kBM = 128;                          // rows per MMA block
 constexpr int kNT = 64;                           // jobs per tile (MMA N <= 64)
-constexpr int kAS = 4;                            // A stages in TMEM (dequantisation runs up to kAS steps ahead)
-constexpr int kLB = 4;                            // activation lookahead (K-steps)
+constexpr int kKS = 128;                          // K per pipeline step (two 64-wide operand sub-tiles)
+constexpr int kAS = 2;                            // A stages in TMEM (dequantisation runs up to kAS steps ahead)
+constexpr int kLB = 2;                            // activation lookahead (steps)
 constexpr int kRB = kLB + kAS;                    // activation ring: slot of step t - kAS is free at step t
-constexpr int kRS = 4;                            // weight span ring (three spans in flight)
+constexpr int kRS = 4;                            // weight span ring (two spans in flight)
 constexpr int kTiles = 8;                         // per-step MMA completion barriers
 constexpr int kSpanBytes = kBM * 128;             // one block of one span: 128 rows x 128 B
 constexpr int kRawSlot = 2 * kSpanBytes;          // two blocks
-constexpr int kBBytes = kNT * 128;                // 64 rows x 128 B
+constexpr int kSub = kNT * 128;                   // one 64-wide K sub-tile of 64 rows (128 B per row)
+constexpr int kBSlot = 2 * kSub;                  // activation ring slot: the step's two sub-tiles
 constexpr int kLoraRows = 64;                     // real LoRA-A rows per M tile
-constexpr int kLoraSlot = kLoraRows * 128;
+constexpr int kLoraSlot = 2 * kLoraRows * 128;    // LoRA-A ring slot: two sub-tiles of 64 rows
 constexpr int kMaxGroups = MOEQ_MAX_EXPERTS + 1;
-// TMEM columns: accumulator D(buffer b, block k) at 128 b + 64 k; A stage s, block k at 256 + 64 s + 32 k
+// TMEM columns: accumulator D(buffer b, block k) at 128 b + 64 k; A stage s, block k at 256 + 128 s + 64 k
 constexpr uint32_t kTmemA = 256;
 static_assert(kRB * kLoraSlot <= kRS * kRawSlot, "LoRA-A ring must fit in the weight ring");
-static_assert(kTmemA + kAS * 64 <= 512, "TMEM columns");
+static_assert(kTmemA + kAS * 128 <= 512, "TMEM columns");
 
 enum Mode { kGU = 0, kDown = 1, kLoraGU = 2, kLoraDown = 3, kRouterMode = 4 };
 
@@ -102,15 +104,15 @@ __device__ __forceinline__ int rows_per_item(int mode) {
     return mode == kDown ? 2 * kBM : (mode == kLoraGU || mode == kLoraDown) ? kLoraRows : kBM;
 }
 
-__device__ __forceinline__ Geo geo_of(const TcArgs& a, int g, int count) {
+__device__ __forceinline__ Geo geo_of(const TcArgs& a, int mode, int g, int count) {
     const LayerArgs& L = a.L;
     Geo q;
-    q.shared = a.mode != kRouterMode && g == L.E;
+    q.shared = mode != kRouterMode && g == L.E;
     q.skip = count == 0 || (q.shared && !L.has_shared);
     q.mat = q.shared ? 0 : g;
     const int I = q.shared ? L.Is : L.I;
     const int r = L.rank;
-    switch (a.mode) {
+    switch (mode) {
         case kGU: q.M = I; q.K = L.H; break;
         case kDown: q.M = L.H; q.K = I; break;
         case kLoraGU: q.M = L.n_adapters * 2 * r; q.K = L.H; break;
@@ -118,18 +120,10 @@ __device__ __forceinline__ Geo geo_of(const TcArgs& a, int g, int count) {
         default: q.M = L.E; q.K = L.H; q.mat = 0; break;
     }
     if (q.M <= 0) q.skip = true;
-    const int rpi = rows_per_item(a.mode);
+    const int rpi = rows_per_item(mode);
     q.mtiles = q.skip ? 0 : (q.M + rpi - 1) / rpi;
     q.ntiles = q.skip ? 0 : (count + kNT - 1) / kNT;
     return q;
-}
-
-// LoRA-B K-steps appended to each gate/up or down item (K' = adapters x r per matrix)
-__device__ __forceinline__ int lora_steps(const TcArgs& a) {
-    const LayerArgs& L = a.L;
-    if ((a.mode != kGU && a.mode != kDown) || L.rank <= 0 || L.n_adapters <= 0) return 0;
-    const int kp = (a.mode == kGU ? 2 : 1) * L.n_adapters * L.rank;
-    return (kp + 63) / 64;
 }
 
 // Position in this CTA's stream of (item, k-step) tiles.
@@ -186,26 +180,27 @@ __device__ __forceinline__ void dequant8_hilo(uint32_t w0, uint32_t w1, float s,
 __device__ __forceinline__ uint32_t pick4(const uint32_t (&v)[4], int i) {
     return i == 0 ? v[0] : i == 1 ? v[1] : i == 2 ? v[2] : v[3];
 }
-
-__device__ __forceinline__ __nv_bfloat162 bf16x2_of(uint32_t half_word) {
-    return __bfloat162bfloat162(__ushort_as_bfloat16((unsigned short)(half_word & 0xFFFFu)));
+// bf16 number g (0..7) of four words of bf16 pairs
+__device__ __forceinline__ uint32_t bf16_at(const uint32_t (&v)[4], int g) {
+    return (pick4(v, g >> 1) >> (16 * (g & 1))) & 0xFFFFu;
+}
+__device__ __forceinline__ __nv_bfloat162 bf16x2_of(uint32_t h) {
+    return __bfloat162bfloat162(__ushort_as_bfloat16((unsigned short)h));
 }
 
-// This thread's activation chunks (and LoRA-A chunks) of one item.
+// This thread's activation rows (and LoRA-A rows) of one item.
 struct BCtx {
     const uint16_t* src[2];
-    const uint16_t* la[2];  // LoRA-A modes: bf16 A chunks (NULL: zero fill)
+    const uint16_t* la[2];  // LoRA-A modes: bf16 A rows (NULL: zero fill)
     bool live[2];
 };
 
-// LoRA-B operand B of one step, fetched a step ahead.
+// LoRA-B operand B of one step, fetched a step ahead: rows brow, brow + 32; chunk bch; sub-tiles 0, 1
 struct LoraRegs {
-    float4 t[2][2];  // LoRA-A products of this thread's two (job, chunk) pairs, unscaled
-    bool t_live[2];
+    float4 t[2][2][2];  // [row][sub-tile][half], unscaled LoRA-A products
+    uint32_t live;      // bit (2 row + sub)
 };
 
-// One instantiation per mode, so that each kernel holds only its own path (a
-// loop body small enough for the instruction caches).
 template <int kMode>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ __align__(1024) unsigned char tsm_raw[];
@@ -218,18 +213,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     constexpr bool lora_mode = mode == kLoraGU || mode == kLoraDown;
     constexpr bool int8_mode = mode == kRouterMode;
     constexpr bool int4_mode = mode == kGU || mode == kDown;
-    constexpr int SP = int8_mode ? 2 : 4;  // K-steps per weight span (128 B of words per row)
+    constexpr int SP = int8_mode ? 1 : 2;  // steps per weight span (128 B of words per row)
     const int r = L.rank;
-    const int NL = lora_steps(a);
+    const int nar = L.n_adapters * r;   // LoRA-B K' per matrix
+    const int NL = (int4_mode && r > 0 && L.n_adapters > 0) ? (nar + 63) / 64 : 0;
 
-    // shared memory: [activation ring kRB x 8 KB][weight ring kRS x 32 KB]
+    // shared memory: [activation ring kRB x 16 KB][weight ring kRS x 32 KB]
     unsigned char* sB = tsm;
-    unsigned char* sR = sB + kRB * kBBytes;
+    unsigned char* sR = sB + kRB * kBSlot;
     __shared__ uint64_t bar_full[kAS];    // step's operands written: one arrival per dequant warp
     __shared__ uint64_t bar_tile[kTiles]; // MMAs of a step done (tcgen05.commit)
     __shared__ uint64_t bar_acc[2];       // MMAs of an item done, per accumulator buffer
     __shared__ uint64_t bar_raw[kRS];     // span landed: 32 producer-lane arrivals (+ TMA transaction count)
-    __shared__ uint64_t bar_rawfree[kRS]; // span consumed: one arrival per dequant warp + the producer's commit
+    __shared__ uint64_t bar_rawfree[kRS]; // span consumed: one arrival per dequant warp
     __shared__ uint32_t s_tmem;
     __shared__ int s_items[kMaxGroups + 1];
     __shared__ int s_goff[kMaxGroups + 1];
@@ -254,7 +250,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         for (int i = 0; i < kTiles; ++i) tc::mbar_init(&bar_tile[i], 1);
         for (int i = 0; i < kRS; ++i) {
             tc::mbar_init(&bar_raw[i], 32);
-            tc::mbar_init(&bar_rawfree[i], kDeqWarps + 1);
+            tc::mbar_init(&bar_rawfree[i], kDeqWarps);
         }
         tc::mbar_init(&bar_acc[0], 1);
         tc::mbar_init(&bar_acc[1], 1);
@@ -269,7 +265,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         int acc = 0;
         for (int g = 0; g < ngroups; ++g) {
             s_items[g] = acc;
-            const Geo q = geo_of(a, g, s_goff[g + 1] - s_goff[g]);
+            const Geo q = geo_of(a, mode, g, s_goff[g + 1] - s_goff[g]);
             acc += q.mtiles * q.ntiles;
         }
         s_items[ngroups] = acc;
@@ -292,18 +288,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (s_items[mid] <= item) lo = mid;
             else hi = mid - 1;
         }
-        const Geo q = geo_of(a, lo, s_goff[lo + 1] - s_goff[lo]);
+        const Geo q = geo_of(a, mode, lo, s_goff[lo + 1] - s_goff[lo]);
         const int rem = item - s_items[lo];
         p.g = lo;
         p.mt = rem / q.ntiles;
         p.nt = rem % q.ntiles;
-        p.KW = q.K / 64;
+        p.KW = q.K / kKS;
         p.KT = p.KW + NL;
     };
     auto tile_jobs = [&](const Pos& p) { return min(kNT, s_goff[p.g + 1] - s_goff[p.g] - p.nt * kNT); };
-    const int nar = L.n_adapters * r;
+    auto geo = [&](const Pos& p) { return geo_of(a, mode, p.g, s_goff[p.g + 1] - s_goff[p.g]); };
     // spans of an item in the weight ring: its weight spans, then one per LoRA-B step
-    auto wspans = [&](const Pos& p) { return (p.KW + SP - 1) / SP; };
+    auto nspans = [&](const Pos& p) { return (p.KW + SP - 1) / SP + NL; };
 
     if (warp == kDeqWarps) {
         // ====================================================== producer warp: TMA, LoRA-B rows, MMA issue
@@ -312,20 +308,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         Pos pt = pc;  // item of the next span to load
         int pt_span = 0;
         uint32_t issued = 0;  // spans issued
+        int slot_mma[kRS];    // step whose MMAs read the slot directly (LoRA-B rows), or -1
+        for (int i = 0; i < kRS; ++i) slot_mma[i] = -1;
         bool ok = true;
-        // LoRA-B rows of step s into slot: lane -> chunk lane % 8 of rows lane / 8 + 4 i
+        // LoRA-B rows of step s into slot: lane -> chunk lane % 8 of rows lane / 8 + 4 i;
+        // K' column 64 s + 8 c + e of block k = adapter (.. / r), rank index (.. % r) of its matrix
         auto lora_span = [&](const Pos& p, int s, int slot) {
-            const Geo q = geo_of(a, p.g, s_goff[p.g + 1] - s_goff[p.g]);
+            const Geo q = geo(p);
             const uint32_t dst0 = tc::smem_u32(sR + slot * kRawSlot);
-            const int c = lane % 8, cp = 64 * s + 8 * c;
+            const int c = lane % 8, cc = 64 * s + 8 * c;
             for (int blk = 0; blk < 2; ++blk) {
-                int part = 0, cc = cp;
-                if (mode == kGU) {
-                    part = cp < nar ? 0 : 1;
-                    cc = cp - part * nar;
-                }
-                const bool mine = mode == kGU ? part == blk : true;  // gate rows take gate columns only
-                const moe_lora_proj* lp = (mine && cc < nar) ? tlora(L, cc / r, q.shared, mode == kGU ? part : 2) : nullptr;
+                const int which = mode == kGU ? blk : 2;  // gate rows | up rows; down: two row blocks
+                const moe_lora_proj* lp = cc < nar ? tlora(L, cc / r, q.shared, which) : nullptr;
                 const int row0 = mode == kGU ? p.mt * kBM : p.mt * 2 * kBM + blk * kBM;
                 const uint16_t* src = lp ? lp->B + ((int64_t)q.mat * q.M + row0) * r + cc % r : a.act;
                 for (int i = 0; i < kBM / 4; ++i) {
@@ -343,15 +337,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (pt.item >= nitems || !ok) return;
             const uint32_t seq = issued;
             const int slot = seq % kRS;
-            if (seq >= (uint32_t)kRS && !tc::mbar_wait_ok(&bar_rawfree[slot], ((seq / kRS) - 1) & 1u, a.status, &s_ok)) {
-                ok = false;
-                return;
+            if (seq >= (uint32_t)kRS) {
+                if (!tc::mbar_wait_ok(&bar_rawfree[slot], ((seq / kRS) - 1) & 1u, a.status, &s_ok)) {
+                    ok = false;
+                    return;
+                }
+                const int tr = slot_mma[slot];
+                if (tr >= 0 && !tc::mbar_wait_ok(&bar_tile[tr % kTiles], (tr / kTiles) & 1u, a.status, &s_ok)) {
+                    ok = false;
+                    return;
+                }
+                slot_mma[slot] = -1;
             }
-            const int nw = wspans(pt);
+            const int nw = (pt.KW + SP - 1) / SP;
             if (pt_span < nw) {
                 uint64_t* bar = &bar_raw[slot];
                 if (lane == 0) {
-                    const Geo q = geo_of(a, pt.g, s_goff[pt.g + 1] - s_goff[pt.g]);
+                    const Geo q = geo(pt);
                     const uint32_t dst = tc::smem_u32(sR + slot * kRawSlot);
                     const int x = pt_span * 32;  // 32 words = 128 B per row
                     if (mode == kGU) {
@@ -375,18 +377,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 lora_span(pt, pt_span - nw, slot);
             }
             ++issued;
-            if (++pt_span >= nw + NL) {
+            if (++pt_span >= nspans(pt)) {
                 decode(pt.item + NB, pt);
                 pt_span = 0;
             }
         };
-        if (!lora_mode)
-            for (int i = 0; i < kRS - 1; ++i) span_next();
+        if (!lora_mode) {
+            span_next();
+            span_next();
+        }
         uint32_t t = 0, cs = 0, ib = 0;  // steps, spans and items consumed
         while (pc.item < nitems && ok) {
             const bool wstep = pc.kt < pc.KW;
-            const bool opens = !lora_mode && (!wstep || pc.kt % SP == 0);
-            if (opens) span_next();  // keep kRS - 1 spans ahead
+            // a step that opens a span keeps the ring two spans ahead
+            if (!lora_mode && (!wstep || pc.kt % SP == 0)) span_next();
             if (!ok || !tc::mbar_wait_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok)) {
                 ok = false;
                 break;
@@ -398,33 +402,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
             tc::tc_fence_after();
             if (lane == 0) {
-                const int Nmma = (tile_jobs(pc) + 15) / 16 * 16;
-                const uint32_t idesc = tc::idesc_bf16(kBM, Nmma);
-                const uint64_t bd = tc::sdesc_k_sw128(tc::smem_u32(sB + (t % kRB) * kBBytes));
+                const uint32_t idesc = tc::idesc_bf16(kBM, (tile_jobs(pc) + 15) / 16 * 16);
+                const uint32_t bslot = tc::smem_u32(sB + (t % kRB) * kBSlot);
                 const uint32_t dacc = tmem + (ib & 1u) * 128u;
                 if (lora_mode) {  // A: the LoRA-A rows, copied swizzled into the ring
-                    const uint64_t ad = tc::sdesc_k_sw128(tc::smem_u32(sR + (t % kRB) * kLoraSlot));
-                    for (int k = 0; k < 4; ++k) tc::mma_bf16(dacc, ad + 2 * k, bd + 2 * k, idesc, (pc.kt > 0 || k > 0) ? 1u : 0u);
+                    const uint32_t aslot = tc::smem_u32(sR + (t % kRB) * kLoraSlot);
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const uint64_t ad = tc::sdesc_k_sw128(aslot + sub * (kLoraRows * 128));
+                        const uint64_t bd = tc::sdesc_k_sw128(bslot + sub * kSub);
+                        for (int k = 0; k < 4; ++k)
+                            tc::mma_bf16(dacc, ad + 2 * k, bd + 2 * k, idesc, (pc.kt > 0 || sub > 0 || k > 0) ? 1u : 0u);
+                    }
                 } else if (!wstep) {  // LoRA-B step: A = LoRA-B rows of the pseudo-span, one accumulator per block
+                    const uint32_t rs = tc::smem_u32(sR + (cs % kRS) * kRawSlot);
                     for (int blk = 0; blk < 2; ++blk) {
-                        const uint64_t ad = tc::sdesc_k_sw128(tc::smem_u32(sR + (cs % kRS) * kRawSlot + blk * kSpanBytes));
+                        const uint64_t ad = tc::sdesc_k_sw128(rs + blk * kSpanBytes);
+                        const uint64_t bd = tc::sdesc_k_sw128(bslot + (mode == kGU ? blk : 0) * kSub);
                         for (int k = 0; k < 4; ++k) tc::mma_bf16(dacc + blk * 64, ad + 2 * k, bd + 2 * k, idesc, 1u);
                     }
+                    slot_mma[cs % kRS] = (int)t;
                 } else {  // weight step: A = the dequantised tile in TMEM
-                    const uint32_t astage = tmem + kTmemA + (t % kAS) * 64;
+                    const uint32_t astage = tmem + kTmemA + (t % kAS) * 128;
                     for (int blk = 0; blk < 2; ++blk) {
                         // router: hi and lo parts into one accumulator; otherwise one accumulator per block
                         const uint32_t d = dacc + (int8_mode ? 0u : (uint32_t)blk * 64u);
-                        for (int k = 0; k < 4; ++k) {  // K=16 per MMA: 8 TMEM columns, +32 B in the swizzled B tile
-                            const bool first = pc.kt == 0 && k == 0 && (!int8_mode || blk == 0);
-                            tc::mma_bf16_ts(d, astage + blk * 32 + 8 * k, bd + 2 * k, idesc, first ? 0u : 1u);
+                        for (int sub = 0; sub < 2; ++sub) {
+                            const uint64_t bd = tc::sdesc_k_sw128(bslot + sub * kSub);
+                            for (int k = 0; k < 4; ++k) {  // K=16 per MMA: 8 TMEM columns, +32 B in the swizzled B tile
+                                const bool first = pc.kt == 0 && sub == 0 && k == 0 && (!int8_mode || blk == 0);
+                                tc::mma_bf16_ts(d, astage + blk * 64 + sub * 32 + 8 * k, bd + 2 * k, idesc, first ? 0u : 1u);
+                            }
                         }
                     }
                 }
                 tc::mma_commit(&bar_tile[t % kTiles]);
-                // the span's slot is free once these MMAs are done (they read it directly for LoRA-B)
-                if (!lora_mode && (!wstep || pc.kt % SP == SP - 1 || pc.kt == pc.KW - 1))
-                    tc::mma_commit(&bar_rawfree[cs % kRS]);
                 if (pc.kt == pc.KT - 1) tc::mma_commit(&bar_acc[ib & 1u]);
             }
             __syncwarp();
@@ -444,8 +455,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         __syncwarp();
     } else {
         // ====================================================== dequantisation warps
-        // ---- weight rows.  int4: thread -> (block, row), the K-step's 8 words of the row;
-        //      int8: thread -> (row, half of the K-step's 16 words).  Warp w writes TMEM
+        // ---- weight rows.  int4: thread -> (block, row): the step's 16 words of the row;
+        //      int8: thread -> (row, half of the step's 32 words).  Warp w writes TMEM
         //      lanes 32 (w % 4) .. +31, which are its rows.
         const int wrow = tid % kBM;
         const int wblk = int8_mode ? 0 : tid / kBM;
@@ -454,10 +465,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const int group = int8_mode ? L.router.group : L.gate.group;
         const int gshift = group == 64 ? 6 : 5;
         // scale/bias words (pairs of bf16) of one span of this thread's row
-        const int span_groups = (SP * 64) >> gshift;  // 2, 4 or 8
-        const int span_words = span_groups / 2;       // 1, 2 or 4
+        const int span_groups = (SP * kKS) >> gshift;  // 2, 4 or 8
+        const int span_words = span_groups / 2;        // 1, 2 or 4
         auto fetch_sb = [&](const Pos& p, int span, uint32_t (&sv)[4], uint32_t (&bv)[4]) {
-            const Geo q = geo_of(a, p.g, s_goff[p.g + 1] - s_goff[p.g]);
+            const Geo q = geo(p);
             int row;
             const moe_qtensor* W;
             if (mode == kGU) {
@@ -472,8 +483,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
             const bool ok = row < q.M;
             const int ng = q.K >> gshift;
-            const int64_t off = ((int64_t)q.mat * q.M + (ok ? row : 0)) * ng + span * span_groups;
             const int g0 = span * span_groups;
+            const int64_t off = ((int64_t)q.mat * q.M + (ok ? row : 0)) * ng + g0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const bool in = ok && j < span_words && g0 + 2 * j < ng;
@@ -482,14 +493,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
         };
 
-        // ---- activation rows (and LoRA-A rows): rows brow, brow + 32, 16-byte chunk bch
+        // ---- activation rows (and LoRA-A rows): rows brow, brow + 32; 16-byte chunk bch of both sub-tiles
         const int brow = tid / 8, bch = tid % 8;
+        const uint32_t boff0 = tc::sw128_off(brow, bch), boff1 = tc::sw128_off(brow + 32, bch);
         auto make_b = [&](const Pos& p, BCtx& c) {
-            const bool by_token = mode == kGU || mode == kLoraGU;
+            constexpr bool by_token = mode == kGU || mode == kLoraGU;
             const bool live_item = p.item < nitems;
             const int base = live_item ? s_goff[p.g] + p.nt * kNT : 0;
             const int end = live_item ? s_goff[p.g + 1] : 0;
-            const Geo q = geo_of(a, p.g, end - base + p.nt * kNT);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int job = base + brow + 32 * j;
@@ -497,8 +508,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const int64_t rowi = c.live[j] ? (by_token ? a.perm[job].x : job) : 0;
                 c.src[j] = a.act + rowi * a.ld_act + bch * 8;
                 c.la[j] = nullptr;
-                if (lora_mode && live_item) {
-                    const int rpa = mode == kLoraGU ? 2 * r : r;
+            }
+            if (lora_mode && live_item) {
+                const Geo q = geo(p);
+                const int rpa = mode == kLoraGU ? 2 * r : r;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
                     const int R = p.mt * kLoraRows + brow + 32 * j;
                     if (R < q.M) {
                         const int ad = R / rpa, d = R % rpa;
@@ -510,64 +525,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
         };
         auto issue_b = [&](const BCtx& c, int kt, int slot) {
-            const uint32_t base = tc::smem_u32(sB + slot * kBBytes);
-            const uint32_t rb = tc::smem_u32(sR + slot * kLoraSlot);
+            const uint32_t base = tc::smem_u32(sB + slot * kBSlot);
+            const int k0 = kt * kKS;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int row = brow + 32 * j;
-                tc::cp16(base + tc::sw128_off(row, bch), c.src[j] + (c.live[j] ? kt * 64 : 0), c.live[j] ? 16u : 0u);
-                if (lora_mode)  // LoRA-A rows straight into the MMA's swizzled operand layout
-                    tc::cp16(rb + tc::sw128_off(row, bch), c.la[j] ? c.la[j] + kt * 64 : a.act, c.la[j] ? 16u : 0u);
+            for (int sub = 0; sub < 2; ++sub) {
+                const int ko = k0 + 64 * sub;
+                tc::cp16(base + sub * kSub + boff0, c.src[0] + (c.live[0] ? ko : 0), c.live[0] ? 16u : 0u);
+                tc::cp16(base + sub * kSub + boff1, c.src[1] + (c.live[1] ? ko : 0), c.live[1] ? 16u : 0u);
+            }
+            if (lora_mode) {  // LoRA-A rows straight into the MMA's swizzled operand layout
+                const uint32_t rb = tc::smem_u32(sR + slot * kLoraSlot);
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                    const int ko = k0 + 64 * sub;
+                    tc::cp16(rb + sub * (kLoraRows * 128) + boff0, c.la[0] ? c.la[0] + ko : a.act, c.la[0] ? 16u : 0u);
+                    tc::cp16(rb + sub * (kLoraRows * 128) + boff1, c.la[1] ? c.la[1] + ko : a.act, c.la[1] ? 16u : 0u);
+                }
             }
         };
 
-        // ---- LoRA-B operand B: thread holds (job row, chunk) = (brow, bch) and (brow + 32, bch).
-        // K' column c' of step s is 64 s + 8 chunk + e; gate/up: [gate adapters | up adapters].
+        // ---- LoRA-B operand B of step s: sub-tile k holds, for block k's matrix (gate/up: gate, up;
+        // down: down in sub-tile 0), each job's scaled LoRA-A products in its adapter's K' columns
         auto fetch_lora = [&](const Pos& p, int s, LoraRegs& R) {
-            const Geo q = geo_of(a, p.g, s_goff[p.g + 1] - s_goff[p.g]);
+            const Geo q = geo(p);
             const int base = s_goff[p.g] + p.nt * kNT, end = s_goff[p.g + 1];
-            const int cp = 64 * s + 8 * bch;
-            const int part = (mode == kGU && cp >= nar) ? 1 : 0;
-            const int cc = cp - part * nar;
+            const int cc = 64 * s + 8 * bch;
+            const int tw = mode == kGU ? 2 * r : r;
+            R.live = 0;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int job = base + brow + 32 * j;
-                R.t_live[j] = false;
-                if (job < end && cc < nar) {
-                    const int ad = a.perm[job].z;
-                    if (ad == cc / r && tlora(L, ad, q.shared, mode == kGU ? part : 2)) {
-                        const int tw = mode == kGU ? 2 * r : r;
-                        const float4* tp =
-                            reinterpret_cast<const float4*>(a.t_in + (int64_t)job * tw + part * r + cc % r);
-                        R.t[j][0] = tp[0];
-                        R.t[j][1] = tp[1];
-                        R.t_live[j] = true;
-                    }
+                if (job >= end || cc >= nar) continue;
+                const int ad = a.perm[job].z;
+                if (ad != cc / r) continue;
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                    if (mode == kDown && sub == 1) continue;
+                    if (!tlora(L, ad, q.shared, mode == kGU ? sub : 2)) continue;
+                    const float4* tp = reinterpret_cast<const float4*>(a.t_in + (int64_t)job * tw + sub * r + cc % r);
+                    R.t[j][sub][0] = tp[0];
+                    R.t[j][sub][1] = tp[1];
+                    R.live |= 1u << (2 * j + sub);
                 }
             }
         };
-        auto stage_lora = [&](const LoraRegs& R, unsigned char* sBslot) {
+        auto stage_lora = [&](const LoraRegs& R, unsigned char* bslot) {
             const float sc = L.scale;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                uint4 o = make_uint4(0, 0, 0, 0);
-                if (R.t_live[j]) {
-                    const __nv_bfloat162 p0 = __floats2bfloat162_rn(sc * R.t[j][0].x, sc * R.t[j][0].y);
-                    const __nv_bfloat162 p1 = __floats2bfloat162_rn(sc * R.t[j][0].z, sc * R.t[j][0].w);
-                    const __nv_bfloat162 p2 = __floats2bfloat162_rn(sc * R.t[j][1].x, sc * R.t[j][1].y);
-                    const __nv_bfloat162 p3 = __floats2bfloat162_rn(sc * R.t[j][1].z, sc * R.t[j][1].w);
-                    o = make_uint4(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1),
-                                   *reinterpret_cast<const uint32_t*>(&p2), *reinterpret_cast<const uint32_t*>(&p3));
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                    if (mode == kDown && sub == 1) continue;
+                    uint4 o = make_uint4(0, 0, 0, 0);
+                    if (R.live & (1u << (2 * j + sub))) {
+                        const float4 u = R.t[j][sub][0], v = R.t[j][sub][1];
+                        const __nv_bfloat162 p0 = __floats2bfloat162_rn(sc * u.x, sc * u.y);
+                        const __nv_bfloat162 p1 = __floats2bfloat162_rn(sc * u.z, sc * u.w);
+                        const __nv_bfloat162 p2 = __floats2bfloat162_rn(sc * v.x, sc * v.y);
+                        const __nv_bfloat162 p3 = __floats2bfloat162_rn(sc * v.z, sc * v.w);
+                        o = make_uint4(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1),
+                                       *reinterpret_cast<const uint32_t*>(&p2), *reinterpret_cast<const uint32_t*>(&p3));
+                    }
+                    *reinterpret_cast<uint4*>(bslot + sub * kSub + (j ? boff1 : boff0)) = o;
                 }
-                *reinterpret_cast<uint4*>(sBslot + tc::sw128_off(brow + 32 * j, bch)) = o;
-            }
         };
 
         // ---- epilogue of a finished item (accumulator buffer seq % 2)
         auto epilogue = [&](const Pos& p, uint32_t seq) -> bool {
             if (!tc::mbar_wait_ok(&bar_acc[seq & 1u], (seq >> 1) & 1u, a.status, &s_ok)) return false;
             tc::tc_fence_after();
-            const Geo q = geo_of(a, p.g, s_goff[p.g + 1] - s_goff[p.g]);
+            const Geo q = geo(p);
             const int n_here = tile_jobs(p);
             const int base = s_goff[p.g] + p.nt * kNT;
             const uint32_t dacc = tmem + tlane + (seq & 1u) * 128u;
@@ -697,48 +724,49 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 break;
             }
 
-            const int kk = pc.kt % SP;  // K-step inside the span
-            const uint32_t astage = tmem + tlane + kTmemA + (t % kAS) * 64;
+            const int kk = pc.kt % SP;  // step inside the span
+            const uint32_t astage = tmem + tlane + kTmemA + (t % kAS) * 128;
             if (int4_mode && wstep) {
-                // words 8kk .. 8kk+7 = 16-byte chunks 2kk, 2kk+1 of the swizzled 128-byte row
+                // the step's 16 words = 16-byte chunks 4kk .. 4kk+3 of the swizzled 128-byte row;
+                // word w = K elements 8w .. 8w+7 = TMEM columns 4w .. 4w+3 of this block
                 const unsigned char* rowp = sR + (sseq % kRS) * kRawSlot + wblk * kSpanBytes + wrow * 128;
-                const uint4 wa = *reinterpret_cast<const uint4*>(rowp + (((2 * kk) ^ (wrow & 7)) << 4));
-                const uint4 wb = *reinterpret_cast<const uint4*>(rowp + (((2 * kk + 1) ^ (wrow & 7)) << 4));
-                const int ga = (kk * 64) >> gshift, gb = (kk * 64 + 32) >> gshift;  // groups of words 0-3, 4-7
-                const __nv_bfloat162 sa = bf16x2_of(pick4(s_cur, ga >> 1) >> (16 * (ga & 1)));
-                const __nv_bfloat162 ba = bf16x2_of(pick4(b_cur, ga >> 1) >> (16 * (ga & 1)));
-                const __nv_bfloat162 sb = bf16x2_of(pick4(s_cur, gb >> 1) >> (16 * (gb & 1)));
-                const __nv_bfloat162 bb = bf16x2_of(pick4(b_cur, gb >> 1) >> (16 * (gb & 1)));
-                // word j = K elements 8j .. 8j+7 = TMEM columns 4j .. 4j+3 of this block
-                const uint32_t ta = astage + wblk * 32;
-                uint4 o0 = dequant8(wa.x, sa, ba), o1 = dequant8(wa.y, sa, ba);
-                tc::tmem_st8(ta + 0, o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w);
-                o0 = dequant8(wa.z, sa, ba), o1 = dequant8(wa.w, sa, ba);
-                tc::tmem_st8(ta + 8, o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w);
-                o0 = dequant8(wb.x, sb, bb), o1 = dequant8(wb.y, sb, bb);
-                tc::tmem_st8(ta + 16, o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w);
-                o0 = dequant8(wb.z, sb, bb), o1 = dequant8(wb.w, sb, bb);
-                tc::tmem_st8(ta + 24, o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w);
+                const uint32_t ta = astage + wblk * 64;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + (((4 * kk + c) ^ (wrow & 7)) << 4));
+                    const int g = (kk * kKS + 32 * c) >> gshift;  // group of these 4 words within the span
+                    const __nv_bfloat162 s2 = bf16x2_of(bf16_at(s_cur, g)), b2 = bf16x2_of(bf16_at(b_cur, g));
+                    uint32_t v[16];
+                    const uint4 o0 = dequant8(w4.x, s2, b2), o1 = dequant8(w4.y, s2, b2);
+                    const uint4 o2 = dequant8(w4.z, s2, b2), o3 = dequant8(w4.w, s2, b2);
+                    v[0] = o0.x; v[1] = o0.y; v[2] = o0.z; v[3] = o0.w;
+                    v[4] = o1.x; v[5] = o1.y; v[6] = o1.z; v[7] = o1.w;
+                    v[8] = o2.x; v[9] = o2.y; v[10] = o2.z; v[11] = o2.w;
+                    v[12] = o3.x; v[13] = o3.y; v[14] = o3.z; v[15] = o3.w;
+                    tc::tmem_st16(ta + 16 * c, v);
+                }
                 tc::tmem_wait_st();
             } else if (int4_mode) {
-                stage_lora(lr, sB + (t % kRB) * kBBytes);
+                stage_lora(lr, sB + (t % kRB) * kBSlot);
                 if (pc.kt + 1 < pc.KT) fetch_lora(pc, pc.kt + 1 - pc.KW, lr);
             } else if (int8_mode) {
-                // half wh of this K-step's 16 words: chunks 4kk + 2wh, 4kk + 2wh + 1 of the row;
-                // K elements 32 wh .. +31 = TMEM columns 16 wh .. +15 of the hi and lo blocks
+                // half wh of the step's 32 words: chunks 4wh .. 4wh+3 of the row; K elements 64 wh .. +63
+                // = TMEM columns 32 wh .. +31 of the hi and lo blocks
                 const unsigned char* rowp = sR + (sseq % kRS) * kRawSlot + wrow * 128;
-                const int gg = (kk * 64 + wh * 32) >> gshift;
-                const float s = bf16f((uint16_t)(pick4(s_cur, gg >> 1) >> (16 * (gg & 1))));
-                const float b = bf16f((uint16_t)(pick4(b_cur, gg >> 1) >> (16 * (gg & 1))));
-                uint32_t hv[16], lv[16];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + (((4 * kk + 2 * wh + h) ^ (wrow & 7)) << 4));
-                    dequant8_hilo(w4.x, w4.y, s, b, hv + 8 * h, lv + 8 * h);
-                    dequant8_hilo(w4.z, w4.w, s, b, hv + 8 * h + 4, lv + 8 * h + 4);
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int g = (64 * wh + 32 * c2) >> gshift;
+                    const float s = bf16f((uint16_t)bf16_at(s_cur, g)), b = bf16f((uint16_t)bf16_at(b_cur, g));
+                    uint32_t hv[16], lv[16];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + (((4 * wh + 2 * c2 + h) ^ (wrow & 7)) << 4));
+                        dequant8_hilo(w4.x, w4.y, s, b, hv + 8 * h, lv + 8 * h);
+                        dequant8_hilo(w4.z, w4.w, s, b, hv + 8 * h + 4, lv + 8 * h + 4);
+                    }
+                    tc::tmem_st16(astage + 32 * wh + 16 * c2, hv);
+                    tc::tmem_st16(astage + 64 + 32 * wh + 16 * c2, lv);
                 }
-                tc::tmem_st16(astage + 16 * wh, hv);
-                tc::tmem_st16(astage + 32 + 16 * wh, lv);
                 tc::tmem_wait_st();
             }
             // hand the step to the MMA warp: shared-memory operands (this thread's landed
@@ -820,7 +848,7 @@ bool words_tma_ok(const moe_qtensor& q) {
 template <int kMode>
 cudaError_t launch_mode(TcArgs& a, int nsm, cudaStream_t s) {
     static int cached = 0;
-    const size_t smem = kRB * kBBytes + kRS * kRawSlot + 1024;
+    const size_t smem = kRB * kBSlot + kRS * kRawSlot + 1024;
     cudaError_t e = ensure_smem((const void*)tc_gemm_kernel<kMode>, smem, cached);
     if (e != cudaSuccess) return e;
     tc_gemm_kernel<kMode><<<nsm, kTcThreads, smem, s>>>(a);
