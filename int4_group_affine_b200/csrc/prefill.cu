@@ -27,9 +27,9 @@
 // rows of every adapter side by side along K', operand B holds each job's scaled
 // LoRA-A products in its own adapter's columns (zero elsewhere), so the product
 // adds exactly each job's own adapter term into the accumulator.  Operand A is a
-// pseudo-span of the weight ring that the producer warp's lanes fill with
-// cp.async (zero where a column belongs to another matrix); operand B is staged
-// by the dequantisation warps from registers fetched a step ahead.
+// pseudo-span of the weight ring that the dequantisation threads fill with
+// cp.async (zero past the adapters' columns) together with the activations two
+// steps ahead; operand B is staged by them from registers fetched a step ahead.
 //
 //   gate/up: block 0 = gate rows, block 1 = up rows, two accumulators; epilogue
 //            SiLU(g) * u -> h (bf16).
@@ -177,6 +177,9 @@ __device__ __forceinline__ void dequant8_hilo(uint32_t w0, uint32_t w1, float s,
     }
 }
 
+// SiLU with the fast exponential and division (a few ulp; the result is rounded to bf16)
+__device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
 __device__ __forceinline__ uint32_t pick4(const uint32_t (&v)[4], int i) {
     return i == 0 ? v[0] : i == 1 ? v[1] : i == 2 ? v[2] : v[3];
 }
@@ -311,27 +314,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         int slot_mma[kRS];    // step whose MMAs read the slot directly (LoRA-B rows), or -1
         for (int i = 0; i < kRS; ++i) slot_mma[i] = -1;
         bool ok = true;
-        // LoRA-B rows of step s into slot: lane -> chunk lane % 8 of rows lane / 8 + 4 i;
-        // K' column 64 s + 8 c + e of block k = adapter (.. / r), rank index (.. % r) of its matrix
-        auto lora_span = [&](const Pos& p, int s, int slot) {
-            const Geo q = geo(p);
-            const uint32_t dst0 = tc::smem_u32(sR + slot * kRawSlot);
-            const int c = lane % 8, cc = 64 * s + 8 * c;
-            for (int blk = 0; blk < 2; ++blk) {
-                const int which = mode == kGU ? blk : 2;  // gate rows | up rows; down: two row blocks
-                const moe_lora_proj* lp = cc < nar ? tlora(L, cc / r, q.shared, which) : nullptr;
-                const int row0 = mode == kGU ? p.mt * kBM : p.mt * 2 * kBM + blk * kBM;
-                const uint16_t* src = lp ? lp->B + ((int64_t)q.mat * q.M + row0) * r + cc % r : a.act;
-                for (int i = 0; i < kBM / 4; ++i) {
-                    const int row = lane / 8 + 4 * i;
-                    const bool live = lp && row0 + row < q.M;
-                    tc::cp16(dst0 + blk * kSpanBytes + tc::sw128_off(row, c), live ? src + (int64_t)row * r : a.act,
-                             live ? 16u : 0u);
-                }
-            }
-            tc::cp_commit();  // (so that the final drain's wait covers these copies)
-            tc::cp_arrive_noinc(&bar_raw[slot]);
-        };
         // the next span into slot issued % kRS, once the span kRS before it is consumed
         auto span_next = [&]() {
             if (pt.item >= nitems || !ok) return;
@@ -374,7 +356,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     tc::mbar_arrive(bar);
                 }
             } else {
-                lora_span(pt, pt_span - nw, slot);
+                // LoRA-B rows: the dequantisation threads copy them in with the step's
+                // activations; the ring phase of the slot completes here
+                tc::mbar_arrive(&bar_raw[slot]);
             }
             ++issued;
             if (++pt_span >= nspans(pt)) {
@@ -382,6 +366,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 pt_span = 0;
             }
         };
+        if (lane == 0) {  // descriptors into the cache before the first boxes
+            if (mode == kGU) for (int i = 0; i < 4; ++i) tc::tma_prefetch_desc(&a.tm[i]);
+            if (mode == kDown) for (int i = 0; i < 2; ++i) tc::tma_prefetch_desc(&a.tm[i]);
+            if (mode == kRouterMode) tc::tma_prefetch_desc(&a.tm[0]);
+        }
         if (!lora_mode) {
             span_next();
             span_next();
@@ -392,11 +381,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // a step that opens a span keeps the ring two spans ahead
             if (!lora_mode && (!wstep || pc.kt % SP == 0)) span_next();
             if (!ok || !tc::mbar_wait_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok)) {
-                ok = false;
-                break;
-            }
-            // LoRA-B step: its operand A (this warp's own copies) must have landed
-            if (!lora_mode && !wstep && !tc::mbar_wait_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok)) {
                 ok = false;
                 break;
             }
@@ -612,7 +596,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                             const int n = ch * 16 + c;
                             if (n < n_here)
                                 a.h_out[(int64_t)(base + n) * a.ldh + i] =
-                                    f2bf16(silu(__uint_as_float(d0[c])) * __uint_as_float(d1[c]));
+                                    f2bf16(silu_fast(__uint_as_float(d0[c])) * __uint_as_float(d1[c]));
                         }
                     }
                 } else if (mode == kDown) {
@@ -656,19 +640,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             return true;
         };
 
+        // ---- LoRA-B rows of step s (operand A) into ring slot `slot`: thread (block, row) copies its
+        // row's 8 chunks; K' column 64 s + 8 c of block k = adapter (.. / r), rank index (.. % r)
+        auto lora_rows = [&](const Pos& p, int s, int slot) {
+            const Geo q = geo(p);
+            const int which = mode == kGU ? wblk : 2;  // gate rows | up rows; down: two row blocks
+            const int grow = mode == kGU ? p.mt * kBM + wrow : p.mt * 2 * kBM + wblk * kBM + wrow;
+            const bool row_ok = grow < q.M;
+            const uint32_t dst = tc::smem_u32(sR + slot * kRawSlot + wblk * kSpanBytes);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int cc = 64 * s + 8 * c;
+                const moe_lora_proj* lp = (row_ok && cc < nar) ? tlora(L, cc / r, q.shared, which) : nullptr;
+                tc::cp16(dst + tc::sw128_off(wrow, c), lp ? lp->B + ((int64_t)q.mat * q.M + grow) * r + cc % r : a.act,
+                         lp ? 16u : 0u);
+            }
+        };
+
         // ------------------------------------------------------ stream
         Pos pc, pb;  // consumer, activation loader (kLB steps ahead)
         decode(blockIdx.x, pc);
         pb = pc;
+        uint32_t pb_sseq = 0;  // weight-ring span of the loader's step
         BCtx cb;
         make_b(pb, cb);
         auto issue_step = [&](uint32_t seq) {  // loads of the activation loader's step, then advance it
             if (pb.item < nitems) {
-                if (pb.kt < pb.KW) issue_b(cb, pb.kt, seq % kRB);  // LoRA-B steps are staged by the consumer
+                if (pb.kt < pb.KW) issue_b(cb, pb.kt, seq % kRB);
+                else lora_rows(pb, pb.kt - pb.KW, pb_sseq % kRS);  // operand B is staged by the consumer
                 if (++pb.kt == pb.KT) {
                     decode(pb.item + NB, pb);
                     make_b(pb, cb);
                 }
+                if (!lora_mode && pb.item < nitems && (pb.kt >= pb.KW || pb.kt % SP == 0)) ++pb_sseq;
             }
             tc::cp_commit();
         };
@@ -731,20 +735,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 // word w = K elements 8w .. 8w+7 = TMEM columns 4w .. 4w+3 of this block
                 const unsigned char* rowp = sR + (sseq % kRS) * kRawSlot + wblk * kSpanBytes + wrow * 128;
                 const uint32_t ta = astage + wblk * 64;
+                // all four chunks are read before any TMEM store (the stores are compiler
+                // barriers), so the 16 dequantisation chains overlap
+                uint4 w4[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) w4[c] = *reinterpret_cast<const uint4*>(rowp + (((4 * kk + c) ^ (wrow & 7)) << 4));
+                uint32_t v[64];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + (((4 * kk + c) ^ (wrow & 7)) << 4));
                     const int g = (kk * kKS + 32 * c) >> gshift;  // group of these 4 words within the span
                     const __nv_bfloat162 s2 = bf16x2_of(bf16_at(s_cur, g)), b2 = bf16x2_of(bf16_at(b_cur, g));
-                    uint32_t v[16];
-                    const uint4 o0 = dequant8(w4.x, s2, b2), o1 = dequant8(w4.y, s2, b2);
-                    const uint4 o2 = dequant8(w4.z, s2, b2), o3 = dequant8(w4.w, s2, b2);
-                    v[0] = o0.x; v[1] = o0.y; v[2] = o0.z; v[3] = o0.w;
-                    v[4] = o1.x; v[5] = o1.y; v[6] = o1.z; v[7] = o1.w;
-                    v[8] = o2.x; v[9] = o2.y; v[10] = o2.z; v[11] = o2.w;
-                    v[12] = o3.x; v[13] = o3.y; v[14] = o3.z; v[15] = o3.w;
-                    tc::tmem_st16(ta + 16 * c, v);
+                    const uint4 o0 = dequant8(w4[c].x, s2, b2), o1 = dequant8(w4[c].y, s2, b2);
+                    const uint4 o2 = dequant8(w4[c].z, s2, b2), o3 = dequant8(w4[c].w, s2, b2);
+                    uint32_t* vc = v + 16 * c;
+                    vc[0] = o0.x; vc[1] = o0.y; vc[2] = o0.z; vc[3] = o0.w;
+                    vc[4] = o1.x; vc[5] = o1.y; vc[6] = o1.z; vc[7] = o1.w;
+                    vc[8] = o2.x; vc[9] = o2.y; vc[10] = o2.z; vc[11] = o2.w;
+                    vc[12] = o3.x; vc[13] = o3.y; vc[14] = o3.z; vc[15] = o3.w;
                 }
+                tc::tmem_st32(ta, v);
+                tc::tmem_st32(ta + 32, v + 32);
                 tc::tmem_wait_st();
             } else if (int4_mode) {
                 stage_lora(lr, sB + (t % kRB) * kBSlot);
