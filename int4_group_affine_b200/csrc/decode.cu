@@ -37,8 +37,7 @@ constexpr int kMaxJ = MOEQ_DECODE_MAX_JOBS;
 constexpr int kMaxR = 32;                  // LoRA rank handled by the fused path (one lane per k)
 constexpr unsigned kSpinLimit = 1u << 21;  // about a second of polling
 constexpr int kMaxOut = 32;                // output rows per CTA in phase D
-constexpr int kSplit = 8;                  // contributor split of the down LoRA-A sums
-constexpr int kSlices = 8;                 // logit slices per token in the two-level top-K (E <= 512)
+constexpr int kSplit = 8;                  // chunk split of the down LoRA-A dots in phase D
 
 struct DArgs {
     LayerArgs L;
@@ -53,7 +52,7 @@ struct DArgs {
     float* tg;      // [T*K][2r] routed LoRA-A products, by routed slot t*K+k
     float* gus;     // [T][Is][2] shared gate/up pre-activations
     float* h;       // [J][Imax] SwiGLU outputs, slot t*K+k (routed), T*K+t (shared)
-    float* tdp;     // [grid][J][r] per-CTA partial down LoRA-A products
+    float* tdp;     // (unused)
     unsigned long long* bar;  // monotonic arrival counter
     int32_t* status;
 };
@@ -330,7 +329,6 @@ __device__ __forceinline__ const moe_lora_proj* dlora(const LayerArgs& L, int a,
 }
 
 __device__ __forceinline__ float ldb(const moe_lora_proj* lp, int64_t idx) { return lp ? bf16f(lp->B[idx]) : 0.0f; }
-__device__ __forceinline__ float lda(const moe_lora_proj* lp, int64_t idx) { return lp ? bf16f(lp->A[idx]) : 0.0f; }
 
 // MT: token capacity of this instantiation (register arrays), T <= MT.
 template <int MT>
@@ -348,7 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     float* hs = xsum + T * (H / 32);             // [J][Imax] (phase D)
     float* hsum = hs + J * Imax;                 // [J][Imax/32]
     float* wpart = hsum + J * (Imax / 32);       // [kW][2][kMaxT][kMaxR] per-warp partial sums
-    float* zs = wpart;                           // phase B reuses the same space for the logits [T][E]
     float* tdsplit = wpart;                      // phase D reuses it for [kMaxJ][kMaxR][kSplit] sums
 
     __shared__ int s_aid[kMaxT];
@@ -361,9 +358,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     __shared__ float s_td[kMaxJ][kMaxR];
     __shared__ float s_v[kMaxOut][kMaxJ];
     __shared__ int s_tok[kMaxT];
-    __shared__ float s_cz[kMaxT][kSlices * MOEQ_MAX_TOPK];  // top-K candidates per slice
-    __shared__ int s_ce[kMaxT][kSlices * MOEQ_MAX_TOPK];
-    __shared__ float s_den[kMaxT][kSlices];
     unsigned long long bar_target = 0;
 
     const int R = E + (L.has_sgate ? 1 : 0);
@@ -467,111 +461,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!grid_sync(a.bar, bar_target, a.status)) return;
 
     // ------------------------------------------------------------ phase B
-    for (int q = threadIdx.x; q < T * E; q += kThreads) zs[q] = __ldcg(a.logits + q);
     if (threadIdx.x < T) s_sg[threadIdx.x] = L.has_sgate ? 1.0f / (1.0f + expf(-__ldcg(a.gsl + threadIdx.x))) : 1.0f;
-    __syncthreads();
-    // top-K in two levels: each of kSlices warps per token keeps the K best of its
-    // slice of the logits, one warp merges the candidates; ties go to the lower
-    // expert index at both levels.  Then softmax over all E (max = the top-1
-    // logit; the denominator is summed per slice, then over slices in order) and
-    // renormalisation over the chosen K.
-    {
-        const int slen = (E + kSlices - 1) / kSlices;
-        for (int q = warp; q < T * kSlices; q += kW) {
-            const int t = q / kSlices, sidx = q % kSlices, e0 = sidx * slen;
-            float zl[2];
-            int el[2];
-            for (int h = 0; h < 2; ++h) {
-                const int e = e0 + lane + 32 * h;
-                const bool ok = lane + 32 * h < slen && e < E;
-                zl[h] = ok ? zs[t * E + e] : -INFINITY;
-                el[h] = ok ? e : 0x7fffffff;
-            }
-            unsigned taken = 0;
+    // softmax, top-K (ties to the lower expert index) and renormalisation: one warp per
+    // token over its logits, read from L2
+    for (int t = warp; t < T; t += kW) {
+        int ki[MOEQ_MAX_TOPK];
+        float kw[MOEQ_MAX_TOPK];
+        warp_topk<true>(a.logits + (int64_t)t * E, E, K, ki, kw);
+        if (lane == 0)
             for (int k = 0; k < K; ++k) {
-                float bz = -INFINITY;
-                int be = 0x7fffffff;
-                for (int h = 0; h < 2; ++h)
-                    if (!((taken >> h) & 1u) && (zl[h] > bz || (zl[h] == bz && el[h] < be))) {
-                        bz = zl[h];
-                        be = el[h];
-                    }
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    if (oz > bz || (oz == bz && oe < be)) {
-                        bz = oz;
-                        be = oe;
-                    }
-                }
-                for (int h = 0; h < 2; ++h)
-                    if (el[h] == be) taken |= 1u << h;
-                if (lane == 0) {
-                    s_cz[t][sidx * K + k] = bz;
-                    s_ce[t][sidx * K + k] = be;
-                }
+                s_idx[t][k] = ki[k];
+                s_w[t][k] = kw[k];
             }
-        }
-        __syncthreads();
-        for (int t = warp; t < T; t += kW) {  // merge kSlices * K candidates
-            const int nc = kSlices * K;
-            float zl[4];
-            int el[4];
-            for (int h = 0; h < 4; ++h) {
-                const int c = lane + 32 * h;
-                zl[h] = c < nc ? s_cz[t][c] : -INFINITY;
-                el[h] = c < nc ? s_ce[t][c] : 0x7fffffff;
-            }
-            unsigned taken = 0;
-            for (int k = 0; k < K; ++k) {
-                float bz = -INFINITY;
-                int be = 0x7fffffff;
-                for (int h = 0; h < 4; ++h)
-                    if (!((taken >> h) & 1u) && (zl[h] > bz || (zl[h] == bz && el[h] < be))) {
-                        bz = zl[h];
-                        be = el[h];
-                    }
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    if (oz > bz || (oz == bz && oe < be)) {
-                        bz = oz;
-                        be = oe;
-                    }
-                }
-                for (int h = 0; h < 4; ++h)
-                    if (el[h] == be) taken |= 1u << h;
-                if (lane == 0) {
-                    s_idx[t][k] = be < E ? be : 0;
-                    s_w[t][k] = bz;  // the logit for now
-                }
-            }
-        }
-        __syncthreads();
-        for (int q = warp; q < T * kSlices; q += kW) {  // softmax denominator per slice
-            const int t = q / kSlices, sidx = q % kSlices, e0 = sidx * slen;
-            const float m = s_w[t][0];
-            float p = 0.0f;
-            for (int h = 0; h < 2; ++h) {
-                const int e = e0 + lane + 32 * h;
-                if (lane + 32 * h < slen && e < E) p += expf(zs[t * E + e] - m);
-            }
-            p = warp_sum(p);
-            if (lane == 0) s_den[t][sidx] = p;
-        }
-        __syncthreads();
-        if (threadIdx.x < T) {
-            const int t = threadIdx.x;
-            float den = 0.0f;
-            for (int sidx = 0; sidx < kSlices; ++sidx) den += s_den[t][sidx];
-            const float m = s_w[t][0];
-            float pk[MOEQ_MAX_TOPK], psum = 0.0f;
-            for (int k = 0; k < K; ++k) {
-                pk[k] = expf(s_w[t][k] - m) / den;
-                psum += pk[k];
-            }
-            for (int k = 0; k < K; ++k) s_w[t][k] = pk[k] / psum;
-        }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -635,14 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (lp) v = warp_sum(dot_bf16(lp->A + ((int64_t)e * r + d % r) * H, H, xs + t * H, lane));
         if (lane == 0) a.tg[slot * 2 * r + d] = v;
     }
-    // shared expert: LoRA-B delta, SwiGLU and partial down LoRA-A for this CTA's rows.
-    // Lane k < r holds component k; rows of a warp accumulate in registers.
+    // shared expert: LoRA-B delta and SwiGLU for this CTA's rows (lane k < r holds component k)
     if (has_shared) {
-        float pk[MT];
-#pragma unroll
-        for (int m = 0; m < MT; ++m) pk[m] = 0.0f;
         for (int i = s_lo + warp; i < s_hi; i += kW) {
-            float g[MT], u[MT], bg[MT], bu[MT], tgv[MT], tuv[MT], ad[MT];
+            float g[MT], u[MT], bg[MT], bu[MT], tgv[MT], tuv[MT];
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 if (m >= T) break;
@@ -651,13 +548,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 u[m] = gu.y;
                 const moe_lora_proj* lg = dlora(L, s_aid[m], true, 0);
                 const moe_lora_proj* lu = dlora(L, s_aid[m], true, 1);
-                const moe_lora_proj* ld = dlora(L, s_aid[m], true, 2);
                 const bool kk = lane < r;
                 bg[m] = kk ? ldb(lg, (int64_t)i * r + lane) : 0.0f;
                 bu[m] = kk ? ldb(lu, (int64_t)i * r + lane) : 0.0f;
                 tgv[m] = kk && lg ? __ldcg(a.ts + m * 2 * r + lane) : 0.0f;
                 tuv[m] = kk && lu ? __ldcg(a.ts + m * 2 * r + r + lane) : 0.0f;
-                ad[m] = kk ? lda(ld, (int64_t)lane * Is + i) : 0.0f;
             }
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
@@ -666,19 +561,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 const float uv = u[m] + L.scale * warp_sum(bu[m] * tuv[m]);
                 const float hv = silu(gv) * uv;
                 if (lane == 0) a.h[(int64_t)(T * K + m) * Imax + i] = hv;
-                pk[m] = fmaf(ad[m], hv, pk[m]);
-            }
-        }
-        if (r > 0) {
-#pragma unroll
-            for (int m = 0; m < MT; ++m)
-                if (lane < r) wpart[((warp * 2 + 0) * kMaxT + m) * kMaxR + lane] = m < T ? pk[m] : 0.0f;
-            __syncthreads();
-            for (int q = threadIdx.x; q < T * r; q += kThreads) {
-                const int m = q / r, k = q % r;
-                float p = 0.0f;
-                for (int w = 0; w < kW; ++w) p += wpart[((w * 2 + 0) * kMaxT + m) * kMaxR + k];
-                a.tdp[((int64_t)cta * J + T * K + m) * r + k] = p;
             }
         }
     }
@@ -686,35 +568,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
     // ------------------------------------------------------------ phase C
     {
-        const int u_lo = c_hi > c_lo ? c_lo / I : 0;
-        float pk[2][MT];  // partial down LoRA-A: [expert - u_lo][job], lane k
-#pragma unroll
-        for (int e2 = 0; e2 < 2; ++e2)
-#pragma unroll
-            for (int m = 0; m < MT; ++m) pk[e2][m] = 0.0f;
         for (int q = c_lo + warp; q < c_hi; q += kW) {
             const int u = q / I, i = q % I, e = s_uexp[u], nt = s_ucnt[u];
             const int64_t row = (int64_t)e * I + i;
             const int ng = H / L.gate.group;
             int toks[MT];
-            float bg[MT], bu[MT], tgv[MT], tuv[MT], ad[MT];
+            float bg[MT], bu[MT], tgv[MT], tuv[MT];
             const bool kk = lane < r;
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 toks[m] = 0;
-                bg[m] = bu[m] = tgv[m] = tuv[m] = ad[m] = 0.0f;
+                bg[m] = bu[m] = tgv[m] = tuv[m] = 0.0f;
                 if (m >= nt) continue;
                 const int slot = s_uslot[u][m], t = slot / K;
                 toks[m] = t;
                 const moe_lora_proj* lg = dlora(L, s_aid[t], false, 0);
                 const moe_lora_proj* lu = dlora(L, s_aid[t], false, 1);
-                const moe_lora_proj* ld = dlora(L, s_aid[t], false, 2);
                 if (kk) {
                     bg[m] = ldb(lg, row * r + lane);
                     bu[m] = ldb(lu, row * r + lane);
                     tgv[m] = lg ? __ldcg(a.tg + slot * 2 * r + lane) : 0.0f;
                     tuv[m] = lu ? __ldcg(a.tg + slot * 2 * r + r + lane) : 0.0f;
-                    ad[m] = lda(ld, ((int64_t)e * r + lane) * I + i);
                 }
             }
             float ag[MT], au[MT];
@@ -724,7 +598,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                      L.gate.group, H, xs, xsum, toks, nt, ag, lane, 32);
             dot_int4<MT>(L.up.packed + row * (H / 8), L.up.scales + row * ng, L.up.biases + row * ng, L.up.group, H,
                      xs, xsum, toks, nt, au, lane, 32);
-            const int eu = u - u_lo;  // 0 or 1: a CTA range spans at most two experts
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 if (m >= nt) break;
@@ -733,25 +606,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 const float uu = warp_sum(au[m]) + L.scale * warp_sum(bu[m] * tuv[m]);
                 const float hv = silu(g) * uu;
                 if (lane == 0) a.h[(int64_t)slot * Imax + i] = hv;
-                if (eu == 0) pk[0][m] = fmaf(ad[m], hv, pk[0][m]);
-                else pk[1][m] = fmaf(ad[m], hv, pk[1][m]);
-            }
-        }
-        if (r > 0 && c_hi > c_lo) {
-#pragma unroll
-            for (int e2 = 0; e2 < 2; ++e2)
-#pragma unroll
-                for (int m = 0; m < MT; ++m)
-                    if (lane < r) wpart[((warp * 2 + e2) * kMaxT + m) * kMaxR + lane] = pk[e2][m];
-            __syncthreads();
-            const int u_hi = (c_hi - 1) / I;
-            for (int q = threadIdx.x; q < (u_hi - u_lo + 1) * kMaxT * r; q += kThreads) {
-                const int e2 = q / (kMaxT * r), m = (q / r) % kMaxT, k = q % r;
-                const int u = u_lo + e2;
-                if (m >= s_ucnt[u]) continue;
-                float p = 0.0f;
-                for (int w = 0; w < kW; ++w) p += wpart[((w * 2 + e2) * kMaxT + m) * kMaxR + k];
-                a.tdp[((int64_t)cta * J + s_uslot[u][m]) * r + k] = p;
             }
         }
     }
@@ -760,28 +614,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // ------------------------------------------------------------ phase D
     stage_f32(hs, hsum, a.h, Imax, T * K, I);
     if (has_shared) stage_f32(hs + T * K * I, hsum + T * K * (I / 32), a.h + (int64_t)T * K * Imax, Imax, T, Is);
-    // t_d of every job: partials of the CTAs that own its rows, in CTA order
-    // (kSplit interleaved partial sums, then those in order).
+    __syncthreads();
+    // t_d = A_d h of every job, from the staged h: each CTA computes all of them (the A_d
+    // rows come from L2), so no cross-CTA reduction is needed.  Thread task (slot, k, p)
+    // sums the 32-element chunks c = p (mod kSplit); the kSplit partials are then added in
+    // order.
     for (int q = threadIdx.x; q < J * r * kSplit; q += kThreads) {
-        const int slot = q / (r * kSplit), k = (q / kSplit) % r, sp = q % kSplit;
+        const int slot = q / (r * kSplit), k = (q / kSplit) % r, p = q % kSplit;
+        const bool shared = slot >= T * K;
+        const int t = shared ? slot - T * K : slot / K;
+        const int n = shared ? Is : I;
+        const moe_lora_proj* ld = dlora(L, s_aid[t], shared, 2);
         float v = 0.0f;
-        int first = 0, last = -1;
-        if (slot < T * K) {
-            int u = 0;
-            while (u < U && s_uexp[u] != s_idx[slot / K][slot % K]) ++u;
-            first = (u * I) / perC;
-            last = ((u + 1) * I - 1) / perC;
-        } else if (has_shared) {
-            last = (Is - 1) / per_s;
+        if (ld) {
+            const int e = shared ? 0 : s_idx[t][slot % K];
+            const uint16_t* arow = ld->A + ((int64_t)e * r + k) * n;
+            const float* hrow = shared ? hs + T * K * I + (slot - T * K) * Is : hs + slot * I;
+            for (int c = p; c < n / 32; c += kSplit) {  // chunk c: 32 elements, swizzled like stage_f32
+                const uint4* a4 = reinterpret_cast<const uint4*>(arow + c * 32);
+                const uint4 w4[4] = {a4[0], a4[1], a4[2], a4[3]};
+                const int rot = (c & 7) << 2;
+                const float* hr = hrow + (c << 5);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t ww[4] = {w4[u].x, w4[u].y, w4[u].z, w4[u].w};
+#pragma unroll
+                    for (int h2 = 0; h2 < 4; ++h2) {
+                        const int j0 = 8 * u + 2 * h2;
+                        v = fmaf(__uint_as_float(ww[h2] << 16), hr[(j0 + rot) & 31], v);
+                        v = fmaf(__uint_as_float(ww[h2] & 0xFFFF0000u), hr[(j0 + 1 + rot) & 31], v);
+                    }
+                }
+            }
         }
-        for (int cc = first + sp; cc <= last; cc += kSplit) v += __ldcg(a.tdp + ((int64_t)cc * J + slot) * r + k);
-        tdsplit[(slot * kMaxR + k) * kSplit + sp] = v;
+        tdsplit[(slot * kMaxR + k) * kSplit + p] = v;
     }
     __syncthreads();
     for (int q = threadIdx.x; q < J * r; q += kThreads) {
         const int slot = q / r, k = q % r;
         float v = 0.0f;
-        for (int sp = 0; sp < kSplit; ++sp) v += tdsplit[(slot * kMaxR + k) * kSplit + sp];
+        for (int p = 0; p < kSplit; ++p) v += tdsplit[(slot * kMaxR + k) * kSplit + p];
         s_td[slot][k] = v;
     }
     __syncthreads();
