@@ -131,6 +131,7 @@ WsPlan plan_of(const Dims& d) {
     p.h = take((size_t)d.J * d.Imax * 4);
     p.ypart = take((size_t)d.J * d.H * 4);
     p.xn = take((size_t)d.T * d.H * 2);
+    p.xp = take(d.T >= kTcMinTokens ? (size_t)d.T * d.H * 2 : 0);
     const bool dec = d.T <= MOEQ_DECODE_MAX_TOKENS && d.J <= MOEQ_DECODE_MAX_JOBS;
     p.dts = take(dec ? (size_t)d.T * 2 * d.r * 4 : 0);
     p.dtg = take(dec ? (size_t)d.T * d.K * 2 * d.r * 4 : 0);
@@ -161,6 +162,7 @@ Work work_of(const Dims& d, const WsPlan& p, void* ws) {
     w.h = (float*)(b + p.h);
     w.ypart = (float*)(b + p.ypart);
     w.xn = (uint16_t*)(b + p.xn);
+    w.xp = (uint16_t*)(b + p.xp);
     w.T = d.T;
     w.K = d.K;
     w.E = d.E;
@@ -236,8 +238,11 @@ moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* ada
         // many tokens: expert-grouped GEMMs on the tcgen05 tensor cores; the SwiGLU
         // activations go to the workspace's h region as bf16 (the down GEMM's operand)
         uint16_t* hb = reinterpret_cast<uint16_t*>(wk.h);
+        // the int4 tiles hold each 8-group of K in the order 0 4 1 5 2 6 3 7: the gate/up
+        // operand is x in that order, and h is written in it for the down GEMM
+        LAUNCH(kKpermKind, launch_kperm(x, (int64_t)T * la.H, wk.xp, s));
         if (la.rank > 0) LAUNCH(kTcLoraGUKind, launch_tc_gemm(la, kTcLoraGU, x, la.H, wk, nullptr, wk.Imax, s));
-        LAUNCH(kTcGUKind, launch_tc_gemm(la, kTcGU, x, la.H, wk, hb, wk.Imax, s));
+        LAUNCH(kTcGUKind, launch_tc_gemm(la, kTcGU, wk.xp, la.H, wk, hb, wk.Imax, s));
         if (la.rank > 0) LAUNCH(kTcLoraDownKind, launch_tc_gemm(la, kTcLoraDown, hb, wk.Imax, wk, nullptr, wk.Imax, s));
         LAUNCH(kTcDownKind, launch_tc_gemm(la, kTcDown, hb, wk.Imax, wk, nullptr, wk.Imax, s));
         LAUNCH(kCombine, launch_combine(wk, residual, y, s));

@@ -57,11 +57,12 @@ struct Work {
     float* h;            // [J][Imax] SwiGLU activations
     float* ypart;        // [J][H] per-job weighted outputs
     uint16_t* xn;        // [T][H] normalised input (block mode)
+    uint16_t* xp;        // [T][H] input in the permuted K order of the tensor-core int4 tiles
     int T, K, E, H, I, Is, Imax, A1, C, nb, J, r;
 };
 
 struct WsPlan {
-    size_t status, n_active, idx, w, sg, logits, gs, cnt, goff, active, perm, wperm, inv, tgu, td, h, ypart, xn;
+    size_t status, n_active, idx, w, sg, logits, gs, cnt, goff, active, perm, wperm, inv, tgu, td, h, ypart, xn, xp;
     size_t bar, dts, dtg, dgus, dtdp;  // fused decode scratch (sizes zero when T is too large for it)
     size_t total;
 };
@@ -103,7 +104,7 @@ struct DecodeScratch {
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
     kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kTcLoraGUKind, kTcGUKind,
-    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKindCount
+    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kKindCount
 };
 void timing_begin(cudaStream_t s);
 void timing_mark(int kind, cudaStream_t s);
@@ -138,6 +139,9 @@ enum TcMode { kTcGU = 0, kTcDown = 1, kTcLoraGU = 2, kTcLoraDown = 3 };
 bool tc_supported(const LayerArgs& L);
 cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, int ld_act, const Work& wk,
                            const uint16_t* hb_out, int ldh, cudaStream_t s);
+// x [elems] bf16 -> xp: each 8-element group reordered 0 4 1 5 2 6 3 7 (the K order
+// of the tensor-core int4 tiles)
+cudaError_t launch_kperm(const uint16_t* x, int64_t elems, uint16_t* xp, cudaStream_t s);
 // router logits [T][E] on the tensor cores (the shared-expert gate row is not included)
 bool tc_router_supported(const moe_qtensor& router, int H, int E);
 cudaError_t launch_tc_router(const moe_qtensor& router, const float* logit_bias, const uint16_t* x, int T, int H,

@@ -142,8 +142,11 @@ __device__ __forceinline__ const moe_lora_proj* tlora(const LayerArgs& L, int a,
     return (q->A && q->B) ? q : nullptr;
 }
 
-// 8 nibbles of one word -> 8 bf16 (s*q + b, one rounding), as 4 pairs in element order.
-__device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
+// 8 nibbles of one word -> 8 bf16 (s*q + b, one rounding) as the pairs
+// (q0, q4), (q1, q5), (q2, q6), (q3, q7): the K order of every 8-group is
+// permuted to 0 4 1 5 2 6 3 7, and the activations the MMA multiplies them with
+// are stored in the same order (permute_k8), so the products are unchanged.
+__device__ __forceinline__ uint4 dequant8p(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
     const __nv_bfloat162 k128 = __float2bfloat162_rn(128.0f);
     uint32_t r[4];
 #pragma unroll
@@ -153,13 +156,17 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bf
         __nv_bfloat162 d = __hfma2(q, s2, b2);
         r[j] = *reinterpret_cast<uint32_t*>(&d);
     }
-    uint4 o;
-    o.x = __byte_perm(r[0], r[1], 0x5410);  // e0 e1
-    o.y = __byte_perm(r[2], r[3], 0x5410);  // e2 e3
-    o.z = __byte_perm(r[0], r[1], 0x7632);  // e4 e5
-    o.w = __byte_perm(r[2], r[3], 0x7632);  // e6 e7
-    return o;
+    return make_uint4(r[0], r[1], r[2], r[3]);
 }
+
+// The same K permutation applied to 8 bf16 in element order (one 16-byte chunk).
+__device__ __forceinline__ uint4 permute_k8(uint4 u) {
+    return make_uint4(__byte_perm(u.x, u.z, 0x5410), __byte_perm(u.x, u.z, 0x7632), __byte_perm(u.y, u.w, 0x5410),
+                      __byte_perm(u.y, u.w, 0x7632));
+}
+
+// Position of K element i in the permuted order.
+__device__ __forceinline__ int kperm_pos(int i) { return (i & ~7) | ((i & 3) << 1) | ((i >> 2) & 1); }
 
 // Two int8 words (8 codes) -> hi = bf16(w) and lo = bf16(w - hi) for w = s*q + b in fp32.
 __device__ __forceinline__ void dequant8_hilo(uint32_t w0, uint32_t w1, float s, float b, uint32_t* hi, uint32_t* lo) {
@@ -590,12 +597,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 tc::tmem_wait_ld();
                 if (mode == kGU) {
                     const int i = p.mt * kBM + row;
+                    const int ip = kperm_pos(i);  // h is the down GEMM's operand: permuted K order
                     if (i < q.M) {
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
                             const int n = ch * 16 + c;
                             if (n < n_here)
-                                a.h_out[(int64_t)(base + n) * a.ldh + i] =
+                                a.h_out[(int64_t)(base + n) * a.ldh + ip] =
                                     f2bf16(silu_fast(__uint_as_float(d0[c])) * __uint_as_float(d1[c]));
                         }
                     }
@@ -690,6 +698,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
         };
         if (!lora_mode) sb_next();
+        uint32_t ss0[4] = {0, 0, 0, 0}, sb0[4] = {0, 0, 0, 0}, ss1[4] = {0, 0, 0, 0}, sb1[4] = {0, 0, 0, 0};
         LoraRegs lr;
         // the epilogue of an item runs kAS steps after its last step, when its MMAs are done
         bool ep_pend = false;
@@ -717,6 +726,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     b_cur[j] = b_nxt[j];
                 }
                 sb_next();
+                if (int4_mode) {
+                    // bf16 scale and bias of each 32-word chunk of the span's two steps
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int g0 = gshift == 6 ? c >> 1 : c, g1 = gshift == 6 ? 2 + (c >> 1) : 4 + c;
+                        ss0[c] = bf16_at(s_cur, g0);
+                        sb0[c] = bf16_at(b_cur, g0);
+                        ss1[c] = bf16_at(s_cur, g1);
+                        sb1[c] = bf16_at(b_cur, g1);
+                    }
+                }
             }
             // inputs of the first LoRA-B step, fetched during the last weight step so their latency
             // overlaps it (later LoRA-B steps fetch theirs right after staging the previous one)
@@ -726,6 +746,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (span_start && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) {
                 good = false;
                 break;
+            }
+            if (mode == kLoraDown) {  // this thread's own LoRA-A chunks into h's permuted K order
+                unsigned char* rb = sR + (t % kRB) * kLoraSlot;
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        uint4* c4 = reinterpret_cast<uint4*>(rb + sub * (kLoraRows * 128) + (j ? boff1 : boff0));
+                        *c4 = permute_k8(*c4);
+                    }
             }
 
             const int kk = pc.kt % SP;  // step inside the span
@@ -743,10 +773,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 uint32_t v[64];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const int g = (kk * kKS + 32 * c) >> gshift;  // group of these 4 words within the span
-                    const __nv_bfloat162 s2 = bf16x2_of(bf16_at(s_cur, g)), b2 = bf16x2_of(bf16_at(b_cur, g));
-                    const uint4 o0 = dequant8(w4[c].x, s2, b2), o1 = dequant8(w4[c].y, s2, b2);
-                    const uint4 o2 = dequant8(w4[c].z, s2, b2), o3 = dequant8(w4[c].w, s2, b2);
+                    const __nv_bfloat162 s2 = bf16x2_of(kk ? ss1[c] : ss0[c]), b2 = bf16x2_of(kk ? sb1[c] : sb0[c]);
+                    const uint4 o0 = dequant8p(w4[c].x, s2, b2), o1 = dequant8p(w4[c].y, s2, b2);
+                    const uint4 o2 = dequant8p(w4[c].z, s2, b2), o3 = dequant8p(w4[c].w, s2, b2);
                     uint32_t* vc = v + 16 * c;
                     vc[0] = o0.x; vc[1] = o0.y; vc[2] = o0.z; vc[3] = o0.w;
                     vc[4] = o1.x; vc[5] = o1.y; vc[6] = o1.z; vc[7] = o1.w;
@@ -878,7 +907,28 @@ cudaError_t launch_kernel(TcArgs& a, cudaStream_t s) {
     }
 }
 
+
+// Activations into the permuted K order of the int4 tiles, one 16-byte chunk per thread.
+__global__ void kperm_kernel(const uint4* __restrict__ x, int64_t n, uint4* __restrict__ xp) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        xp[i] = permute_k8(x[i]);
+}
+
 }  // namespace
+
+// K-order permutation of bf16 activations (see permute_k8).
+cudaError_t launch_kperm(const uint16_t* x, int64_t elems, uint16_t* xp, cudaStream_t s) {
+    const int64_t n = elems / 8;
+    if (n == 0) return cudaSuccess;
+    int nsm = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (n + 255) / 256;
+    const int blocks = (int)(want < 8LL * nsm ? want : 8LL * nsm);
+    kperm_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(x), n, reinterpret_cast<uint4*>(xp));
+    return cudaGetLastError();
+}
+
 
 // Host-side conditions of the tensor-core expert path.
 bool tc_supported(const LayerArgs& L) {
