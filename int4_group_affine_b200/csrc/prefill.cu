@@ -53,7 +53,9 @@ namespace moeq {
 namespace {
 
 constexpr int kDeqWarps = 8;                      // dequantisation warps
-constexpr int kTcThreads = (kDeqWarps + 1) * 32;  // + the producer warp (TMA, LoRA-B rows, MMA issue)
+constexpr int kMmaWarp = kDeqWarps;               // MMA issue
+constexpr int kLoadWarp = kDeqWarps + 1;          // TMA spans, activation rows, LoRA rows
+constexpr int kTcThreads = (kDeqWarps + 2) * 32;
 constexpr int kBM = 128;                          // rows per MMA block
 constexpr int kNT = 64;                           // jobs per tile (MMA N <= 64)
 constexpr int kKS = 128;                          // K per pipeline step (two 64-wide operand sub-tiles)
@@ -61,7 +63,7 @@ constexpr int kAS = 2;                            // A stages in TMEM (dequantis
 constexpr int kLB = 2;                            // activation lookahead (steps)
 constexpr int kRB = kLB + kAS;                    // activation ring: slot of step t - kAS is free at step t
 constexpr int kRS = 4;                            // weight span ring (two spans in flight)
-constexpr int kTiles = 8;                         // per-step MMA completion barriers
+constexpr int kTiles = 16;                        // per-step MMA completion barriers
 constexpr int kSpanBytes = kBM * 128;             // one block of one span: 128 rows x 128 B
 constexpr int kRawSlot = 2 * kSpanBytes;          // two blocks
 constexpr int kSub = kNT * 128;                   // one 64-wide K sub-tile of 64 rows (128 B per row)
@@ -231,11 +233,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     // shared memory: [activation ring kRB x 16 KB][weight ring kRS x 32 KB]
     unsigned char* sB = tsm;
     unsigned char* sR = sB + kRB * kBSlot;
-    __shared__ uint64_t bar_full[kAS];    // step's operands written: one arrival per dequant warp
-    __shared__ uint64_t bar_tile[kTiles]; // MMAs of a step done (tcgen05.commit)
-    __shared__ uint64_t bar_acc[2];       // MMAs of an item done, per accumulator buffer
-    __shared__ uint64_t bar_raw[kRS];     // span landed: 32 producer-lane arrivals (+ TMA transaction count)
-    __shared__ uint64_t bar_rawfree[kRS]; // span consumed: one arrival per dequant warp
+    __shared__ uint64_t bar_full[kAS];     // step's A stage (or LoRA-B operand B) written: one arrival per dequant warp
+    __shared__ uint64_t bar_bfull[kRB];    // step's activation slot (and LoRA-A rows) landed: 32 loader lanes
+    __shared__ uint64_t bar_tile[kTiles];  // MMAs of a step done (tcgen05.commit)
+    __shared__ uint64_t bar_acc[2];        // MMAs of an item done, per accumulator buffer
+    __shared__ uint64_t bar_raw[kRS];      // span landed: 32 loader lanes (+ TMA transaction count)
+    __shared__ uint64_t bar_rawfree[kRS];  // span consumed: one arrival per dequant warp
     __shared__ uint32_t s_tmem;
     __shared__ int s_items[kMaxGroups + 1];
     __shared__ int s_goff[kMaxGroups + 1];
@@ -251,12 +254,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     } else {
         for (int g = tid; g <= ngroups; g += kTcThreads) s_goff[g] = a.goff[g];
     }
-    if (warp == kDeqWarps) {
+    if (warp == kMmaWarp) {
         tc::tmem_alloc(&s_tmem, 512);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
         for (int i = 0; i < kAS; ++i) tc::mbar_init(&bar_full[i], kDeqWarps);
+        for (int i = 0; i < kRB; ++i) tc::mbar_init(&bar_bfull[i], 32);
         for (int i = 0; i < kTiles; ++i) tc::mbar_init(&bar_tile[i], 1);
         for (int i = 0; i < kRS; ++i) {
             tc::mbar_init(&bar_raw[i], 32);
@@ -308,86 +312,180 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     };
     auto tile_jobs = [&](const Pos& p) { return min(kNT, s_goff[p.g + 1] - s_goff[p.g] - p.nt * kNT); };
     auto geo = [&](const Pos& p) { return geo_of(a, mode, p.g, s_goff[p.g + 1] - s_goff[p.g]); };
-    // spans of an item in the weight ring: its weight spans, then one per LoRA-B step
-    auto nspans = [&](const Pos& p) { return (p.KW + SP - 1) / SP + NL; };
+    // a step opens a span of the weight ring: every LoRA-B step, and every SP-th weight step
+    auto opens = [&](const Pos& p) { return !lora_mode && (p.kt >= p.KW || p.kt % SP == 0); };
+    auto advance = [&](Pos& p) {
+        if (++p.kt == p.KT) decode(p.item + NB, p);
+    };
 
-    if (warp == kDeqWarps) {
-        // ====================================================== producer warp: TMA, LoRA-B rows, MMA issue
-        Pos pc;
-        decode(blockIdx.x, pc);
-        Pos pt = pc;  // item of the next span to load
-        int pt_span = 0;
-        uint32_t issued = 0;  // spans issued
-        int slot_mma[kRS];    // step whose MMAs read the slot directly (LoRA-B rows), or -1
+    if (warp == kLoadWarp) {
+        // ====================================================== loader warp: TMA spans, activation rows,
+        // LoRA rows.  It runs ahead of the MMAs by up to kRB steps (activation slots) and of the
+        // dequantisation by up to kRS spans (weight ring).
+        Pos pl;
+        decode(blockIdx.x, pl);
+        uint32_t t = 0, cs = 0;  // step and span of pl
+        uint32_t issued = 0;     // spans issued
+        int slot_mma[kRS];       // step whose MMAs read the slot directly (LoRA-B rows), or -1
         for (int i = 0; i < kRS; ++i) slot_mma[i] = -1;
         bool ok = true;
-        // the next span into slot issued % kRS, once the span kRS before it is consumed
-        auto span_next = [&]() {
-            if (pt.item >= nitems || !ok) return;
-            const uint32_t seq = issued;
-            const int slot = seq % kRS;
-            if (seq >= (uint32_t)kRS) {
-                if (!tc::mbar_wait_ok(&bar_rawfree[slot], ((seq / kRS) - 1) & 1u, a.status, &s_ok)) {
-                    ok = false;
-                    return;
-                }
-                const int tr = slot_mma[slot];
-                if (tr >= 0 && !tc::mbar_wait_ok(&bar_tile[tr % kTiles], (tr / kTiles) & 1u, a.status, &s_ok)) {
-                    ok = false;
-                    return;
-                }
-                slot_mma[slot] = -1;
-            }
-            const int nw = (pt.KW + SP - 1) / SP;
-            if (pt_span < nw) {
-                uint64_t* bar = &bar_raw[slot];
-                if (lane == 0) {
-                    const Geo q = geo(pt);
-                    const uint32_t dst = tc::smem_u32(sR + slot * kRawSlot);
-                    const int x = pt_span * 32;  // 32 words = 128 B per row
-                    if (mode == kGU) {
-                        const int y = q.mat * q.M + pt.mt * kBM;
-                        tc::mbar_arrive_expect_tx(bar, 2 * kSpanBytes);
-                        tc::tma_load_2d(dst, &a.tm[q.shared ? 2 : 0], x, y, bar);
-                        tc::tma_load_2d(dst + kSpanBytes, &a.tm[q.shared ? 3 : 1], x, y, bar);
-                    } else if (mode == kDown) {
-                        const int y = q.mat * q.M + pt.mt * 2 * kBM;
-                        tc::mbar_arrive_expect_tx(bar, 2 * kSpanBytes);
-                        tc::tma_load_2d(dst, &a.tm[q.shared ? 1 : 0], x, y, bar);
-                        tc::tma_load_2d(dst + kSpanBytes, &a.tm[q.shared ? 1 : 0], x, y + kBM, bar);
-                    } else {
-                        tc::mbar_arrive_expect_tx(bar, kSpanBytes);
-                        tc::tma_load_2d(dst, &a.tm[0], x, pt.mt * kBM, bar);
+        // this lane's 16 activation rows of the current item (chunk lane % 8, rows lane / 8 + 4 i)
+        const int c8 = lane % 8, r0 = lane / 8;
+        int64_t rowoff[16];
+        uint32_t rowlive = 0;
+        const uint16_t* lrow[16];
+        auto item_rows = [&](const Pos& p) {
+            constexpr bool by_token = mode == kGU || mode == kLoraGU;
+            const int base = s_goff[p.g] + p.nt * kNT, end = s_goff[p.g + 1];
+            const Geo q = geo(p);
+            rowlive = 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int job = base + r0 + 4 * i;
+                const bool live = p.item < nitems && job < end;
+                rowoff[i] = live ? (int64_t)(by_token ? a.perm[job].x : job) * a.ld_act + c8 * 8 : 0;
+                if (live) rowlive |= 1u << i;
+                lrow[i] = nullptr;
+                if (lora_mode && p.item < nitems) {
+                    const int rpa = mode == kLoraGU ? 2 * r : r;
+                    const int R = p.mt * kLoraRows + r0 + 4 * i;
+                    if (R < q.M) {
+                        const int ad = R / rpa, d = R % rpa;
+                        const int which = mode == kLoraGU ? (d < r ? 0 : 1) : 2;
+                        const moe_lora_proj* lp = tlora(L, ad, q.shared, which);
+                        if (lp) lrow[i] = lp->A + ((int64_t)q.mat * r + (mode == kLoraGU ? d % r : d)) * q.K + c8 * 8;
                     }
-                } else {
-                    tc::mbar_arrive(bar);
                 }
-            } else {
-                // LoRA-B rows: the dequantisation threads copy them in with the step's
-                // activations; the ring phase of the slot completes here
-                tc::mbar_arrive(&bar_raw[slot]);
-            }
-            ++issued;
-            if (++pt_span >= nspans(pt)) {
-                decode(pt.item + NB, pt);
-                pt_span = 0;
             }
         };
+        item_rows(pl);
+        while (pl.item < nitems && ok) {
+            const bool wstep = pl.kt < pl.KW;
+            // ---- the weight-ring span this step opens
+            if (opens(pl)) {
+                const int slot = cs % kRS;
+                if (cs >= (uint32_t)kRS) {
+                    if (!tc::mbar_wait_ok(&bar_rawfree[slot], ((cs / kRS) - 1) & 1u, a.status, &s_ok)) {
+                        ok = false;
+                        break;
+                    }
+                    const int tr = slot_mma[slot];
+                    if (tr >= 0 && !tc::mbar_wait_ok(&bar_tile[tr % kTiles], (tr / kTiles) & 1u, a.status, &s_ok)) {
+                        ok = false;
+                        break;
+                    }
+                    slot_mma[slot] = -1;
+                }
+                if (wstep) {
+                    uint64_t* bar = &bar_raw[slot];
+                    if (lane == 0) {
+                        const Geo q = geo(pl);
+                        const uint32_t dst = tc::smem_u32(sR + slot * kRawSlot);
+                        const int x = (pl.kt / SP) * 32;  // 32 words = 128 B per row
+                        if (mode == kGU) {
+                            const int y = q.mat * q.M + pl.mt * kBM;
+                            tc::mbar_arrive_expect_tx(bar, 2 * kSpanBytes);
+                            tc::tma_load_2d(dst, &a.tm[q.shared ? 2 : 0], x, y, bar);
+                            tc::tma_load_2d(dst + kSpanBytes, &a.tm[q.shared ? 3 : 1], x, y, bar);
+                        } else if (mode == kDown) {
+                            const int y = q.mat * q.M + pl.mt * 2 * kBM;
+                            tc::mbar_arrive_expect_tx(bar, 2 * kSpanBytes);
+                            tc::tma_load_2d(dst, &a.tm[q.shared ? 1 : 0], x, y, bar);
+                            tc::tma_load_2d(dst + kSpanBytes, &a.tm[q.shared ? 1 : 0], x, y + kBM, bar);
+                        } else {
+                            tc::mbar_arrive_expect_tx(bar, kSpanBytes);
+                            tc::tma_load_2d(dst, &a.tm[0], x, pl.mt * kBM, bar);
+                        }
+                    } else {
+                        tc::mbar_arrive(bar);
+                    }
+                    ++issued;
+                } else {
+                    // LoRA-B rows of step s: lane -> chunk c8 of rows r0 + 4 i; K' column 64 s + 8 c of
+                    // block k = adapter (.. / r), rank index (.. % r) of block k's matrix
+                    const Geo q = geo(pl);
+                    const int s = pl.kt - pl.KW, cc = 64 * s + 8 * c8;
+                    const uint32_t dst0 = tc::smem_u32(sR + slot * kRawSlot);
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int which = mode == kGU ? blk : 2;  // gate rows | up rows; down: two row blocks
+                        const moe_lora_proj* lp = cc < nar ? tlora(L, cc / r, q.shared, which) : nullptr;
+                        const int row0 = mode == kGU ? pl.mt * kBM : pl.mt * 2 * kBM + blk * kBM;
+                        const uint16_t* src = lp ? lp->B + ((int64_t)q.mat * q.M + row0) * r + cc % r : a.act;
+                        for (int i = 0; i < kBM / 4; ++i) {
+                            const int row = r0 + 4 * i;
+                            const bool live = lp && row0 + row < q.M;
+                            tc::cp16(dst0 + blk * kSpanBytes + tc::sw128_off(row, c8),
+                                     live ? src + (int64_t)row * r : a.act, live ? 16u : 0u);
+                        }
+                    }
+                    tc::cp_commit();
+                    tc::cp_arrive_noinc(&bar_raw[slot]);
+                    slot_mma[slot] = (int)t;
+                    ++issued;
+                }
+            }
+            // ---- the step's activation slot (after the MMAs kRB steps back)
+            const int bslot = t % kRB;
+            if (t >= (uint32_t)kRB &&
+                !tc::mbar_wait_ok(&bar_tile[(t - kRB) % kTiles], ((t - kRB) / kTiles) & 1u, a.status, &s_ok)) {
+                ok = false;
+                break;
+            }
+            if (wstep || lora_mode) {
+                const uint32_t bb = tc::smem_u32(sB + bslot * kBSlot);
+                const int k0 = pl.kt * kKS;
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const bool live = (rowlive >> i) & 1u;
+                        tc::cp16(bb + sub * kSub + tc::sw128_off(r0 + 4 * i, c8),
+                                 a.act + (live ? rowoff[i] + k0 + 64 * sub : 0), live ? 16u : 0u);
+                    }
+                if (lora_mode) {  // LoRA-A rows straight into the MMA's swizzled operand layout
+                    const uint32_t rb = tc::smem_u32(sR + bslot * kLoraSlot);
+#pragma unroll
+                    for (int sub = 0; sub < 2; ++sub)
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            tc::cp16(rb + sub * (kLoraRows * 128) + tc::sw128_off(r0 + 4 * i, c8),
+                                     lrow[i] ? lrow[i] + k0 + 64 * sub : a.act, lrow[i] ? 16u : 0u);
+                }
+                tc::cp_commit();
+                tc::cp_arrive_noinc(&bar_bfull[bslot]);
+            } else {
+                tc::mbar_arrive(&bar_bfull[bslot]);  // LoRA-B step: its operand B is staged by the dequantisation
+            }
+            ++t;
+            const int item0 = pl.item;
+            advance(pl);
+            if (!lora_mode && pl.item < nitems && opens(pl)) ++cs;
+            if (pl.item != item0) item_rows(pl);
+        }
+        // drain (bounded): this warp's copies; the latest span issued into each slot
+        tc::cp_wait<0>();
+        if (lane == 0) {
+            for (uint32_t sq = issued > (uint32_t)kRS ? issued - kRS : 0; sq < issued; ++sq)
+                tc::mbar_wait(&bar_raw[sq % kRS], (sq / kRS) & 1u, a.status);
+            if (!ok) s_ok = 0;
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ====================================================== MMA warp
         if (lane == 0) {  // descriptors into the cache before the first boxes
             if (mode == kGU) for (int i = 0; i < 4; ++i) tc::tma_prefetch_desc(&a.tm[i]);
             if (mode == kDown) for (int i = 0; i < 2; ++i) tc::tma_prefetch_desc(&a.tm[i]);
             if (mode == kRouterMode) tc::tma_prefetch_desc(&a.tm[0]);
         }
-        if (!lora_mode) {
-            span_next();
-            span_next();
-        }
+        Pos pc;
+        decode(blockIdx.x, pc);
         uint32_t t = 0, cs = 0, ib = 0;  // steps, spans and items consumed
+        bool ok = true;
         while (pc.item < nitems && ok) {
             const bool wstep = pc.kt < pc.KW;
-            // a step that opens a span keeps the ring two spans ahead
-            if (!lora_mode && (!wstep || pc.kt % SP == 0)) span_next();
-            if (!ok || !tc::mbar_wait_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok)) {
+            if (!tc::mbar_wait_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok) ||
+                !tc::mbar_wait_ok(&bar_bfull[t % kRB], (t / kRB) & 1u, a.status, &s_ok) ||
+                (!lora_mode && !wstep && !tc::mbar_wait_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok))) {
                 ok = false;
                 break;
             }
@@ -411,7 +509,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         const uint64_t bd = tc::sdesc_k_sw128(bslot + (mode == kGU ? blk : 0) * kSub);
                         for (int k = 0; k < 4; ++k) tc::mma_bf16(dacc + blk * 64, ad + 2 * k, bd + 2 * k, idesc, 1u);
                     }
-                    slot_mma[cs % kRS] = (int)t;
                 } else {  // weight step: A = the dequantised tile in TMEM
                     const uint32_t astage = tmem + kTmemA + (t % kAS) * 128;
                     for (int blk = 0; blk < 2; ++blk) {
@@ -432,15 +529,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             __syncwarp();
             ++t;
             if (pc.kt == pc.KT - 1) ++ib;
-            if (++pc.kt == pc.KT) decode(pc.item + NB, pc);
-            if (!lora_mode && pc.item < nitems && (pc.kt >= pc.KW || pc.kt % SP == 0)) ++cs;
+            advance(pc);
+            if (!lora_mode && pc.item < nitems && opens(pc)) ++cs;
         }
-        // drain (bounded): this warp's copies, the last MMAs, the latest span issued into each slot
-        tc::cp_wait<0>();
-        if (lane == 0) {
+        if (lane == 0) {  // drain (bounded): the last MMAs
             if (t > 0) tc::mbar_wait(&bar_tile[(t - 1) % kTiles], ((t - 1) / kTiles) & 1u, a.status);
-            for (uint32_t sq = issued > (uint32_t)kRS ? issued - kRS : 0; sq < issued; ++sq)
-                tc::mbar_wait(&bar_raw[sq % kRS], (sq / kRS) & 1u, a.status);
             if (!ok) s_ok = 0;
         }
         __syncwarp();
@@ -484,59 +577,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
         };
 
-        // ---- activation rows (and LoRA-A rows): rows brow, brow + 32; 16-byte chunk bch of both sub-tiles
+        // ---- LoRA-B operand B of step s (thread: job rows brow, brow + 32; chunk bch of both
+        // sub-tiles): sub-tile k holds, for block k's matrix (gate/up: gate, up; down: down in
+        // sub-tile 0), each job's scaled LoRA-A products in its adapter's K' columns
         const int brow = tid / 8, bch = tid % 8;
         const uint32_t boff0 = tc::sw128_off(brow, bch), boff1 = tc::sw128_off(brow + 32, bch);
-        auto make_b = [&](const Pos& p, BCtx& c) {
-            constexpr bool by_token = mode == kGU || mode == kLoraGU;
-            const bool live_item = p.item < nitems;
-            const int base = live_item ? s_goff[p.g] + p.nt * kNT : 0;
-            const int end = live_item ? s_goff[p.g + 1] : 0;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int job = base + brow + 32 * j;
-                c.live[j] = job < end;
-                const int64_t rowi = c.live[j] ? (by_token ? a.perm[job].x : job) : 0;
-                c.src[j] = a.act + rowi * a.ld_act + bch * 8;
-                c.la[j] = nullptr;
-            }
-            if (lora_mode && live_item) {
-                const Geo q = geo(p);
-                const int rpa = mode == kLoraGU ? 2 * r : r;
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int R = p.mt * kLoraRows + brow + 32 * j;
-                    if (R < q.M) {
-                        const int ad = R / rpa, d = R % rpa;
-                        const int which = mode == kLoraGU ? (d < r ? 0 : 1) : 2;
-                        const moe_lora_proj* lp = tlora(L, ad, q.shared, which);
-                        if (lp) c.la[j] = lp->A + ((int64_t)q.mat * r + (mode == kLoraGU ? d % r : d)) * q.K + bch * 8;
-                    }
-                }
-            }
-        };
-        auto issue_b = [&](const BCtx& c, int kt, int slot) {
-            const uint32_t base = tc::smem_u32(sB + slot * kBSlot);
-            const int k0 = kt * kKS;
-#pragma unroll
-            for (int sub = 0; sub < 2; ++sub) {
-                const int ko = k0 + 64 * sub;
-                tc::cp16(base + sub * kSub + boff0, c.src[0] + (c.live[0] ? ko : 0), c.live[0] ? 16u : 0u);
-                tc::cp16(base + sub * kSub + boff1, c.src[1] + (c.live[1] ? ko : 0), c.live[1] ? 16u : 0u);
-            }
-            if (lora_mode) {  // LoRA-A rows straight into the MMA's swizzled operand layout
-                const uint32_t rb = tc::smem_u32(sR + slot * kLoraSlot);
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                    const int ko = k0 + 64 * sub;
-                    tc::cp16(rb + sub * (kLoraRows * 128) + boff0, c.la[0] ? c.la[0] + ko : a.act, c.la[0] ? 16u : 0u);
-                    tc::cp16(rb + sub * (kLoraRows * 128) + boff1, c.la[1] ? c.la[1] + ko : a.act, c.la[1] ? 16u : 0u);
-                }
-            }
-        };
-
-        // ---- LoRA-B operand B of step s: sub-tile k holds, for block k's matrix (gate/up: gate, up;
-        // down: down in sub-tile 0), each job's scaled LoRA-A products in its adapter's K' columns
         auto fetch_lora = [&](const Pos& p, int s, LoraRegs& R) {
             const Geo q = geo(p);
             const int base = s_goff[p.g] + p.nt * kNT, end = s_goff[p.g + 1];
@@ -648,43 +693,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             return true;
         };
 
-        // ---- LoRA-B rows of step s (operand A) into ring slot `slot`: thread (block, row) copies its
-        // row's 8 chunks; K' column 64 s + 8 c of block k = adapter (.. / r), rank index (.. % r)
-        auto lora_rows = [&](const Pos& p, int s, int slot) {
-            const Geo q = geo(p);
-            const int which = mode == kGU ? wblk : 2;  // gate rows | up rows; down: two row blocks
-            const int grow = mode == kGU ? p.mt * kBM + wrow : p.mt * 2 * kBM + wblk * kBM + wrow;
-            const bool row_ok = grow < q.M;
-            const uint32_t dst = tc::smem_u32(sR + slot * kRawSlot + wblk * kSpanBytes);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int cc = 64 * s + 8 * c;
-                const moe_lora_proj* lp = (row_ok && cc < nar) ? tlora(L, cc / r, q.shared, which) : nullptr;
-                tc::cp16(dst + tc::sw128_off(wrow, c), lp ? lp->B + ((int64_t)q.mat * q.M + grow) * r + cc % r : a.act,
-                         lp ? 16u : 0u);
-            }
-        };
-
         // ------------------------------------------------------ stream
-        Pos pc, pb;  // consumer, activation loader (kLB steps ahead)
+        Pos pc;
         decode(blockIdx.x, pc);
-        pb = pc;
-        uint32_t pb_sseq = 0;  // weight-ring span of the loader's step
-        BCtx cb;
-        make_b(pb, cb);
-        auto issue_step = [&](uint32_t seq) {  // loads of the activation loader's step, then advance it
-            if (pb.item < nitems) {
-                if (pb.kt < pb.KW) issue_b(cb, pb.kt, seq % kRB);
-                else lora_rows(pb, pb.kt - pb.KW, pb_sseq % kRS);  // operand B is staged by the consumer
-                if (++pb.kt == pb.KT) {
-                    decode(pb.item + NB, pb);
-                    make_b(pb, cb);
-                }
-                if (!lora_mode && pb.item < nitems && (pb.kt >= pb.KW || pb.kt % SP == 0)) ++pb_sseq;
-            }
-            tc::cp_commit();
-        };
-        for (int i = 0; i < kLB; ++i) issue_step(i);
         // scale/bias registers: current span and the next one
         uint32_t s_cur[4] = {0, 0, 0, 0}, b_cur[4] = {0, 0, 0, 0}, s_nxt[4] = {0, 0, 0, 0}, b_nxt[4] = {0, 0, 0, 0};
         Pos pn = pc;  // item of the next span whose scales are fetched
@@ -712,8 +723,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         while (pc.item < nitems) {
             const bool wstep = pc.kt < pc.KW;
             const bool span_start = !lora_mode && wstep && pc.kt % SP == 0;
-            // the MMAs of step t - kAS must be done before TMEM stage t % kAS and activation slot
-            // (t + kLB) % kRB are rewritten
+            // the MMAs of step t - kAS must be done before TMEM stage t % kAS (and, for a LoRA-B
+            // step, activation slot t % kRB) is rewritten
             if (t >= (uint32_t)kAS &&
                 !tc::mbar_wait_ok(&bar_tile[(t - kAS) % kTiles], ((t - kAS) / kTiles) & 1u, a.status, &s_ok)) {
                 good = false;
@@ -741,13 +752,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // inputs of the first LoRA-B step, fetched during the last weight step so their latency
             // overlaps it (later LoRA-B steps fetch theirs right after staging the previous one)
             if (NL > 0 && pc.kt + 1 == pc.KW) fetch_lora(pc, 0, lr);
-            issue_step(t + kLB);
-            tc::cp_wait<kLB>();  // this step's group (issued kLB steps ago) has landed
             if (span_start && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) {
                 good = false;
                 break;
             }
-            if (mode == kLoraDown) {  // this thread's own LoRA-A chunks into h's permuted K order
+            if (mode == kLoraDown) {  // the LoRA-A rows into h's permuted K order, in place
+                if (!tc::mbar_wait_ok(&bar_bfull[t % kRB], (t / kRB) & 1u, a.status, &s_ok)) {
+                    good = false;
+                    break;
+                }
                 unsigned char* rb = sR + (t % kRB) * kLoraSlot;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub)
@@ -808,9 +821,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
                 tc::tmem_wait_st();
             }
-            // hand the step to the MMA warp: shared-memory operands (this thread's landed
-            // cp.async data and generic writes) made visible to the tensor core, TMEM stores
-            // complete, then one arrival per warp
+            // hand the step to the MMA warp: shared-memory operands written here made visible to
+            // the tensor core, TMEM stores complete, then one arrival per warp
             tc::fence_async_smem();
             tc::tc_fence_before();
             __syncwarp();
@@ -836,18 +848,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     break;
                 }
             }
-            // advance the consumer
-            if (++pc.kt == pc.KT) decode(pc.item + NB, pc);
-            if (!lora_mode && pc.item < nitems && (pc.kt >= pc.KW || pc.kt % SP == 0)) ++sseq;  // next step opens a span
+            advance(pc);
+            if (!lora_mode && pc.item < nitems && opens(pc)) ++sseq;
         }
         if (good && ep_pend && !epilogue(ep_pos, ep_seq)) good = false;
-        // no cp.async may still target this CTA's shared memory at exit
-        tc::cp_wait<0>();
-        if (!good) s_ok = 0;  // left early: let the producer stop waiting
+        if (!good) s_ok = 0;  // left early: let the other warps stop waiting
     }
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == kDeqWarps) tc::tmem_dealloc(tmem, 512);
+    if (warp == kMmaWarp) tc::tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------ host side
