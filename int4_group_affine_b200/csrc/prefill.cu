@@ -2,34 +2,41 @@
 // the many-token case: the 8-bit router, gate/up with fused SwiGLU, down with
 // the routing weight, and the two LoRA-A products.
 //
-// Swap-AB: a tile is weight rows (M = 128, one TMEM lane each) by up to 64 jobs
-// of one expert group (N), over K in steps of 64.
+// Swap-AB: a tile is weight rows (M = 128 per block, one TMEM lane each) by up
+// to 64 jobs of one expert group (N), over K in steps of 128 (two 64-wide
+// operand sub-tiles).
 //
 // Weights stream through the tensor memory accelerator: for each span of 128
-// bytes of packed words per row (K = 256 for int4, 128 for int8) the producer
-// warp loads a 128-row box per block with cp.async.bulk.tensor (128-byte
-// swizzle) into a ring of four slots, three spans ahead, so DRAM sees whole
-// 128-byte lines.  Each dequantisation thread owns one weight row (half of one
-// for int8) and thus one TMEM lane: it prefetches the row's scales and biases
-// into registers one span ahead, dequantises the row's 64 weights of each K-step
-// into bf16 (w = fma(q, s, b), one rounding) and writes them with tcgen05.st
-// into one of four TMEM stages, the MMA's A operand; the dequantised tile never
-// touches shared memory, whose bandwidth then serves the MMA's B reads.
-// Activations (rows gathered by token, or the h rows of the jobs) come in with
-// cp.async four K-steps ahead into a K-major 128-byte-swizzled ring (operand B).
-// One producer lane issues the MMAs (4 x K=16 per block) and commits them to
-// mbarriers; accumulators are double-buffered in TMEM and each item's epilogue
-// runs a few steps after its last MMA, so the dequantisation never waits on the
-// tensor core at item boundaries.
+// bytes of packed words per row (K = 256 for int4, 128 for int8) the loader warp
+// loads a 128-row box per block with cp.async.bulk.tensor (128-byte swizzle)
+// into a ring of four slots, so DRAM sees whole 128-byte lines.  Each
+// dequantisation thread owns one weight row and thus one TMEM lane: it keeps the
+// row's scales and biases in registers one span ahead, dequantises the row's
+// weights of each K-step into bf16 (w = fma(q, s, b), one rounding) and writes
+// them with tcgen05.st into one of two TMEM stages, the A operand of the MMA; the
+// dequantised tile never touches shared memory.  Within every 8 consecutive K
+// the tiles hold the order 0 4 1 5 2 6 3 7, the order in which the nibbles of a
+// word come out of two shift-and-mask steps, so no byte permutes are spent; the
+// activations carry the same order (x permuted once, h written permuted by the
+// gate/up epilogue), and a dot product does not depend on the order of its terms.
+//
+// Activations (operand B) fill a K-major 128-byte-swizzled ring of four slots,
+// two steps ahead of the dequantisation: TMA boxes where the rows are contiguous
+// (the h rows of the jobs for down, the tokens for the router), cp.async by the
+// loader's lanes where they are scattered (gate/up gathers x by token) or come
+// with adapter rows (LoRA-A).  One lane of the MMA warp issues the MMAs (8 x
+// K=16 per block per step) and commits them to per-step mbarriers; accumulators
+// are double-buffered in TMEM and each item's epilogue runs a few steps after its
+// last MMA, so the dequantisation never waits on the tensor core at item ends.
 //
 // The unmerged LoRA-B term (alpha/r) B (A x) is one more MMA K-step per item
 // (per 64 columns of K' = adapters x r per matrix): operand A holds the LoRA-B
 // rows of every adapter side by side along K', operand B holds each job's scaled
 // LoRA-A products in its own adapter's columns (zero elsewhere), so the product
 // adds exactly each job's own adapter term into the accumulator.  Operand A is a
-// pseudo-span of the weight ring that the dequantisation threads fill with
-// cp.async (zero past the adapters' columns) together with the activations two
-// steps ahead; operand B is staged by them from registers fetched a step ahead.
+// pseudo-span of the weight ring that the loader fills with cp.async (zero past
+// the adapters' columns); operand B is staged by the dequantisation threads from
+// registers fetched a step ahead.
 //
 //   gate/up: block 0 = gate rows, block 1 = up rows, two accumulators; epilogue
 //            SiLU(g) * u -> h (bf16).
@@ -41,9 +48,10 @@
 //   LoRA-A:  bf16 A rows of every adapter, copied by cp.async straight into the
 //            swizzled operand layout, 64 real rows per tile.
 //
-// Warp roles: 8 dequantisation warps (loads of activations and scales, dequant,
-// epilogue) and one producer warp (TMA spans, LoRA-B rows, MMA issue); they hand
-// steps over through mbarriers, so no CTA-wide barrier sits in the K loop.
+// Warp roles: 8 dequantisation warps (scales, dequant, LoRA-B operand, epilogue),
+// one MMA warp and one loader warp (weight spans, activations, LoRA rows); they
+// hand steps over through mbarriers, so no CTA-wide barrier sits in the K loop.
+// Every wait is bounded in time and raises MOE_ERR_TIMEOUT when it gives up.
 // Persistent grid: CTA c takes items c, c + grid, ...
 #include <cudaTypedefs.h>
 
@@ -80,6 +88,8 @@ enum Mode { kGU = 0, kDown = 1, kLoraGU = 2, kLoraDown = 3, kRouterMode = 4 };
 
 struct TcArgs {
     CUtensorMap tm[4];    // weight words: gate/up {gate, up, s_gate, s_up}; down {down, s_down}; router {router}
+    CUtensorMap tmb;      // bf16 activations in 64 x 64 boxes: down the h rows of the jobs, router the
+                          // token rows of x
     LayerArgs L;
     int mode;
     const uint16_t* act;  // bf16 activation rows: x (by token) or h (by job)
@@ -223,6 +233,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     constexpr int mode = kMode;
     constexpr bool lora_mode = mode == kLoraGU || mode == kLoraDown;
+    // activation tiles by TMA boxes (rows contiguous in the activation matrix); the gate/up
+    // rows are tokens scattered over x and the LoRA-A modes add the adapters' rows: cp.async
+    constexpr bool tma_b = mode == kDown || mode == kRouterMode;
     constexpr bool int8_mode = mode == kRouterMode;
     constexpr bool int4_mode = mode == kGU || mode == kDown;
     constexpr int SP = int8_mode ? 1 : 2;  // steps per weight span (128 B of words per row)
@@ -335,6 +348,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         uint32_t rowlive = 0;
         const uint16_t* lrow[16];
         auto item_rows = [&](const Pos& p) {
+            if (tma_b) return;
             constexpr bool by_token = mode == kGU || mode == kLoraGU;
             const int base = s_goff[p.g] + p.nt * kNT, end = s_goff[p.g + 1];
             const Geo q = geo(p);
@@ -431,7 +445,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 ok = false;
                 break;
             }
-            if (wstep || lora_mode) {
+            if (wstep && tma_b) {
+                // activations by TMA: one 64 x 64 box per sub-tile (the tile's jobs for down, its
+                // tokens for the router), landing in the MMA's swizzled layout
+                const uint32_t bb = tc::smem_u32(sB + bslot * kBSlot);
+                uint64_t* bar = &bar_bfull[bslot];
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar, kBSlot);
+                if (lane < 2)
+                    tc::tma_load_2d(bb + lane * kSub, &a.tmb, pl.kt * kKS + 64 * lane, s_goff[pl.g] + pl.nt * kNT, bar);
+                if (lane != 0) tc::mbar_arrive(bar);
+            } else if (wstep || lora_mode) {
                 const uint32_t bb = tc::smem_u32(sB + bslot * kBSlot);
                 const int k0 = pl.kt * kKS;
 #pragma unroll
@@ -467,72 +490,83 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         if (lane == 0) {
             for (uint32_t sq = issued > (uint32_t)kRS ? issued - kRS : 0; sq < issued; ++sq)
                 tc::mbar_wait(&bar_raw[sq % kRS], (sq / kRS) & 1u, a.status);
+            if (tma_b)
+                for (uint32_t sq = t > (uint32_t)kRB ? t - kRB : 0; sq < t; ++sq)
+                    tc::mbar_wait(&bar_bfull[sq % kRB], (sq / kRB) & 1u, a.status);
             if (!ok) s_ok = 0;
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        // ====================================================== MMA warp
-        if (lane == 0) {  // descriptors into the cache before the first boxes
+        // ====================================================== MMA warp: lane 0 alone, so that
+        // between two steps it does little more than wait and issue
+        if (lane == 0) {
             if (mode == kGU) for (int i = 0; i < 4; ++i) tc::tma_prefetch_desc(&a.tm[i]);
             if (mode == kDown) for (int i = 0; i < 2; ++i) tc::tma_prefetch_desc(&a.tm[i]);
             if (mode == kRouterMode) tc::tma_prefetch_desc(&a.tm[0]);
-        }
-        Pos pc;
-        decode(blockIdx.x, pc);
-        uint32_t t = 0, cs = 0, ib = 0;  // steps, spans and items consumed
-        bool ok = true;
-        while (pc.item < nitems && ok) {
-            const bool wstep = pc.kt < pc.KW;
-            if (!tc::mbar_wait_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok) ||
-                !tc::mbar_wait_ok(&bar_bfull[t % kRB], (t / kRB) & 1u, a.status, &s_ok) ||
-                (!lora_mode && !wstep && !tc::mbar_wait_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok))) {
-                ok = false;
-                break;
-            }
-            tc::tc_fence_after();
-            if (lane == 0) {
-                const uint32_t idesc = tc::idesc_bf16(kBM, (tile_jobs(pc) + 15) / 16 * 16);
-                const uint32_t bslot = tc::smem_u32(sB + (t % kRB) * kBSlot);
+            if (tma_b) tc::tma_prefetch_desc(&a.tmb);
+            // descriptors of the activation sub-tiles: the base one plus the start-address offset
+            // (16-byte units in the low bits; shared addresses stay below 2^18)
+            const uint64_t bdesc0 = tc::sdesc_k_sw128(tc::smem_u32(sB));
+            auto bdesc = [&](int b, int sub) { return bdesc0 + (uint64_t)((b * kBSlot + sub * kSub) >> 4); };
+            Pos pc;
+            decode(blockIdx.x, pc);
+            uint32_t t = 0, cs = 0, ib = 0;  // steps, spans and items consumed
+            bool ok = true;
+            uint32_t idesc = tc::idesc_bf16(kBM, (tile_jobs(pc) + 15) / 16 * 16);
+            while (pc.item < nitems) {
+                const bool wstep = pc.kt < pc.KW;
+                if (!tc::mbar_spin_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok) ||
+                    !tc::mbar_spin_ok(&bar_bfull[t % kRB], (t / kRB) & 1u, a.status, &s_ok) ||
+                    (!lora_mode && !wstep && !tc::mbar_spin_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok))) {
+                    ok = false;
+                    break;
+                }
+                tc::tc_fence_after();
                 const uint32_t dacc = tmem + (ib & 1u) * 128u;
+                const int b = t % kRB;
                 if (lora_mode) {  // A: the LoRA-A rows, copied swizzled into the ring
-                    const uint32_t aslot = tc::smem_u32(sR + (t % kRB) * kLoraSlot);
+                    const uint32_t aslot = tc::smem_u32(sR + b * kLoraSlot);
+#pragma unroll
                     for (int sub = 0; sub < 2; ++sub) {
                         const uint64_t ad = tc::sdesc_k_sw128(aslot + sub * (kLoraRows * 128));
-                        const uint64_t bd = tc::sdesc_k_sw128(bslot + sub * kSub);
+#pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            tc::mma_bf16(dacc, ad + 2 * k, bd + 2 * k, idesc, (pc.kt > 0 || sub > 0 || k > 0) ? 1u : 0u);
+                            tc::mma_bf16(dacc, ad + 2 * k, bdesc(b, sub) + 2 * k, idesc, (pc.kt > 0 || sub > 0 || k > 0) ? 1u : 0u);
                     }
                 } else if (!wstep) {  // LoRA-B step: A = LoRA-B rows of the pseudo-span, one accumulator per block
                     const uint32_t rs = tc::smem_u32(sR + (cs % kRS) * kRawSlot);
+#pragma unroll
                     for (int blk = 0; blk < 2; ++blk) {
                         const uint64_t ad = tc::sdesc_k_sw128(rs + blk * kSpanBytes);
-                        const uint64_t bd = tc::sdesc_k_sw128(bslot + (mode == kGU ? blk : 0) * kSub);
+                        const uint64_t bd = bdesc(b, mode == kGU ? blk : 0);
+#pragma unroll
                         for (int k = 0; k < 4; ++k) tc::mma_bf16(dacc + blk * 64, ad + 2 * k, bd + 2 * k, idesc, 1u);
                     }
                 } else {  // weight step: A = the dequantised tile in TMEM
                     const uint32_t astage = tmem + kTmemA + (t % kAS) * 128;
+                    const uint32_t first = pc.kt == 0 ? 0u : 1u;
+#pragma unroll
                     for (int blk = 0; blk < 2; ++blk) {
                         // router: hi and lo parts into one accumulator; otherwise one accumulator per block
                         const uint32_t d = dacc + (int8_mode ? 0u : (uint32_t)blk * 64u);
-                        for (int sub = 0; sub < 2; ++sub) {
-                            const uint64_t bd = tc::sdesc_k_sw128(bslot + sub * kSub);
-                            for (int k = 0; k < 4; ++k) {  // K=16 per MMA: 8 TMEM columns, +32 B in the swizzled B tile
-                                const bool first = pc.kt == 0 && sub == 0 && k == 0 && (!int8_mode || blk == 0);
-                                tc::mma_bf16_ts(d, astage + blk * 64 + sub * 32 + 8 * k, bd + 2 * k, idesc, first ? 0u : 1u);
-                            }
-                        }
+#pragma unroll
+                        for (int sub = 0; sub < 2; ++sub)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)  // K=16 per MMA: 8 TMEM columns, +32 B in the swizzled B tile
+                                tc::mma_bf16_ts(d, astage + blk * 64 + sub * 32 + 8 * k, bdesc(b, sub) + 2 * k, idesc,
+                                                (sub == 0 && k == 0 && (!int8_mode || blk == 0)) ? first : 1u);
                     }
                 }
                 tc::mma_commit(&bar_tile[t % kTiles]);
-                if (pc.kt == pc.KT - 1) tc::mma_commit(&bar_acc[ib & 1u]);
+                const bool last = pc.kt == pc.KT - 1;
+                if (last) tc::mma_commit(&bar_acc[ib & 1u]);
+                ++t;
+                if (last) ++ib;
+                advance(pc);
+                if (last && pc.item < nitems) idesc = tc::idesc_bf16(kBM, (tile_jobs(pc) + 15) / 16 * 16);
+                if (!lora_mode && pc.item < nitems && opens(pc)) ++cs;
             }
-            __syncwarp();
-            ++t;
-            if (pc.kt == pc.KT - 1) ++ib;
-            advance(pc);
-            if (!lora_mode && pc.item < nitems && opens(pc)) ++cs;
-        }
-        if (lane == 0) {  // drain (bounded): the last MMAs
+            // drain (bounded): the last MMAs
             if (t > 0) tc::mbar_wait(&bar_tile[(t - 1) % kTiles], ((t - 1) / kTiles) & 1u, a.status);
             if (!ok) s_ok = 0;
         }
@@ -826,10 +860,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             tc::fence_async_smem();
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(&bar_full[t % kAS]);
-                if (!lora_mode && (!wstep || kk == SP - 1 || pc.kt == pc.KW - 1)) tc::mbar_arrive(&bar_rawfree[sseq % kRS]);
+            if (lane == 0) tc::mbar_arrive(&bar_full[t % kAS]);
+            // A LoRA-B step's span (rows the MMAs read directly) is released only once it has
+            // landed: the loader must have seen the slot's previous release complete before this
+            // one completes, or its parity wait would alias two phases ahead.
+            if (!lora_mode && !wstep && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) {
+                good = false;
+                break;
             }
+            if (lane == 0 && !lora_mode && (!wstep || kk == SP - 1 || pc.kt == pc.KW - 1))
+                tc::mbar_arrive(&bar_rawfree[sseq % kRS]);
             ++t;
 
             if (pc.kt == pc.KT - 1) {  // this step ends an item: its epilogue is deferred
@@ -882,6 +922,23 @@ cudaError_t encode_words(CUtensorMap* m, const void* base, int64_t rows, int64_t
     const cuuint32_t box[2] = {32, (cuuint32_t)kBM};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Tensor map over bf16 rows [rows][cols] (row pitch ld elements) in boxes of 64 columns x
+// box_rows rows, 128-byte swizzled like the MMA's K-major operand; rows past the end read
+// as zero.
+cudaError_t encode_act(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    if (((uintptr_t)base & 15) || (ld * 2) % 16 || cols > ld) return cudaErrorInvalidValue;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -990,6 +1047,8 @@ cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, in
     a.t_in = mode == kTcGU ? wk.tgu : wk.td;
     a.status = wk.status;
     cudaError_t e = cudaSuccess;
+    if (mode == kTcDown) e = encode_act(&a.tmb, act, wk.J, ld_act, ld_act, kNT);
+    if (e != cudaSuccess) return e;
     if (mode == kTcGU) {
         e = encode_words(&a.tm[0], L.gate.packed, (int64_t)L.E * L.I, L.H / 8);
         if (e == cudaSuccess) e = encode_words(&a.tm[1], L.up.packed, (int64_t)L.E * L.I, L.H / 8);
@@ -1019,6 +1078,7 @@ cudaError_t launch_tc_router(const moe_qtensor& router, const float* logit_bias,
     a.T = T;
     a.status = status;
     cudaError_t e = encode_words(&a.tm[0], router.packed, E, H / 4);
+    if (e == cudaSuccess) e = encode_act(&a.tmb, x, T, H, H, kNT);
     if (e != cudaSuccess) return e;
     return launch_kernel(a, s);
 }

@@ -62,6 +62,35 @@ __device__ __forceinline__ bool mbar_wait_ok(uint64_t* bar, uint32_t parity, int
     return false;
 }
 
+// Non-suspending test of a phase (for a dedicated issuing thread that must react at once).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// As mbar_wait_ok, by polling without suspension.
+__device__ __forceinline__ bool mbar_spin_ok(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* ok) {
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_test(bar, parity)) return true;
+        if ((i & 63) == 63) {
+            if (*ok == 0) return false;
+            if (globaltimer_ns() - t0 > 2000000000ull) break;
+        }
+    }
+    raise_status(status, MOE_ERR_TIMEOUT);
+    *ok = 0;
+    return false;
+}
+
 // Arrive on `bar` once all cp.async copies this thread issued so far have landed
 // (the arrival counts toward the barrier's expected count).
 __device__ __forceinline__ void cp_arrive_noinc(uint64_t* bar) {
