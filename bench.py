@@ -200,7 +200,19 @@ KIND_UNIT = {"router_logits": "router", "tc_router": "router", "gate_up": "gate_
              "tc_lora_down": "lora_down", "decode_fused": "layer"}
 
 
-def kernel_roofline(kind, dur_ms, nbytes, nflops, peaks, src, timed_s):
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
+# dominant kernel, from one ncu capture of the kernel as it stands; the capture's
+# summary sits under profiles/ (named here).  An entry is removed whenever its
+# kernel changes, so the bench reports null rather than a stale figure.
+NCU_TRAFFIC = {
+    # one gate/up launch over the 2048-token prompt of one layer
+    ("prefill", "tc_gate_up"): (333590784 + 9545728, "profiles/tc_gate_up_down_prefill_layer.md"),
+    # one launch of the fused decode kernel, one token, top-4
+    ("decode_k4", "decode_fused"): (10939136 + 256, "profiles/decode_fused_decode_k4.md"),
+}
+
+
+def kernel_roofline(kind, dur_ms, nbytes, nflops, peaks, src, timed_s, workload=None):
     """Roofline entry of one kernel: the bound is whichever of HBM time and bf16
     tensor time is larger for its algorithmic bytes and flops; the tensor peak is
     the burst figure for a timed region under a second, else the sustained one."""
@@ -220,8 +232,11 @@ def kernel_roofline(kind, dur_ms, nbytes, nflops, peaks, src, timed_s):
     else:
         roof = {"kernel": kind, "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(gbs / hbm, 4), "peak_source": "%s hbm_gbs" % src, "tensor": tensor}
-    roof.update({"traffic": None, "launch_us": round(dur_ms * 1e3, 3), "bytes_per_launch": int(nbytes),
-                 "flops_per_launch": int(nflops)})
+    tr = NCU_TRAFFIC.get((workload, kind))
+    roof.update({"traffic": tr[0] if tr else None, "launch_us": round(dur_ms * 1e3, 3),
+                 "bytes_per_launch": int(nbytes), "flops_per_launch": int(nflops)})
+    if tr:
+        roof["traffic_source"] = "ncu capture, " + tr[1]
     return roof
 
 
@@ -455,7 +470,7 @@ def run_moe(args, world, rank, local):
     if dom is not None and dom in KIND_UNIT:
         unit = KIND_UNIT[dom]
         roof = kernel_roofline(dom, kt[dom][0] / kt[dom][1], acc["kernel_bytes"][unit], acc["kernel_flops"][unit],
-                               peaks, src, ms * 1e-3)
+                               peaks, src, ms * 1e-3, args.workload)
     step_bytes = acc["weight_bytes"] + acc["act_bytes"]
     step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
     value = tokens_per_step * K * world / (ms * 1e-3)
