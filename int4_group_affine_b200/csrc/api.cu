@@ -135,8 +135,7 @@ WsPlan plan_of(const Dims& d) {
     const bool dec = d.T <= MOEQ_DECODE_MAX_TOKENS && d.J <= MOEQ_DECODE_MAX_JOBS;
     p.dts = take(dec ? (size_t)d.T * 2 * d.r * 4 : 0);
     p.dtg = take(dec ? (size_t)d.T * d.K * 2 * d.r * 4 : 0);
-    p.dgus = take(dec ? (size_t)d.T * std::max(d.Is, 1) * 2 * 4 : 0);
-    p.dtdp = take(dec ? (size_t)MOEQ_DECODE_MAX_CTAS * d.J * d.r * 4 : 0);
+    p.dtdp = take(dec ? (size_t)MOEQ_DECODE_MAX_CTAS * 3 * d.T * d.r * 4 : 0);
     p.total = o;
     return p;
 }
@@ -270,7 +269,6 @@ bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id
     sc.gsl = (float*)(b + p.gs);
     sc.ts = (float*)(b + p.dts);
     sc.tg = (float*)(b + p.dtg);
-    sc.gus = (float*)(b + p.dgus);
     sc.h = (float*)(b + p.h);
     sc.tdp = (float*)(b + p.dtdp);
     sc.bar = (unsigned long long*)(b + p.bar);

@@ -63,7 +63,7 @@ struct Work {
 
 struct WsPlan {
     size_t status, n_active, idx, w, sg, logits, gs, cnt, goff, active, perm, wperm, inv, tgu, td, h, ypart, xn, xp;
-    size_t bar, dts, dtg, dgus, dtdp;  // fused decode scratch (sizes zero when T is too large for it)
+    size_t bar, dts, dtg, dtdp;  // fused decode scratch (sizes zero when T is too large for it)
     size_t total;
 };
 
@@ -93,11 +93,16 @@ inline cudaError_t ensure_smem(const void* fn, size_t bytes, int& cached) {
 #define MOEQ_DECODE_MAX_JOBS 32
 #define MOEQ_DECODE_MAX_CTAS 256
 
-// Scratch of the fused decode kernel (all inside the forward workspace).
+#define MOEQ_DECODE_MAX_RANK 32
+
+// Scratch of the fused decode kernel (all inside the forward workspace).  Besides the
+// status word and the arrival counter, bytes 16..255 of the workspace header (zeroed by
+// moe_workspace_init) hold the kernel's per-launch ready flags.
 struct DecodeScratch {
-    float *logits, *gsl, *ts, *tg, *gus, *h, *tdp;
+    float *logits, *gsl, *ts, *tg, *h;
+    float* tdp;               // [MOEQ_DECODE_MAX_CTAS][3][T][rank] partial sums
     unsigned long long* bar;  // monotonic arrival counter: starts zeroed (workspace header)
-    int32_t* status;
+    int32_t* status;          // workspace base (status word)
 };
 
 // ------------------------------------------------------------- timing
