@@ -207,6 +207,8 @@ KIND_UNIT = {"router_logits": "router", "tc_router": "router", "gate_up": "gate_
 NCU_TRAFFIC = {
     # one gate/up launch over the 2048-token prompt of one layer
     ("prefill", "tc_gate_up"): (333590784 + 9545728, "profiles/tc_gate_up_down_prefill_layer.md"),
+    # one launch of the fused decode kernel, one token, top-4
+    ("decode_k4", "decode_fused"): (11296000, "profiles/decode_fused_decode_k4.md"),
 }
 
 
