@@ -242,22 +242,28 @@ def kernel_roofline(kind, dur_ms, nbytes, nflops, peaks, src, timed_s, workload=
 
 # ----------------------------------------------------------------- distributed plumbing
 def dist_setup(n_gpus):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE); NCCL on GPUs.  Without
+    a GPU the ranks join a gloo group on the CPU, which is how the multi-rank plumbing is
+    tested."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    cuda = torch.cuda.is_available()
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
-    else:
+        if cuda:
+            torch.cuda.set_device(local)
+        dist.init_process_group("nccl" if cuda else "gloo", timeout=datetime.timedelta(seconds=180))
+    elif cuda:
         torch.cuda.set_device(0)
     return world, rank, local
 
 
 def barrier(world):
     import torch
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -268,9 +274,16 @@ def max_over_ranks(v, world):
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank_step, steps, world, ms):
+    """Whole-job throughput: the units every rank processed in `steps` steps over the
+    slowest rank's time `ms` (replicas: the same work on each rank, weak scaling)."""
+    return units_per_rank_step * steps * world / (ms * 1e-3)
 
 
 def capture_steps(step, first, count):
@@ -473,7 +486,7 @@ def run_moe(args, world, rank, local):
                                peaks, src, ms * 1e-3, args.workload)
     step_bytes = acc["weight_bytes"] + acc["act_bytes"]
     step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
-    value = tokens_per_step * K * world / (ms * 1e-3)
+    value = job_throughput(tokens_per_step, K, world, ms)
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms_step, 6), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -574,7 +587,7 @@ def run_e2e(moeq, shape, layers, xs_host, aids_host, K, W, copies, n_inputs, sta
     del g
     toks = T * (len(layers) if stack else 1)
     h2d = T * H * 2 + (0 if ha is None else T * 4)
-    return {"value": round(toks * K * world / (ms * 1e-3), 2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    return {"value": round(job_throughput(toks, K, world, ms), 2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": T * H * 2, "ms_per_step": round(ms / K, 6)}
 
 
@@ -643,7 +656,7 @@ def run_mixed(args, world, rank, local):
                 "bytes_per_launch": per}
     step_gbs = L * layer_bytes / (ms_step * 1e-3) / 1e9
     out = {
-        "metric": METRIC, "value": round(T * K * world / (ms * 1e-3), 2), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": round(job_throughput(T, K, world, ms), 2), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(ms_step, 6), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "ternary/int4 weights, bf16 activations, fp32 accumulate",
         "data": "synthetic (seeded generator; no trained weights)",
