@@ -246,13 +246,19 @@ __device__ void stage_f32(float* dst, float* dsum, const float* src, int ld, int
     }
 }
 
-// 32 nibbles -> 32 floats.
+// 32 nibbles q -> 32 floats 128 + q: the nibble goes into bits 16..19 of 128.0f (whose
+// upper 7 mantissa bits count in units of 1), one shift and one and-or each.  Products
+// (128 + q) x are exact in fp32 for bf16 x; the caller removes the 128 through the bias
+// term: s sum (128 + q) x + (b - 128 s) sum x = sum (s q + b) x.
 __device__ __forceinline__ void unpack4(const uint4 q4, float* qf) {
     const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
     for (int w = 0; w < 4; ++w)
 #pragma unroll
-        for (int f = 0; f < 8; ++f) qf[w * 8 + f] = u2f_small((qw[w] >> (4 * f)) & 15u);
+        for (int f = 0; f < 8; ++f) {
+            const uint32_t at16 = f <= 4 ? qw[w] << (16 - 4 * f) : qw[w] >> (4 * f - 16);
+            qf[w * 8 + f] = __uint_as_float((at16 & 0x000F0000u) | 0x43000000u);
+        }
 }
 
 // sum over chunk c of q[j] * v[j] for a staged (swizzled) vector row v.
@@ -302,11 +308,12 @@ __device__ __noinline__ void dot_int4(const uint32_t* __restrict__ prow, const u
         if (c >= nc) break;
         float qf[32];
         unpack4(q[it], qf);
+        const float b128 = fmaf(-128.0f, s[it], b[it]);
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             if (m >= nv) break;
             const float a = chunk_qdot(qf, vbase + vid[m] * n, c);
-            acc[m] = fmaf(s[it], a, fmaf(b[it], vsum[vid[m] * nc + c], acc[m]));
+            acc[m] = fmaf(s[it], a, fmaf(b128, vsum[vid[m] * nc + c], acc[m]));
         }
     }
 }
