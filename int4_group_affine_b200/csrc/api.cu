@@ -214,7 +214,8 @@ moe_status router_enqueue(const uint16_t* x, const moe_qtensor& router, const mo
                           int T, int H, int E, float* logits, float* gs, int32_t* status, cudaStream_t s) {
     if (T >= kTcMinTokens && tc_router_supported(router, H, E)) {
         LAUNCH(kTcRouterKind, launch_tc_router(router, lb, x, T, H, E, logits, status, s));
-        if (sg) LAUNCH(kRouter, launch_router_logits(x, router, sg, nullptr, T, H, 0, logits, gs, s));
+        if (sg && aligned(x, 16) && H % 16 == 0) LAUNCH(kRouter, launch_sgate_logits(x, *sg, T, H, gs, s));
+        else if (sg) LAUNCH(kRouter, launch_router_logits(x, router, sg, nullptr, T, H, 0, logits, gs, s));
         return MOE_OK;
     }
     LAUNCH(kRouter, launch_router_logits(x, router, sg, lb, T, H, E, logits, gs, s));

@@ -125,6 +125,9 @@ cudaError_t launch_dequant_mixed(const moe_mixed_tensor& t, int G, float* out, c
 cudaError_t launch_router_logits(const uint16_t* x, const moe_qtensor& router, const moe_qtensor* sgate,
                                  const float* logit_bias, int T, int H, int E, float* logits, float* gs,
                                  cudaStream_t s);
+// the shared-expert gate logit of every token alone (x rows 16-byte aligned, H % 16 == 0)
+cudaError_t launch_sgate_logits(const uint16_t* x, const moe_qtensor& sgate, int T, int H, float* gs,
+                                cudaStream_t s);
 cudaError_t launch_topk(const float* logits, const float* gs, bool has_sgate, int T, int E, int K, int32_t* idx,
                         float* w, float* sg, cudaStream_t s);
 

@@ -302,8 +302,9 @@ __global__ void __launch_bounds__(kDWarps * 32) down_kernel(Work wk, const __gri
 }
 
 // --------------------------------------------------------------- combine
-// y[t][o] = sum_{k<K} ypart[inv(t,k)][o] + ypart[inv(t,K)][o] (+ residual).
-__global__ void combine_kernel(Work wk, const uint16_t* __restrict__ residual, uint16_t* __restrict__ y) {
+// y[t][o] = sum_{k<K} ypart[inv(t,k)][o] + ypart[inv(t,K)][o] (+ residual), in that order.
+// Any alignment of y: one output per thread.
+__global__ void combine_scalar_kernel(Work wk, const uint16_t* __restrict__ residual, uint16_t* __restrict__ y) {
     const int t = blockIdx.y;
     const int o = blockIdx.x * blockDim.x + threadIdx.x;
     if (o >= wk.H || t >= wk.T) return;
@@ -312,6 +313,43 @@ __global__ void combine_kernel(Work wk, const uint16_t* __restrict__ residual, u
     for (int k = 0; k < kend; ++k) acc += wk.ypart[(int64_t)wk.inv[(int64_t)t * (wk.K + 1) + k] * wk.H + o];
     if (residual) acc += bf16f(residual[(int64_t)t * wk.H + o]);
     y[(int64_t)t * wk.H + o] = f2bf16(acc);
+}
+
+// The same for 8-byte aligned y and residual: a thread takes 4 consecutive outputs, with
+// the loads of all of the token's jobs in flight together.
+__global__ void combine_kernel(Work wk, const uint16_t* __restrict__ residual, uint16_t* __restrict__ y) {
+    const int t = blockIdx.y;
+    const int o4 = blockIdx.x * blockDim.x + threadIdx.x;
+    if (o4 * 4 >= wk.H || t >= wk.T) return;
+    const int kend = wk.K + (wk.Is > 0 ? 1 : 0);
+    float4 v[MOEQ_MAX_TOPK + 1];
+#pragma unroll
+    for (int k = 0; k <= MOEQ_MAX_TOPK; ++k) {
+        v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k < kend) {
+            const int64_t row = wk.inv[(int64_t)t * (wk.K + 1) + k];
+            v[k] = reinterpret_cast<const float4*>(wk.ypart + row * wk.H)[o4];
+        }
+    }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k <= MOEQ_MAX_TOPK; ++k) {
+        if (k >= kend) break;
+        acc.x += v[k].x;
+        acc.y += v[k].y;
+        acc.z += v[k].z;
+        acc.w += v[k].w;
+    }
+    if (residual) {
+        const uint2 r = reinterpret_cast<const uint2*>(residual + (int64_t)t * wk.H)[o4];
+        acc.x += __uint_as_float(r.x << 16);
+        acc.y += __uint_as_float(r.x & 0xFFFF0000u);
+        acc.z += __uint_as_float(r.y << 16);
+        acc.w += __uint_as_float(r.y & 0xFFFF0000u);
+    }
+    const uint2 out = make_uint2((uint32_t)f2bf16(acc.x) | ((uint32_t)f2bf16(acc.y) << 16),
+                                 (uint32_t)f2bf16(acc.z) | ((uint32_t)f2bf16(acc.w) << 16));
+    reinterpret_cast<uint2*>(y + (int64_t)t * wk.H)[o4] = out;
 }
 
 }  // namespace
@@ -363,8 +401,13 @@ cudaError_t launch_down(const Work& wk, const LayerArgs& L, int max_groups, cuda
 
 cudaError_t launch_combine(const Work& wk, const uint16_t* residual, uint16_t* y, cudaStream_t s) {
     if (wk.T == 0) return cudaSuccess;
-    dim3 grid((wk.H + 255) / 256, wk.T);
-    combine_kernel<<<grid, 256, 0, s>>>(wk, residual, y);
+    if (((uintptr_t)y & 7) || ((uintptr_t)residual & 7) || wk.H % 4) {
+        dim3 grid((wk.H + 255) / 256, wk.T);
+        combine_scalar_kernel<<<grid, 256, 0, s>>>(wk, residual, y);
+    } else {
+        dim3 grid((wk.H / 4 + 127) / 128, wk.T);
+        combine_kernel<<<grid, 128, 0, s>>>(wk, residual, y);
+    }
     return cudaGetLastError();
 }
 

@@ -4,26 +4,59 @@
 namespace moeq {
 namespace {
 
-__global__ void rmsnorm_kernel(const uint16_t* __restrict__ x, int H, float eps, uint16_t* __restrict__ xn) {
-    __shared__ float red[32];
-    const int t = blockIdx.x;
-    const uint16_t* xr = x + (int64_t)t * H;
+// One CTA of 256 threads per token; the row comes in 16-byte pieces (8 values), kept in
+// registers between the sum of squares and the scaling (rows up to 8192 values; longer
+// rows re-read the rest).
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict__ x, int H, float eps,
+                                                     uint16_t* __restrict__ xn) {
+    __shared__ float red[8];
+    const int t = blockIdx.x, nv = H / 8;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (int64_t)t * H);
+    uint4* yr = reinterpret_cast<uint4*>(xn + (int64_t)t * H);
+    auto sumsq = [](const uint4& u) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        float ss = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
+            ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+        }
+        return ss;
+    };
+    auto scaled = [](const uint4& u, float inv) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t lo = f2bf16(__uint_as_float(w[k] << 16) * inv);
+            const uint32_t hi = f2bf16(__uint_as_float(w[k] & 0xFFFF0000u) * inv);
+            o[k] = lo | (hi << 16);
+        }
+        return make_uint4(o[0], o[1], o[2], o[3]);
+    };
+    uint4 keep[4];
     float ss = 0.0f;
-    for (int j = threadIdx.x; j < H; j += blockDim.x) {
-        const float v = bf16f(xr[j]);
-        ss = fmaf(v, v, ss);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int v = threadIdx.x + 256 * j;
+        keep[j] = v < nv ? xr[v] : make_uint4(0u, 0u, 0u, 0u);
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) ss += sumsq(keep[j]);
+    for (int v = threadIdx.x + 1024; v < nv; v += 256) ss += sumsq(xr[v]);
     ss = warp_sum(ss);
     if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = ss;
     __syncthreads();
-    if (threadIdx.x < 32) {
-        float v = threadIdx.x < blockDim.x / 32 ? red[threadIdx.x] : 0.0f;
-        v = warp_sum(v);
-        if (threadIdx.x == 0) red[0] = v;
+    float tot = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    const float inv = 1.0f / sqrtf(tot / (float)H + eps);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int v = threadIdx.x + 256 * j;
+        if (v < nv) yr[v] = scaled(keep[j], inv);
     }
-    __syncthreads();
-    const float inv = 1.0f / sqrtf(red[0] / (float)H + eps);
-    for (int j = threadIdx.x; j < H; j += blockDim.x) xn[(int64_t)t * H + j] = f2bf16(bf16f(xr[j]) * inv);
+    for (int v = threadIdx.x + 1024; v < nv; v += 256) yr[v] = scaled(xr[v], inv);
 }
 
 }  // namespace

@@ -77,6 +77,50 @@ router_logits_kernel(const uint16_t* __restrict__ x, moe_qtensor router, moe_qte
     }
 }
 
+// The shared-expert gate alone (the routed logits come from the tensor cores): one warp
+// per token dots the int8 row (H bytes, read from L2) with the token's x, 16 weights per
+// lane and step in 16-byte pieces, every piece of a step in flight together;
+// w = s*q + b in fp32 as in router_logits_kernel.
+__global__ void __launch_bounds__(256) sgate_logits_kernel(const uint16_t* __restrict__ x, moe_qtensor sg, int T,
+                                                           int H, float* __restrict__ gs) {
+    const int t = blockIdx.x * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (t >= T) return;
+    const int nv = H / 16;
+    const uint4* pw = reinterpret_cast<const uint4*>(sg.packed);
+    const uint4* px = reinterpret_cast<const uint4*>(x + (int64_t)t * H);
+    float acc = 0.0f;
+    for (int v0 = lane; v0 < nv; v0 += 32 * 4) {
+        uint4 q[4], xa[4], xb[4];
+        float s[4], b[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int v = v0 + 32 * j;
+            if (v < nv) {
+                q[j] = pw[v];
+                xa[j] = px[2 * v];
+                xb[j] = px[2 * v + 1];
+                const int g = v * 16 / sg.group;
+                s[j] = bf16f(sg.scales[g]);
+                b[j] = bf16f(sg.biases[g]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (v0 + 32 * j >= nv) break;
+            const uint32_t qs[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+            const uint32_t xw[8] = {xa[j].x, xa[j].y, xa[j].z, xa[j].w, xb[j].x, xb[j].y, xb[j].z, xb[j].w};
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float w = __fmaf_rn(s[j], u2f_small((qs[e / 4] >> (8 * (e % 4))) & 0xFFu), b[j]);
+                const float xv = __uint_as_float(e % 2 ? xw[e / 2] & 0xFFFF0000u : xw[e / 2] << 16);
+                acc = fmaf(w, xv, acc);
+            }
+        }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) gs[t] = acc;
+}
+
 // One warp per token: softmax over E logits, K rounds of warp argmax.
 __global__ void topk_kernel(const float* __restrict__ logits, const float* gs, int has_sgate, int T,
                             int E, int K, int32_t* __restrict__ idx, float* __restrict__ w,
@@ -174,6 +218,13 @@ cudaError_t launch_router_logits(const uint16_t* x, const moe_qtensor& router, c
         router_logits_kernel<kRouterTokMax / 2>
             <<<grid, kRouterWarps * 32, smem, s>>>(x, router, sg, has, logit_bias, T, H, E, logits, gs);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sgate_logits(const uint16_t* x, const moe_qtensor& sgate, int T, int H, float* gs,
+                                cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    sgate_logits_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, sgate, T, H, gs);
     return cudaGetLastError();
 }
 
