@@ -315,12 +315,8 @@ __global__ void combine_scalar_kernel(Work wk, const uint16_t* __restrict__ resi
     y[(int64_t)t * wk.H + o] = f2bf16(acc);
 }
 
-// The same for 8-byte aligned y and residual: a thread takes 4 consecutive outputs, with
-// the loads of all of the token's jobs in flight together.
-__global__ void combine_kernel(Work wk, const uint16_t* __restrict__ residual, uint16_t* __restrict__ y) {
-    const int t = blockIdx.y;
-    const int o4 = blockIdx.x * blockDim.x + threadIdx.x;
-    if (o4 * 4 >= wk.H || t >= wk.T) return;
+__device__ __forceinline__ void combine4(const Work& wk, const uint16_t* __restrict__ residual,
+                                         uint16_t* __restrict__ y, int t, int o4) {
     const int kend = wk.K + (wk.Is > 0 ? 1 : 0);
     float4 v[MOEQ_MAX_TOPK + 1];
 #pragma unroll
@@ -351,6 +347,14 @@ __global__ void combine_kernel(Work wk, const uint16_t* __restrict__ residual, u
                                  (uint32_t)f2bf16(acc.z) | ((uint32_t)f2bf16(acc.w) << 16));
     reinterpret_cast<uint2*>(y + (int64_t)t * wk.H)[o4] = out;
 }
+
+// The same for 8-byte aligned y and residual: a thread takes 4 consecutive outputs of one
+// token, with the loads of all of the token's jobs in flight together.
+__global__ void combine_kernel(Work wk, const uint16_t* __restrict__ residual, uint16_t* __restrict__ y) {
+    const int t = blockIdx.y, o4 = blockIdx.x * blockDim.x + threadIdx.x;
+    if (o4 * 4 < wk.H && t < wk.T) combine4(wk, residual, y, t, o4);
+}
+
 
 }  // namespace
 
