@@ -209,6 +209,8 @@ NCU_TRAFFIC = {
     ("prefill", "tc_gate_up"): (333590784 + 9545728, "profiles/tc_gate_up_down_prefill_layer.md"),
     # one launch of the fused decode kernel, one token, top-4
     ("decode_k4", "decode_fused"): (11296000, "profiles/decode_fused_decode_k4.md"),
+    # one gate/up launch of the mixed ternary/4-bit MLP, one token
+    ("mixed_b1", "mixed_gate_up"): (2014976, "profiles/mixed_gate_up_down_mixed_b1.md"),
 }
 
 
@@ -651,9 +653,12 @@ def run_mixed(args, world, rank, local):
     if per:
         dur = kt[dom][0] / kt[dom][1]
         gbs = per / (dur * 1e-3) / 1e9
+        tr = NCU_TRAFFIC.get((args.workload, dom))
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(gbs / hbm, 4), "traffic": None, "peak_source": src, "launch_us": round(dur * 1e3, 3),
-                "bytes_per_launch": per}
+                "frac": round(gbs / hbm, 4), "traffic": tr[0] if tr else None, "peak_source": "%s hbm_gbs" % src,
+                "launch_us": round(dur * 1e3, 3), "bytes_per_launch": per}
+        if tr:
+            roof["traffic_source"] = "ncu capture, " + tr[1]
     step_gbs = L * layer_bytes / (ms_step * 1e-3) / 1e9
     out = {
         "metric": METRIC, "value": round(job_throughput(T, K, world, ms), 2), "unit": "tokens/s", "n_gpus": world,
