@@ -212,7 +212,8 @@ moe_status ws_check(void* ws, size_t ws_bytes, size_t need) {
 // kTcMinTokens tokens on, the gate row then by the CUDA-core kernel alone.
 moe_status router_enqueue(const uint16_t* x, const moe_qtensor& router, const moe_qtensor* sg, const float* lb,
                           int T, int H, int E, float* logits, float* gs, int32_t* status, cudaStream_t s) {
-    if (T >= kTcMinTokens && tc_router_supported(router, H, E)) {
+    // the tensor-core router reads x through a TMA map: 16-byte aligned rows only
+    if (T >= kTcMinTokens && aligned(x, 16) && H % 8 == 0 && tc_router_supported(router, H, E)) {
         LAUNCH(kTcRouterKind, launch_tc_router(router, lb, x, T, H, E, logits, status, s));
         if (sg && aligned(x, 16) && H % 16 == 0) LAUNCH(kRouter, launch_sgate_logits(x, *sg, T, H, gs, s));
         else if (sg) LAUNCH(kRouter, launch_router_logits(x, router, sg, nullptr, T, H, 0, logits, gs, s));

@@ -325,6 +325,59 @@ def test_block_tiny():
         np.max(np.abs(synth.bf16_to_f32(exp))) * 2.0 ** -7
 
 
+def _offset_copy(t):
+    """A copy of t whose data starts 2 bytes past an aligned allocation."""
+    flat = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+    v = flat[1:].view(t.shape)
+    v.copy_(t)
+    return v
+
+
+def test_buffers_two_bytes_off_take_the_element_wise_paths():
+    """The API asks only 2-byte alignment of these buffers: a router input, an RMSNorm input and
+    output, and an FFN output 2 bytes past a 16-byte boundary go through the kernels that read
+    and write element by element, with the same results."""
+    m, ly = _mods()
+    shape, T = workloads.TINY, 20  # enough tokens for the tensor-core path of the aligned case
+    t, L, x, _ = _router_case(shape, 205, T)
+    d = ly.DeviceLayer.from_host(shape, t)
+    xd = ly.to_device(x)
+    xo = _offset_copy(xd)
+    assert xo.data_ptr() % 16 == 2
+    E, K = shape.E, shape.K
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, K), dtype=torch.float32, device="cuda")
+    sg = torch.empty(T, dtype=torch.float32, device="cuda")
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    m.moe_router_topk(xo, d.L.router, d.L.shared_gate, d.t.get("logit_bias"), T, shape.H, E, K, idx, w, sg, logits)
+    torch.cuda.synchronize()
+    y_r, idx_r, w_r, sg_r, logits_r = L.ffn(x)
+    assert np.allclose(logits.cpu().numpy(), logits_r, rtol=1e-5, atol=1e-5)
+    ties = check_routing(idx.cpu().numpy(), idx_r, logits_r, K)
+    assert np.allclose(w.cpu().numpy()[~ties], w_r[~ties], rtol=1e-5, atol=1e-6)
+    assert np.allclose(sg.cpu().numpy(), sg_r, rtol=1e-6, atol=1e-6)
+    # RMSNorm, input and output both off
+    xn = _offset_copy(torch.zeros_like(xd))
+    m.moe_rmsnorm(xo, T, shape.H, 1e-6, xn)
+    torch.cuda.synchronize()
+    got = ly.to_host(xn.contiguous(), np.uint16)
+    exp = oracle.rmsnorm_bf16(x, shape.H, 1e-6)
+    assert np.mean(got == exp) > 0.99
+    assert np.max(np.abs(synth.bf16_to_f32(got).astype(np.float64) - synth.bf16_to_f32(exp))) <= \
+        np.max(np.abs(synth.bf16_to_f32(exp))) * 2.0 ** -7
+    # the FFN output off (x itself must be 16-byte aligned)
+    ws, nb = d.workspace(T)
+    y = _offset_copy(torch.zeros_like(xd))
+    m.moe_ffn_forward(d.L, xd, None, T, y, ws, nb)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status(ws) == 0
+    y_ref = y_r
+    near = near_tie_tokens(logits_r, K)
+    if near.any():
+        y_ref = oracle_for_gpu_routing(L, x, None, idx.cpu().numpy(), logits_r, y_r)
+    assert_close_output(bf16_dev_to_f64(y.contiguous()), y_ref, "ffn, output 2 bytes off")
+
+
 def assert_close_block(out, ref, x):
     """Block outputs are bf16(x + y): equal up to one bf16 step of the sum plus the FFN tolerance."""
     y = ref - x
@@ -404,7 +457,7 @@ def mixed_layer():
     return s, W, q
 
 
-@pytest.mark.parametrize("T", [1, 5, 16])
+@pytest.mark.parametrize("T", [1, 2, 5, 9, 16])
 def test_mixed_linear_full_size(mixed_layer, T):
     m, ly = _mods()
     s, W, q = mixed_layer
