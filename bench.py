@@ -208,7 +208,7 @@ NCU_TRAFFIC = {
     # one gate/up launch over the 2048-token prompt of one layer
     ("prefill", "tc_gate_up"): (333590784 + 9545728, "profiles/tc_gate_up_down_prefill_layer.md"),
     # one launch of the fused decode kernel, one token, top-4
-    ("decode_k4", "decode_fused"): (11296000, "profiles/decode_fused_decode_k4.md"),
+    ("decode_k4", "decode_fused"): (11294208, "profiles/decode_fused_decode_k4.md"),
     # one gate/up launch of the mixed ternary/4-bit MLP, one token
     ("mixed_b1", "mixed_gate_up"): (2014976, "profiles/mixed_gate_up_down_mixed_b1.md"),
 }
