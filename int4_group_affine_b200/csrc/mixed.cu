@@ -1,7 +1,8 @@
-// mixed.cu - a7: EdgeRazor mixed ternary / 4-bit weight-only GEMV/GEMM on CUDA
-// cores.  y_o = s_o * sum_j q_oj x_j: the integer codes are dotted with the
-// activations and the per-row scale is applied once at the end (the weight-only
-// form of the EdgeRazor matmul decomposition).
+// mixed.cu - a7: EdgeRazor mixed ternary / 4-bit weight-only GEMV/GEMM.
+// y_o = s_o * sum_j q_oj x_j: the integer codes are dotted with the activations and
+// the per-row scale is applied once at the end (the weight-only form of the EdgeRazor
+// matmul decomposition).  Up to a few tokens on CUDA cores (below); batches on warp-level
+// tensor-core tiles (further down).
 //
 // Row layout: super-groups of G rows, the first 4-bit (in/8 words, nibble q+8),
 // the rest ternary (in/16 words, 2-bit field q+1).  A warp owns one output row
@@ -235,6 +236,237 @@ size_t stage_bytes(int n, int mt) { return (size_t)mt * n * sizeof(float) + (siz
 
 int mt_for(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : kMT; }
 
+// ------------------------------------------------------------------ batches: mma.sync tiles
+// From kQMinTokens tokens on, the same products on the tensor cores with warp-level
+// mma.sync (m16n8k16, bf16 in, fp32 accumulate): the codes are small integers, exact in
+// bf16, so the tile is q (not s q) and the per-row scale is applied once at the end.  A CTA
+// of kQWarps warps owns 16 output rows; warp w the K slice [w n/kQWarps, (w+1) n/kQWarps);
+// each lane builds its A fragment straight from its two rows' packed words.  The inputs of
+// up to kQTok tokens per pass are staged as bf16 (an fp32 input as two bf16 planes hi and
+// lo = bf16(v - hi), two MMAs into one accumulator, about 16 bits of each value); the
+// warps' partial tiles are added in fixed order in shared memory.  The K loop of a warp is
+// only n/kQWarps long and N is at most 16 tokens: the kernel is bound by issue and latency,
+// not by the tensor pipe, which is why the warp-level MMA serves here.
+constexpr int kQWarps = 16;
+constexpr int kQTok = 16;        // tokens per pass: two n-tiles of 8
+constexpr int kQMinTokens = 4;
+
+enum QMode { kQLinear = 0, kQGateUp = 1, kQDown = 2 };
+
+struct QArgs {
+    moe_mixed_tensor W0, W1;  // the matrix (gate for kQGateUp), and up
+    int G, T;
+    const uint16_t* xb;       // bf16 inputs [T][n] (linear, gate/up)
+    const float* xf;          // fp32 inputs [T][n] (down)
+    float* yf;                // linear: [T][out]; gate/up: h [T][out]
+    uint16_t* yb;             // down: bf16 [T][out]
+    const uint16_t* res;      // down: residual [T][out] or null
+};
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two code fields of t (bits 0.. and bits `step`.., `mask` wide) as the bf16 pair
+// (f0 - off, f1 - off), low half first: the fields go into the mantissa of bf16 128.0
+// (bits 0x4300), whose last mantissa bit counts 1, and 128 + off is subtracted exactly.
+template <int kStep, uint32_t kMask>
+__device__ __forceinline__ uint32_t code_pair(uint32_t t, __nv_bfloat162 sub) {
+    const uint32_t v = (t & kMask) | ((t << (16 - kStep)) & (kMask << 16)) | 0x43004300u;
+    __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(&v);
+    p = __hsub2(p, sub);
+    return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+// This lane's A-fragment pairs of one row for the 4 k16 blocks of a 64-wide K superblock:
+// frag[kb][0] = K (2c, 2c+1), frag[kb][1] = K (2c+8, 2c+9) of block kb (c = lane % 4).
+__device__ __forceinline__ void row_frags(const uint32_t* pw, bool four, int k64, int c, uint32_t (&frag)[4][2]) {
+    if (four) {  // 8 words of 8 nibbles (value + 8)
+        const uint4* v4 = reinterpret_cast<const uint4*>(pw) + k64 * 2;
+        const uint4 u0 = v4[0], u1 = v4[1];
+        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        const __nv_bfloat162 sub = __floats2bfloat162_rn(136.0f, 136.0f);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+            frag[kb][0] = code_pair<4, 0xFu>(w[2 * kb] >> (8 * c), sub);
+            frag[kb][1] = code_pair<4, 0xFu>(w[2 * kb + 1] >> (8 * c), sub);
+        }
+    } else {  // 4 words of 16 two-bit fields (value + 1)
+        const uint4 u = reinterpret_cast<const uint4*>(pw)[k64];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        const __nv_bfloat162 sub = __floats2bfloat162_rn(129.0f, 129.0f);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+            frag[kb][0] = code_pair<2, 0x3u>(w[kb] >> (4 * c), sub);
+            frag[kb][1] = code_pair<2, 0x3u>(w[kb] >> (4 * c + 16), sub);
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t bits_of(__nv_bfloat162 v) { return *reinterpret_cast<const uint32_t*>(&v); }
+
+template <int kMode>
+__global__ void __launch_bounds__(kQWarps * 32) mixed_mma_kernel(const __grid_constant__ QArgs a) {
+    constexpr int kPlanes = kMode == kQDown ? 2 : 1;
+    constexpr int kMats = kMode == kQGateUp ? 2 : 1;
+    extern __shared__ float4 smem_f4[];
+    const int n = a.W0.in, P = n + 8, out = a.W0.out;
+    uint16_t* planes = reinterpret_cast<uint16_t*>(smem_f4);  // [kPlanes][kQTok][P] bf16
+    float* part = reinterpret_cast<float*>(planes + (size_t)kPlanes * kQTok * P);  // [kQWarps][kMats][16][kQTok]
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, g = lane >> 2, c = lane & 3;
+    const int r0 = blockIdx.x * 16, ks = n / kQWarps;
+    const uint32_t* pw[kMats][2];
+    bool four[kMats][2];
+#pragma unroll
+    for (int m = 0; m < kMats; ++m)
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const moe_mixed_tensor& M = m ? a.W1 : a.W0;
+            const int row = r0 + g + 8 * rr;
+            pw[m][rr] = M.packed + mixed_row_offset(row, n, a.G);
+            four[m][rr] = a.G > 0 && row % a.G == 0;
+        }
+    for (int t0 = 0; t0 < a.T; t0 += kQTok) {
+        const int nt = min(kQTok, a.T - t0);
+        __syncthreads();  // the previous pass is done with the planes and the partial tiles
+        if constexpr (kMode == kQDown) {  // fp32 inputs: hi and lo planes, 4 values per piece
+            const int per = n / 4, total = kQTok * per;
+            for (int i0 = threadIdx.x; i0 < total; i0 += 4 * blockDim.x) {
+                float4 v[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + j * blockDim.x, tok = i / per;
+                    v[j] = i < total && tok < nt ? reinterpret_cast<const float4*>(a.xf + (int64_t)(t0 + tok) * n)[i % per]
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + j * blockDim.x;
+                    if (i >= total) break;
+                    const int tok = i / per, q = i % per;
+                    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[j].x, v[j].y);
+                    const __nv_bfloat162 h1 = __floats2bfloat162_rn(v[j].z, v[j].w);
+                    const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+                    const __nv_bfloat162 l0 = __floats2bfloat162_rn(v[j].x - f0.x, v[j].y - f0.y);
+                    const __nv_bfloat162 l1 = __floats2bfloat162_rn(v[j].z - f1.x, v[j].w - f1.y);
+                    reinterpret_cast<uint2*>(planes + (size_t)tok * P)[q] = make_uint2(bits_of(h0), bits_of(h1));
+                    reinterpret_cast<uint2*>(planes + (size_t)(kQTok + tok) * P)[q] = make_uint2(bits_of(l0), bits_of(l1));
+                }
+            }
+        } else {  // bf16 inputs, 8 values per piece
+            const int per = n / 8, total = kQTok * per;
+            for (int i0 = threadIdx.x; i0 < total; i0 += 4 * blockDim.x) {
+                uint4 v[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + j * blockDim.x, tok = i / per;
+                    v[j] = i < total && tok < nt ? reinterpret_cast<const uint4*>(a.xb + (int64_t)(t0 + tok) * n)[i % per]
+                                                 : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + j * blockDim.x;
+                    if (i >= total) break;
+                    reinterpret_cast<uint4*>(planes + (size_t)(i / per) * P)[i % per] = v[j];
+                }
+            }
+        }
+        __syncthreads();
+        float acc[kMats][2][4];
+#pragma unroll
+        for (int m = 0; m < kMats; ++m)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[m][j][e] = 0.0f;
+        for (int s = 0; s < ks / 64; ++s) {
+            const int k64 = warp * (ks / 64) + s;  // 64-wide K superblock of the row
+            uint32_t fa[kMats][2][4][2];
+#pragma unroll
+            for (int m = 0; m < kMats; ++m)
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) row_frags(pw[m][rr], four[m][rr], k64, c, fa[m][rr]);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+                const int k = k64 * 64 + 16 * kb + 2 * c;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                    for (int pl = 0; pl < kPlanes; ++pl) {
+                        const uint16_t* bp = planes + (size_t)(pl * kQTok + 8 * j + g) * P + k;
+                        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(bp);
+                        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(bp + 8);
+#pragma unroll
+                        for (int m = 0; m < kMats; ++m)
+                            mma_bf16_16816(acc[m][j], fa[m][0][kb][0], fa[m][1][kb][0], fa[m][0][kb][1], fa[m][1][kb][1],
+                                           b0, b1);
+                    }
+                }
+            }
+        }
+        // this warp's partial tile: rows g, g + 8, tokens 8 j + 2 c, + 1
+#pragma unroll
+        for (int m = 0; m < kMats; ++m)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float* pp = part + ((size_t)(warp * kMats + m) * 16 + g) * kQTok + 8 * j + 2 * c;
+                pp[0] = acc[m][j][0];
+                pp[1] = acc[m][j][1];
+                pp[8 * kQTok] = acc[m][j][2];
+                pp[8 * kQTok + 1] = acc[m][j][3];
+            }
+        __syncthreads();
+        // the warps' partials in fixed order, the row scale and the epilogue: thread (row, token)
+        for (int q = threadIdx.x; q < 16 * kQTok; q += blockDim.x) {
+            const int row = q / kQTok, tok = q % kQTok, o = r0 + row;
+            if (tok >= nt) continue;
+            float v[kMats];
+#pragma unroll
+            for (int m = 0; m < kMats; ++m) {
+                float sm = 0.0f;
+                for (int w = 0; w < kQWarps; ++w) sm += part[((size_t)(w * kMats + m) * 16 + row) * kQTok + tok];
+                v[m] = sm * bf16f((m ? a.W1 : a.W0).scales[o]);
+            }
+            const int64_t i = (int64_t)(t0 + tok) * out + o;
+            if constexpr (kMode == kQLinear) {
+                a.yf[i] = v[0];
+            } else if constexpr (kMode == kQGateUp) {
+                a.yf[i] = silu(v[0]) * v[kMats - 1];
+            } else {
+                a.yb[i] = f2bf16(v[0] + (a.res ? bf16f(a.res[i]) : 0.0f));
+            }
+        }
+    }
+}
+
+size_t mma_smem(int mode, int n) {
+    const int planes = mode == kQDown ? 2 : 1, mats = mode == kQGateUp ? 2 : 1;
+    return (size_t)planes * kQTok * (n + 8) * 2 + (size_t)kQWarps * mats * 16 * kQTok * 4;
+}
+
+// The tensor-core path applies: enough tokens, K a multiple of 64 per warp, whole 16-row
+// tiles, 16-byte aligned packed rows and inputs, and the staging fits in shared memory.
+bool mma_ok(int mode, const moe_mixed_tensor& W, const void* in, int T) {
+    if (T < kQMinTokens || W.in % (64 * kQWarps) || W.out % 16) return false;
+    if (((uintptr_t)W.packed & 15) || ((uintptr_t)in & 15)) return false;
+    return mma_smem(mode, W.in) <= 220 * 1024;
+}
+
+template <int kMode>
+cudaError_t launch_mma(const QArgs& a, cudaStream_t s) {
+    static int cached = 0;
+    const size_t smem = mma_smem(kMode, a.W0.in);
+    cudaError_t e = ensure_smem((const void*)mixed_mma_kernel<kMode>, smem, cached);
+    if (e != cudaSuccess) return e;
+    mixed_mma_kernel<kMode><<<a.W0.out / 16, kQWarps * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 #define MOEQ_MIXED_DISPATCH(MTV, CALL) \
@@ -247,6 +479,15 @@ int mt_for(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : kMT; }
 
 cudaError_t launch_mixed_linear(const moe_mixed_tensor& W, int G, const uint16_t* x, int T, float* y, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
+    if (mma_ok(kQLinear, W, x, T)) {
+        QArgs a = {};
+        a.W0 = W;
+        a.G = G;
+        a.T = T;
+        a.xb = x;
+        a.yf = y;
+        return launch_mma<kQLinear>(a, s);
+    }
     const int mt = mt_for(T);
     const size_t smem = stage_bytes(W.in, mt);
     cudaError_t e = cudaSuccess;
@@ -266,6 +507,16 @@ cudaError_t launch_mixed_linear(const moe_mixed_tensor& W, int G, const uint16_t
 cudaError_t launch_mixed_gate_up(const moe_mixed_tensor& g, const moe_mixed_tensor& u, int G, const uint16_t* x,
                                  int T, float* h, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
+    if (mma_ok(kQGateUp, g, x, T) && ((uintptr_t)u.packed & 15) == 0) {
+        QArgs a = {};
+        a.W0 = g;
+        a.W1 = u;
+        a.G = G;
+        a.T = T;
+        a.xb = x;
+        a.yf = h;
+        return launch_mma<kQGateUp>(a, s);
+    }
     const int mt = mt_for(T);
     const size_t smem = stage_bytes(g.in, mt);
     cudaError_t e = cudaSuccess;
@@ -285,6 +536,16 @@ cudaError_t launch_mixed_gate_up(const moe_mixed_tensor& g, const moe_mixed_tens
 cudaError_t launch_mixed_down(const moe_mixed_tensor& d, int G, const float* h, int T, const uint16_t* residual,
                               uint16_t* y, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
+    if (mma_ok(kQDown, d, h, T)) {
+        QArgs a = {};
+        a.W0 = d;
+        a.G = G;
+        a.T = T;
+        a.xf = h;
+        a.yb = y;
+        a.res = residual;
+        return launch_mma<kQDown>(a, s);
+    }
     const int mt = mt_for(T);
     const size_t smem = stage_bytes(d.in, mt);
     cudaError_t e = cudaSuccess;
