@@ -16,7 +16,7 @@ using namespace moeq;
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kTcMinTokens = 16;  // from this many tokens on, the expert GEMMs use the tensor cores
+constexpr int kTcMinTokens = 9;  // from this many tokens on, the expert GEMMs use the tensor cores
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 

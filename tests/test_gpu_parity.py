@@ -216,7 +216,7 @@ def _check_ffn(shape, t, x, aid, n_adapters=None, what=""):
     return assert_close_output(y, y_ref, what), y, y_ref
 
 
-@pytest.mark.parametrize("T", [4, 1, 37, 70])
+@pytest.mark.parametrize("T", [4, 1, 12, 37, 70])
 def test_ffn_tiny(T):
     shape = workloads.TINY
     t, x, aid = _ffn_case(shape, 400, T=T)
