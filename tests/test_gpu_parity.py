@@ -457,7 +457,7 @@ def mixed_layer():
     return s, W, q
 
 
-@pytest.mark.parametrize("T", [1, 2, 5, 9, 16])
+@pytest.mark.parametrize("T", [1, 2, 5, 9, 16, 20])
 def test_mixed_linear_full_size(mixed_layer, T):
     m, ly = _mods()
     s, W, q = mixed_layer
