@@ -73,56 +73,97 @@ def measured_peaks():
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples (200 ms) taken while the timed region runs."""
+    """SM clock and throttle reasons sampled while the timed region runs.
 
+    NVML is read every 5 ms from a thread, so that a timed region of a few tens of
+    milliseconds still holds several samples; the GPU is found by its PCI address, which
+    CUDA_VISIBLE_DEVICES does not renumber.  Without NVML, nvidia-smi samples every 200 ms.
+    Reads only: no setting of the GPU is touched.
+    """
+
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.005
 
-    def __init__(self, gpu_index):
-        self.samples = []
+    def __init__(self, cuda_index):
+        self.samples = []  # (wall time, sm MHz, max sm MHz, set of active reasons)
         self.proc = None
-        self.gpu = gpu_index
+        self.source = None
+        self._halt = threading.Event()
+        target = None
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            handle = self._nvml_handle(pynvml, cuda_index)
+            bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap)
+            smax = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+            target = lambda: self._poll_nvml(pynvml, handle, bits, smax)  # noqa: E731
+            self.source = "nvml every %g ms" % (1e3 * self.PERIOD_S)
+        except Exception:
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", str(cuda_index), "--query-gpu=" + self.FIELDS,
+                                              "--format=csv,noheader,nounits", "-lms", "200"],
+                                             stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                return
+            target = self._read_smi
+            self.source = "nvidia-smi every 200 ms"
+        self.thread = threading.Thread(target=target, daemon=True)
         self.thread.start()
 
-    def _read(self):
+    @staticmethod
+    def _nvml_handle(pynvml, cuda_index):
+        try:
+            import torch
+            pr = torch.cuda.get_device_properties(cuda_index)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(
+                "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id))
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+
+    def _poll_nvml(self, pynvml, handle, bits, smax):
+        while not self._halt.is_set():
+            try:
+                sm = float(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM))
+                mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+            except Exception:
+                return
+            self.samples.append((time.time(), sm, smax, {n for n, b in zip(self.NAMES, bits) if mask & b}))
+            self._halt.wait(self.PERIOD_S)
+
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.samples.append((time.time(), [c.strip() for c in line.split(",")]))
+            c = [f.strip() for f in line.split(",")]
+            try:
+                sm, smax = float(c[1]), float(c[2])
+            except (ValueError, IndexError):
+                continue
+            self.samples.append((time.time(), sm, smax,
+                                 {n for n, v in zip(self.NAMES, c[5:9]) if v.lower().startswith("active")}))
 
     def stop(self):
+        self._halt.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if getattr(self, "thread", None) is not None:
+            self.thread.join(timeout=5)
 
     def summary(self, t0, t1):
-        inside = [s for t, s in self.samples if t0 <= t <= t1]
-        used = inside if inside else [s for _, s in self.samples]
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        used = inside if inside else self.samples
         if not used:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        sm, smax, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for s in used:
-            try:
-                sm.append(float(s[1]))
-                smax.append(float(s[2]))
-            except (ValueError, IndexError):
-                continue
-            for n, v in zip(names, s[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(inside),
-                "window": "timed region" if inside else "whole run (timed region shorter than one sample)"}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        return {"sm_mhz": statistics.median(s[1] for s in used), "sm_max_mhz": max(s[2] for s in used),
+                "reasons": sorted(set().union(*(s[3] for s in used))), "samples": len(inside),
+                "window": "timed region" if inside else "whole run (timed region shorter than one sample)",
+                "source": self.source}
 
 
 # ----------------------------------------------------------------- byte / flop accounting
