@@ -242,9 +242,9 @@ moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* ada
         // the int4 tiles hold each 8-group of K in the order 0 4 1 5 2 6 3 7: the gate/up
         // operand is x in that order, and h is written in it for the down GEMM
         LAUNCH(kKpermKind, launch_kperm(x, (int64_t)T * la.H, wk.xp, s));
-        if (la.rank > 0) LAUNCH(kTcLoraGUKind, launch_tc_gemm(la, kTcLoraGU, x, la.H, wk, nullptr, wk.Imax, s));
+        if (la.rank > 0) LAUNCH(kTcLoraGUKind, launch_lora_a_mma(la, 0, x, la.H, wk, s));
         LAUNCH(kTcGUKind, launch_tc_gemm(la, kTcGU, wk.xp, la.H, wk, hb, wk.Imax, s));
-        if (la.rank > 0) LAUNCH(kTcLoraDownKind, launch_tc_gemm(la, kTcLoraDown, hb, wk.Imax, wk, nullptr, wk.Imax, s));
+        if (la.rank > 0) LAUNCH(kTcLoraDownKind, launch_lora_a_mma(la, 1, hb, wk.Imax, wk, s));
         LAUNCH(kTcDownKind, launch_tc_gemm(la, kTcDown, hb, wk.Imax, wk, nullptr, wk.Imax, s));
         LAUNCH(kCombine, launch_combine(wk, residual, y, s));
         return MOE_OK;

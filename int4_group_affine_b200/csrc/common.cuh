@@ -136,6 +136,10 @@ cudaError_t launch_index_build_counts(const Work& wk, const int32_t* adapter_id,
                                       int32_t* counts_out, cudaStream_t s);
 
 cudaError_t launch_lora_a(const Work& wk, const LayerArgs& L, int phase, const uint16_t* x, cudaStream_t s);
+// LoRA-A products of the expert-grouped jobs on mma.sync tiles (down = 0: [J][2r] from x
+// by token; down = 1: [J][r] from the bf16 h rows of the jobs, stored in the int4 tiles' K order)
+cudaError_t launch_lora_a_mma(const LayerArgs& L, int down, const uint16_t* act, int ld, const Work& wk,
+                              cudaStream_t s);
 cudaError_t launch_gate_up(const Work& wk, const LayerArgs& L, const uint16_t* x, int max_groups, cudaStream_t s);
 cudaError_t launch_down(const Work& wk, const LayerArgs& L, int max_groups, cudaStream_t s);
 cudaError_t launch_combine(const Work& wk, const uint16_t* residual, uint16_t* y, cudaStream_t s);
