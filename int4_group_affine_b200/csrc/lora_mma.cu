@@ -54,7 +54,7 @@ __device__ __forceinline__ const moe_lora_proj* lora_rows(const LayerArgs& L, in
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -68,6 +68,15 @@ __device__ __forceinline__ uint4 to_tile_order(uint4 u) {
 }
 
 __device__ __forceinline__ uint4 ld16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+// Bring [p, p + bytes) into L2 without waiting (bulk prefetch; p and bytes multiples of 16)
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    for (uint32_t o = 0; o < bytes; o += 65536u) {
+        const uint32_t n = bytes - o < 65536u ? bytes - o : 65536u;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<const char*>(p) + o), "r"(n)
+                     : "memory");
+    }
+}
 
 __device__ __forceinline__ int pow2_ceil4(int v) { return v <= 1 ? 1 : v <= 2 ? 2 : 4; }
 
@@ -120,6 +129,31 @@ __global__ void __launch_bounds__(kLWarps * 32, 1) lora_a_mma_kernel(const __gri
         const int nj = min(kLJobs, s_goff[grp + 1] - j0);
         const int K = a.down ? (shared ? L.Is : L.I) : L.H;
         const int nch = K / 32;
+        if (!a.down && L.n_adapters == 1 && (threadIdx.x == 32 || threadIdx.x == 33)) {
+            // one adapter: the A blocks of this item and of this CTA's next item start towards L2
+            // before the job list is read (the down products read h, which is still in L2)
+            int g2 = grp;
+            if (threadIdx.x == 33) {
+                const int nx = it + (int)gridDim.x;
+                g2 = -1;
+                if (nx < total) {
+                    int l2 = 0, h2 = E;
+                    while (l2 < h2) {
+                        const int mid = (l2 + h2 + 1) / 2;
+                        if (s_pre[mid] <= nx) l2 = mid;
+                        else h2 = mid - 1;
+                    }
+                    g2 = l2;
+                    const int jn = s_goff[g2] + (nx - s_pre[g2]) * kLJobs;
+                    prefetch_l2(a.perm + jn, (uint32_t)min(kLJobs, s_goff[g2 + 1] - jn) * 16u);
+                }
+            }
+            if (g2 >= 0)
+                for (int which = 0; which < 2; ++which) {
+                    const moe_lora_proj* lp = lora_rows(L, 0, g2 == E, which);
+                    if (lp) prefetch_l2(lp->A + (int64_t)(g2 == E ? 0 : g2) * r * L.H, (uint32_t)r * L.H * 2);
+                }
+        }
         __syncthreads();  // the previous item is done with s_z and s_part
         if (threadIdx.x < kLJobs) {
             int tok = 0, z = -1;
@@ -139,6 +173,18 @@ __global__ void __launch_bounds__(kLWarps * 32, 1) lora_a_mma_kernel(const __gri
         const int zf = s_z[0], zl = s_z[nj - 1];
         const int ad_lo = (zf < 0 || zf >= L.n_adapters) ? L.n_adapters : zf;
         const int ad_hi = (zl < 0 || zl >= L.n_adapters) ? L.n_adapters - 1 : zl;
+        if (!a.down) {
+            // gate/up: the x rows of the jobs and (several adapters) every present adapter's A
+            // blocks start towards L2 together, so the K loops below mostly wait on L2, not HBM
+            const int t = threadIdx.x;
+            const int npf = L.n_adapters > 1 ? 2 * (ad_hi - ad_lo + 1) : 0;
+            if (t < npf) {
+                const moe_lora_proj* lp = lora_rows(L, ad_lo + t / 2, shared, t % 2);
+                if (lp) prefetch_l2(lp->A + (int64_t)(shared ? 0 : grp) * r * K, (uint32_t)r * K * 2);
+            } else if (t >= 64 && t < 64 + nj) {
+                prefetch_l2(a.act + (int64_t)s_tok[t - 64] * a.ld, (uint32_t)K * 2);
+            }
+        }
 
         for (int ad = ad_lo; ad <= ad_hi; ++ad) {
             // this adapter's jobs: a contiguous run [jlo, jlo + na) of the item ("none" sorts last)
@@ -187,15 +233,23 @@ __global__ void __launch_bounds__(kLWarps * 32, 1) lora_a_mma_kernel(const __gri
 #pragma unroll
                         for (int t = 0; t < 4; ++t) wv[u][t] = live && wr[t] ? ld16(wr[t] + off) : z4;
                     }
+                    if (a.down)
 #pragma unroll
-                    for (int u = 0; u < kLUnroll; ++u)
+                        for (int u = 0; u < kLUnroll; ++u)
 #pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            if (kLCols * ngi + 8 * t >= R) continue;  // n8 tile past the rows (warp-uniform)
-                            const uint4 w = a.down ? to_tile_order(wv[u][t]) : wv[u][t];
-                            mma16816(acc[t], xa[u].x, xb[u].x, xa[u].y, xb[u].y, w.x, w.y);
-                            mma16816(acc[t], xa[u].z, xb[u].z, xa[u].w, xb[u].w, w.z, w.w);
-                        }
+                            for (int t = 0; t < 4; ++t) wv[u][t] = to_tile_order(wv[u][t]);
+                    // consecutive MMAs go to different accumulators
+#pragma unroll
+                    for (int u = 0; u < kLUnroll; ++u) {
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            if (kLCols * ngi + 8 * t < R)  // n8 tile inside the rows (warp-uniform)
+                                mma16816(acc[t], xa[u].x, xb[u].x, xa[u].y, xb[u].y, wv[u][t].x, wv[u][t].y);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            if (kLCols * ngi + 8 * t < R)
+                                mma16816(acc[t], xa[u].z, xb[u].z, xa[u].w, xb[u].w, wv[u][t].z, wv[u][t].w);
+                    }
                 }
                 // partial tile: rows g and g + 8 of the m tile, columns 8 t + 2 c (+1) of the row group
 #pragma unroll
