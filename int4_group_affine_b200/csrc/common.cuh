@@ -147,7 +147,7 @@ cudaError_t launch_combine(const Work& wk, const uint16_t* residual, uint16_t* y
 cudaError_t launch_rmsnorm(const uint16_t* x, int T, int H, float eps, uint16_t* xn, cudaStream_t s);
 
 // tcgen05 grouped GEMM modes (csrc/prefill.cu)
-enum TcMode { kTcGU = 0, kTcDown = 1, kTcLoraGU = 2, kTcLoraDown = 3 };
+enum TcMode { kTcGU = 0, kTcDown = 1 };
 bool tc_supported(const LayerArgs& L);
 cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, int ld_act, const Work& wk,
                            const uint16_t* hb_out, int ldh, cudaStream_t s);

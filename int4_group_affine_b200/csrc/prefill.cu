@@ -1,6 +1,7 @@
 // prefill.cu - expert-grouped GEMMs on the tcgen05 tensor cores (sm_100a) for
-// the many-token case: the 8-bit router, gate/up with fused SwiGLU, down with
-// the routing weight, and the two LoRA-A products.
+// the many-token case: the 8-bit router, gate/up with fused SwiGLU and down with
+// the routing weight, each with its LoRA-B term (the LoRA-A products come from
+// warp-level tiles, lora_mma.cu).
 //
 // Swap-AB: a tile is weight rows (M = 128 per block, one TMEM lane each) by up
 // to 64 jobs of one expert group (N), over K in steps of 128 (two 64-wide
@@ -23,8 +24,7 @@
 // Activations (operand B) fill a K-major 128-byte-swizzled ring of four slots,
 // two steps ahead of the dequantisation: TMA boxes where the rows are contiguous
 // (the h rows of the jobs for down, the tokens for the router), cp.async by the
-// loader's lanes where they are scattered (gate/up gathers x by token) or come
-// with adapter rows (LoRA-A).  One lane of the MMA warp issues the MMAs (8 x
+// loader's lanes where they are scattered (gate/up gathers x by token).  One lane of the MMA warp issues the MMAs (8 x
 // K=16 per block per step) and commits them to per-step mbarriers; accumulators
 // are double-buffered in TMEM and each item's epilogue runs a few steps after its
 // last MMA, so the dequantisation never waits on the tensor core at item ends.
@@ -45,11 +45,9 @@
 //   router:  int8 rows; block 0 = bf16(w), block 1 = bf16(w - bf16(w)), both
 //            into one accumulator, so the logits carry ~16 bits of each weight;
 //            epilogue adds the logit bias -> logits.
-//   LoRA-A:  bf16 A rows of every adapter, copied by cp.async straight into the
-//            swizzled operand layout, 64 real rows per tile.
 //
 // Warp roles: 8 dequantisation warps (scales, dequant, LoRA-B operand, epilogue),
-// one MMA warp and one loader warp (weight spans, activations, LoRA rows); they
+// one MMA warp and one loader warp (weight spans, activations, LoRA-B rows); they
 // hand steps over through mbarriers, so no CTA-wide barrier sits in the K loop.
 // Every wait is bounded in time and raises MOE_ERR_TIMEOUT when it gives up.
 // Persistent grid: CTA c takes items c, c + grid, ...
@@ -76,15 +74,12 @@ constexpr int kSpanBytes = kBM * 128;             // one block of one span: 128 
 constexpr int kRawSlot = 2 * kSpanBytes;          // two blocks
 constexpr int kSub = kNT * 128;                   // one 64-wide K sub-tile of 64 rows (128 B per row)
 constexpr int kBSlot = 2 * kSub;                  // activation ring slot: the step's two sub-tiles
-constexpr int kLoraRows = 64;                     // real LoRA-A rows per M tile
-constexpr int kLoraSlot = 2 * kLoraRows * 128;    // LoRA-A ring slot: two sub-tiles of 64 rows
 constexpr int kMaxGroups = MOEQ_MAX_EXPERTS + 1;
 // TMEM columns: accumulator D(buffer b, block k) at 128 b + 64 k; A stage s, block k at 256 + 128 s + 64 k
 constexpr uint32_t kTmemA = 256;
-static_assert(kRB * kLoraSlot <= kRS * kRawSlot, "LoRA-A ring must fit in the weight ring");
 static_assert(kTmemA + kAS * 128 <= 512, "TMEM columns");
 
-enum Mode { kGU = 0, kDown = 1, kLoraGU = 2, kLoraDown = 3, kRouterMode = 4 };
+enum Mode { kGU = 0, kDown = 1, kRouterMode = 4 };
 
 struct TcArgs {
     CUtensorMap tm[4];    // weight words: gate/up {gate, up, s_gate, s_up}; down {down, s_down}; router {router}
@@ -100,7 +95,6 @@ struct TcArgs {
     uint16_t* h_out;      // gate/up: [J][ldh] bf16
     int ldh;
     float* ypart;         // down: [J][H]
-    float* t_out;         // LoRA-A gate/up: [J][2r], LoRA-A down: [J][r]
     const float* t_in;    // gate/up: [J][2r], down: [J][r]
     float* logits;        // router: [T][E]
     int T;                // router: tokens
@@ -113,7 +107,7 @@ struct Geo {  // one expert group's geometry in the current mode
 };
 
 __device__ __forceinline__ int rows_per_item(int mode) {
-    return mode == kDown ? 2 * kBM : (mode == kLoraGU || mode == kLoraDown) ? kLoraRows : kBM;
+    return mode == kDown ? 2 * kBM : kBM;
 }
 
 __device__ __forceinline__ Geo geo_of(const TcArgs& a, int mode, int g, int count) {
@@ -127,8 +121,6 @@ __device__ __forceinline__ Geo geo_of(const TcArgs& a, int mode, int g, int coun
     switch (mode) {
         case kGU: q.M = I; q.K = L.H; break;
         case kDown: q.M = L.H; q.K = I; break;
-        case kLoraGU: q.M = L.n_adapters * 2 * r; q.K = L.H; break;
-        case kLoraDown: q.M = L.n_adapters * r; q.K = I; break;
         default: q.M = L.E; q.K = L.H; q.mat = 0; break;
     }
     if (q.M <= 0) q.skip = true;
@@ -232,7 +224,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     const LayerArgs& L = a.L;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     constexpr int mode = kMode;
-    constexpr bool lora_mode = mode == kLoraGU || mode == kLoraDown;
     // activation tiles by TMA boxes (rows contiguous in the activation matrix); the gate/up
     // rows are tokens scattered over x and the LoRA-A modes add the adapters' rows: cp.async
     constexpr bool tma_b = mode == kDown || mode == kRouterMode;
@@ -326,14 +317,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     auto tile_jobs = [&](const Pos& p) { return min(kNT, s_goff[p.g + 1] - s_goff[p.g] - p.nt * kNT); };
     auto geo = [&](const Pos& p) { return geo_of(a, mode, p.g, s_goff[p.g + 1] - s_goff[p.g]); };
     // a step opens a span of the weight ring: every LoRA-B step, and every SP-th weight step
-    auto opens = [&](const Pos& p) { return !lora_mode && (p.kt >= p.KW || p.kt % SP == 0); };
+    auto opens = [&](const Pos& p) { return p.kt >= p.KW || p.kt % SP == 0; };
     auto advance = [&](Pos& p) {
         if (++p.kt == p.KT) decode(p.item + NB, p);
     };
 
     if (warp == kLoadWarp) {
         // ====================================================== loader warp: TMA spans, activation rows,
-        // LoRA rows.  It runs ahead of the MMAs by up to kRB steps (activation slots) and of the
+        // LoRA-B rows.  It runs ahead of the MMAs by up to kRB steps (activation slots) and of the
         // dequantisation by up to kRS spans (weight ring).
         Pos pl;
         decode(blockIdx.x, pl);
@@ -346,10 +337,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const int c8 = lane % 8, r0 = lane / 8;
         int64_t rowoff[16];
         uint32_t rowlive = 0;
-        const uint16_t* lrow[16];
         auto item_rows = [&](const Pos& p) {
             if (tma_b) return;
-            constexpr bool by_token = mode == kGU || mode == kLoraGU;
+            constexpr bool by_token = mode == kGU;
             const int base = s_goff[p.g] + p.nt * kNT, end = s_goff[p.g + 1];
             const Geo q = geo(p);
             rowlive = 0;
@@ -359,17 +349,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const bool live = p.item < nitems && job < end;
                 rowoff[i] = live ? (int64_t)(by_token ? a.perm[job].x : job) * a.ld_act + c8 * 8 : 0;
                 if (live) rowlive |= 1u << i;
-                lrow[i] = nullptr;
-                if (lora_mode && p.item < nitems) {
-                    const int rpa = mode == kLoraGU ? 2 * r : r;
-                    const int R = p.mt * kLoraRows + r0 + 4 * i;
-                    if (R < q.M) {
-                        const int ad = R / rpa, d = R % rpa;
-                        const int which = mode == kLoraGU ? (d < r ? 0 : 1) : 2;
-                        const moe_lora_proj* lp = tlora(L, ad, q.shared, which);
-                        if (lp) lrow[i] = lp->A + ((int64_t)q.mat * r + (mode == kLoraGU ? d % r : d)) * q.K + c8 * 8;
-                    }
-                }
             }
         };
         item_rows(pl);
@@ -454,7 +433,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 if (lane < 2)
                     tc::tma_load_2d(bb + lane * kSub, &a.tmb, pl.kt * kKS + 64 * lane, s_goff[pl.g] + pl.nt * kNT, bar);
                 if (lane != 0) tc::mbar_arrive(bar);
-            } else if (wstep || lora_mode) {
+            } else if (wstep) {
                 const uint32_t bb = tc::smem_u32(sB + bslot * kBSlot);
                 const int k0 = pl.kt * kKS;
 #pragma unroll
@@ -465,15 +444,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         tc::cp16(bb + sub * kSub + tc::sw128_off(r0 + 4 * i, c8),
                                  a.act + (live ? rowoff[i] + k0 + 64 * sub : 0), live ? 16u : 0u);
                     }
-                if (lora_mode) {  // LoRA-A rows straight into the MMA's swizzled operand layout
-                    const uint32_t rb = tc::smem_u32(sR + bslot * kLoraSlot);
-#pragma unroll
-                    for (int sub = 0; sub < 2; ++sub)
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            tc::cp16(rb + sub * (kLoraRows * 128) + tc::sw128_off(r0 + 4 * i, c8),
-                                     lrow[i] ? lrow[i] + k0 + 64 * sub : a.act, lrow[i] ? 16u : 0u);
-                }
                 tc::cp_commit();
                 tc::cp_arrive_noinc(&bar_bfull[bslot]);
             } else {
@@ -482,7 +452,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             ++t;
             const int item0 = pl.item;
             advance(pl);
-            if (!lora_mode && pl.item < nitems && opens(pl)) ++cs;
+            if (pl.item < nitems && opens(pl)) ++cs;
             if (pl.item != item0) item_rows(pl);
         }
         // drain (bounded): this warp's copies; the latest span issued into each slot
@@ -517,23 +487,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const bool wstep = pc.kt < pc.KW;
                 if (!tc::mbar_spin_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok) ||
                     !tc::mbar_spin_ok(&bar_bfull[t % kRB], (t / kRB) & 1u, a.status, &s_ok) ||
-                    (!lora_mode && !wstep && !tc::mbar_spin_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok))) {
+                    (!wstep && !tc::mbar_spin_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok))) {
                     ok = false;
                     break;
                 }
                 tc::tc_fence_after();
                 const uint32_t dacc = tmem + (ib & 1u) * 128u;
                 const int b = t % kRB;
-                if (lora_mode) {  // A: the LoRA-A rows, copied swizzled into the ring
-                    const uint32_t aslot = tc::smem_u32(sR + b * kLoraSlot);
-#pragma unroll
-                    for (int sub = 0; sub < 2; ++sub) {
-                        const uint64_t ad = tc::sdesc_k_sw128(aslot + sub * (kLoraRows * 128));
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            tc::mma_bf16(dacc, ad + 2 * k, bdesc(b, sub) + 2 * k, idesc, (pc.kt > 0 || sub > 0 || k > 0) ? 1u : 0u);
-                    }
-                } else if (!wstep) {  // LoRA-B step: A = LoRA-B rows of the pseudo-span, one accumulator per block
+                if (!wstep) {  // LoRA-B step: A = LoRA-B rows of the pseudo-span, one accumulator per block
                     const uint32_t rs = tc::smem_u32(sR + (cs % kRS) * kRawSlot);
 #pragma unroll
                     for (int blk = 0; blk < 2; ++blk) {
@@ -564,7 +525,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 if (last) ++ib;
                 advance(pc);
                 if (last && pc.item < nitems) idesc = tc::idesc_bf16(kBM, (tile_jobs(pc) + 15) / 16 * 16);
-                if (!lora_mode && pc.item < nitems && opens(pc)) ++cs;
+                if (pc.item < nitems && opens(pc)) ++cs;
             }
             // drain (bounded): the last MMAs
             if (t > 0) tc::mbar_wait(&bar_tile[(t - 1) % kTiles], ((t - 1) / kTiles) & 1u, a.status);
@@ -698,7 +659,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                             if (o0 + kBM < q.M) yp[o0 + kBM] = wj * __uint_as_float(d1[c]);
                         }
                     }
-                } else if (int8_mode) {
+                } else {  // router
                     const int e = p.mt * kBM + row;
                     if (e < q.M) {
                         const float lb = L.logit_bias ? L.logit_bias[e] : 0.0f;
@@ -706,18 +667,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         for (int c = 0; c < 16; ++c) {
                             const int n = ch * 16 + c;
                             if (n < n_here) a.logits[(int64_t)(base + n) * L.E + e] = __uint_as_float(d0[c]) + lb;
-                        }
-                    }
-                } else {
-                    const int rpa = mode == kLoraGU ? 2 * r : r;
-                    const int R = p.mt * kLoraRows + row;
-                    if (row < kLoraRows && R < q.M) {
-                        const int ad = R / rpa, d = R % rpa;
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const int n = ch * 16 + c;
-                            if (n < n_here && __ldg(&a.perm[base + n].z) == ad)
-                                a.t_out[(int64_t)(base + n) * rpa + d] = __uint_as_float(d0[c]);
                         }
                     }
                 }
@@ -742,7 +691,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 pn_span = 0;
             }
         };
-        if (!lora_mode) sb_next();
+        sb_next();
         uint32_t ss0[4] = {0, 0, 0, 0}, sb0[4] = {0, 0, 0, 0}, ss1[4] = {0, 0, 0, 0}, sb1[4] = {0, 0, 0, 0};
         LoraRegs lr;
         // the epilogue of an item runs kAS steps after its last step, when its MMAs are done
@@ -756,7 +705,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         bool good = true;
         while (pc.item < nitems) {
             const bool wstep = pc.kt < pc.KW;
-            const bool span_start = !lora_mode && wstep && pc.kt % SP == 0;
+            const bool span_start = wstep && pc.kt % SP == 0;
             // the MMAs of step t - kAS must be done before TMEM stage t % kAS (and, for a LoRA-B
             // step, activation slot t % kRB) is rewritten
             if (t >= (uint32_t)kAS &&
@@ -790,21 +739,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 good = false;
                 break;
             }
-            if (mode == kLoraDown) {  // the LoRA-A rows into h's permuted K order, in place
-                if (!tc::mbar_wait_ok(&bar_bfull[t % kRB], (t / kRB) & 1u, a.status, &s_ok)) {
-                    good = false;
-                    break;
-                }
-                unsigned char* rb = sR + (t % kRB) * kLoraSlot;
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub)
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        uint4* c4 = reinterpret_cast<uint4*>(rb + sub * (kLoraRows * 128) + (j ? boff1 : boff0));
-                        *c4 = permute_k8(*c4);
-                    }
-            }
-
             const int kk = pc.kt % SP;  // step inside the span
             const uint32_t astage = tmem + tlane + kTmemA + (t % kAS) * 128;
             if (int4_mode && wstep) {
@@ -864,11 +798,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // A LoRA-B step's span (rows the MMAs read directly) is released only once it has
             // landed: the loader must have seen the slot's previous release complete before this
             // one completes, or its parity wait would alias two phases ahead.
-            if (!lora_mode && !wstep && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) {
+            if (!wstep && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) {
                 good = false;
                 break;
             }
-            if (lane == 0 && !lora_mode && (!wstep || kk == SP - 1 || pc.kt == pc.KW - 1))
+            if (lane == 0 && (!wstep || kk == SP - 1 || pc.kt == pc.KW - 1))
                 tc::mbar_arrive(&bar_rawfree[sseq % kRS]);
             ++t;
 
@@ -889,7 +823,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
             }
             advance(pc);
-            if (!lora_mode && pc.item < nitems && opens(pc)) ++sseq;
+            if (pc.item < nitems && opens(pc)) ++sseq;
         }
         if (good && ep_pend && !epilogue(ep_pos, ep_seq)) good = false;
         if (!good) s_ok = 0;  // left early: let the other warps stop waiting
@@ -967,8 +901,6 @@ cudaError_t launch_kernel(TcArgs& a, cudaStream_t s) {
     switch (a.mode) {
         case kGU: return launch_mode<kGU>(a, nsm, s);
         case kDown: return launch_mode<kDown>(a, nsm, s);
-        case kLoraGU: return launch_mode<kLoraGU>(a, nsm, s);
-        case kLoraDown: return launch_mode<kLoraDown>(a, nsm, s);
         default: return launch_mode<kRouterMode>(a, nsm, s);
     }
 }
@@ -1043,7 +975,6 @@ cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, in
     a.h_out = const_cast<uint16_t*>(hb_out);
     a.ldh = ldh;
     a.ypart = wk.ypart;
-    a.t_out = mode == kTcLoraGU ? wk.tgu : wk.td;
     a.t_in = mode == kTcGU ? wk.tgu : wk.td;
     a.status = wk.status;
     cudaError_t e = cudaSuccess;
