@@ -224,7 +224,7 @@ def test_ffn_tiny(T):
 
 
 @pytest.mark.parametrize("variant", ["k1", "kE", "no_lora", "no_shared", "no_sgate", "multi_adapter", "bias",
-                                     "group32", "rank24", "rank64"])
+                                     "group32", "group32_decode", "rank24", "rank64"])
 def test_ffn_tiny_variants(variant):
     shape = workloads.TINY
     na = None
@@ -236,12 +236,12 @@ def test_ffn_tiny_variants(variant):
         shape = dataclasses.replace(shape, n_adapters=3, random_adapters=True)
     elif variant == "bias":
         shape = dataclasses.replace(shape, logit_bias_std=1.0)
-    elif variant == "group32":
+    elif variant in ("group32", "group32_decode"):
         shape = dataclasses.replace(shape, group=32)
     elif variant in ("rank24", "rank64"):  # LoRA-A products wider than one 32-column warp group
         shape = dataclasses.replace(shape, rank=int(variant[4:]), n_adapters=2, random_adapters=True)
-    t, x, aid = _ffn_case(shape, 410, T=19)
-    if variant == "group32":
+    t, x, aid = _ffn_case(shape, 410, T=3 if variant == "group32_decode" else 19)
+    if variant in ("group32", "group32_decode"):
         w = workloads.moe_weights(shape, seed=410)
         t = quantize_layer(w, group=32)
     if variant == "no_lora":
