@@ -421,6 +421,23 @@ def test_full_size_decode(full_layer, K, T):
     _check_ffn(shape, tt, x, None, n_adapters=1, what="decode K=%d T=%d" % (K, T))
 
 
+@pytest.mark.parametrize("case", ["decode", "multi_tenant"])
+def test_full_size_group32(full_layer, case):
+    """The same Edge0-shaped weights packed at group 32 (twice the scales and biases): one
+    token through the fused decode kernel, 64 multi-tenant tokens through the tensor cores."""
+    shape0, w, _ = full_layer
+    t = quantize_layer(w, group=32)
+    if case == "decode":
+        shape = dataclasses.replace(workloads.DECODE_K4, group=32)
+        t["logit_bias"] = None
+        x, aid = workloads.moe_inputs(shape, seed=520, T=1)
+        _check_ffn(shape, t, x, None, n_adapters=1, what="group 32 decode")
+    else:
+        shape = dataclasses.replace(shape0, group=32)
+        x, aid = workloads.moe_inputs(shape, seed=521)
+        _check_ffn(shape, t, x, aid, what="group 32 multi-tenant")
+
+
 def test_full_size_multi_tenant(full_layer):
     shape, w, t = full_layer
     x, aid = workloads.moe_inputs(shape, seed=0)
