@@ -38,7 +38,7 @@ from synth import workloads  # noqa: E402
 
 METRIC = "MoE-FFN tokens/s; decode HBM GB/s and prefill TFLOP/s as % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-MOE_WORKLOADS = ("decode_k4", "decode_k8", "multi_tenant", "prefill")
+MOE_WORKLOADS = ("decode_k4", "decode_k8", "multi_tenant", "prefill", "decode_k4_g32", "multi_tenant_g32")
 MIXED_WORKLOADS = ("mixed_b1", "mixed_b16")
 
 
@@ -59,7 +59,7 @@ def parse_args(argv=None):
 
 def default_steps(workload):
     return {"decode_k4": 2000, "decode_k8": 2000, "multi_tenant": 1000, "prefill": 3, "mixed_b1": 200,
-            "mixed_b16": 200}[workload]
+            "mixed_b16": 200, "decode_k4_g32": 2000, "multi_tenant_g32": 1000}[workload]
 
 
 def measured_peaks():
@@ -203,8 +203,8 @@ def step_accounting(shape, idx, aid):
     (x bf16, h bf16, per-job outputs fp32).  Flops: 2 per multiply-add the method
     defines (LoRA-A of the adapter each job uses only)."""
     H, E, K, I, Is, r, T = shape.H, shape.E, shape.K, shape.I, shape.Is, shape.rank, idx.shape[0]
-    gu, d = expert_bytes(H, I)
-    sgu, sd = expert_bytes(H, Is)
+    gu, d = expert_bytes(H, I, shape.group)
+    sgu, sd = expert_bytes(H, Is, shape.group)
     lb = lora_bytes(H, I, r)
     slb = lora_bytes(H, Is, r)
     U, P, SP = routing_stats(idx, aid, K, shape.n_adapters)
@@ -212,7 +212,7 @@ def step_accounting(shape, idx, aid):
     J = T * (K + 1)
     h_bytes = (TK * I + T * Is) * 2
     b = {
-        "router": router_bytes(H, E) + T * H * 2 + T * E * 4,
+        "router": router_bytes(H, E, shape.group) + T * H * 2 + T * E * 4,
         "gate_up": U * gu + sgu + P * lb["B_gu"] + SP * slb["B_gu"] + T * H * 2 + h_bytes,
         "down": U * d + sd + P * lb["B_d"] + SP * slb["B_d"] + h_bytes + J * H * 4,
         "lora_gu": P * lb["A_gu"] + SP * slb["A_gu"] + T * H * 2,
@@ -225,7 +225,7 @@ def step_accounting(shape, idx, aid):
         "lora_gu": 2 * TK * 2 * r * H + 2 * T * 2 * r * H if r else 0,
         "lora_down": 2 * TK * r * I + 2 * T * r * Is if r else 0,
     }
-    weights = router_bytes(H, E) + U * (gu + d) + sgu + sd + P * sum(lb.values()) + SP * sum(slb.values())
+    weights = router_bytes(H, E, shape.group) + U * (gu + d) + sgu + sd + P * sum(lb.values()) + SP * sum(slb.values())
     act = 2 * T * H * 2
     b["layer"] = weights + act
     f["layer"] = sum(f.values())
@@ -242,17 +242,27 @@ KIND_UNIT = {"router_logits": "router", "tc_router": "router", "gate_up": "gate_
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# dominant kernel, from one ncu capture of the kernel as it stands; the capture's
-# summary sits under profiles/ (named here).  An entry is removed whenever its
-# kernel changes, so the bench reports null rather than a stale figure.
+# dominant kernel, from one ncu capture of the kernel as it stands (the capture's
+# summary is kept with the profiles).  An entry is removed whenever its kernel
+# changes, so the bench reports null rather than a stale figure.
 NCU_TRAFFIC = {
     # one gate/up launch over the 2048-token prompt of one layer
-    ("prefill", "tc_gate_up"): (333590784 + 9545728, "profiles/tc_gate_up_down_prefill_layer.md"),
-    # one launch of the fused decode kernel, one token, top-4
-    ("decode_k4", "decode_fused"): (11294208, "profiles/decode_fused_decode_k4.md"),
+    ("prefill", "tc_gate_up"): 333590784 + 9545728,
     # one gate/up launch of the mixed ternary/4-bit MLP, one token
-    ("mixed_b1", "mixed_gate_up"): (2014976, "profiles/mixed_gate_up_down_mixed_b1.md"),
+    ("mixed_b1", "mixed_gate_up"): 2014976,
 }
+
+
+def launch_times(kt, ms_graph):
+    """Per-kind (ms per launch, launches) from the event-timed replay, less the event
+    nodes' own cost: the excess of the summed event intervals over the plain graph's
+    time is spread evenly over the launches (each event node adds the same gap), so
+    the per-kind times add up to the plain graph's time and none exceeds a step."""
+    n = sum(c for _, c in kt.values())
+    if not n:
+        return {}
+    excess = max(0.0, sum(t for t, _ in kt.values()) - ms_graph) / n
+    return {k: (max(t / c - excess, 0.0), c) for k, (t, c) in kt.items()}
 
 
 def kernel_roofline(kind, dur_ms, nbytes, nflops, peaks, src, timed_s, workload=None):
@@ -276,10 +286,11 @@ def kernel_roofline(kind, dur_ms, nbytes, nflops, peaks, src, timed_s, workload=
         roof = {"kernel": kind, "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(gbs / hbm, 4), "peak_source": "%s hbm_gbs" % src, "tensor": tensor}
     tr = NCU_TRAFFIC.get((workload, kind))
-    roof.update({"traffic": tr[0] if tr else None, "launch_us": round(dur_ms * 1e3, 3),
-                 "bytes_per_launch": int(nbytes), "flops_per_launch": int(nflops)})
+    roof.update({"traffic": tr, "launch_us": round(dur_ms * 1e3, 3),
+                 "bytes_per_launch": int(nbytes), "flops_per_launch": int(nflops),
+                 "launch_time": "CUDA events in a graph replay, less the event nodes' overhead"})
     if tr:
-        roof["traffic_source"] = "ncu capture, " + tr[1]
+        roof["traffic_source"] = "ncu capture of this kernel"
     return roof
 
 
@@ -433,8 +444,9 @@ def oracle_moe_layer(shape, host0):
                               alpha=shape.alpha, group=shape.group)
 
 
-def cpu_baseline_moe(shape, host0, seed, budget_s, x_inputs, aid_inputs):
-    """Oracle tokens/s on a bounded sample: whole tokens through layer copy 0."""
+def cpu_baseline_moe(shape, host0, seed, budget_s, x_inputs, aid_inputs, layers=1):
+    """Oracle tokens/s on a bounded sample: whole tokens through layer copy 0, divided by
+    the number of layers a step runs (a stack's prompt tokens pass through every layer)."""
     import oracle
     L = oracle_moe_layer(shape, host0)
     done, t0 = 0, time.time()
@@ -449,9 +461,11 @@ def cpu_baseline_moe(shape, host0, seed, budget_s, x_inputs, aid_inputs):
         if time.time() - t0 >= budget_s:
             break
     el = time.time() - t0
-    return {"value": done / el, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-            "sample": "%d tokens of the %s layer (layer copy 0) through the fp64 oracle in %.1f s" %
-                      (done, shape.name, el)}
+    sample = "%d tokens of the %s layer (layer copy 0) through the fp64 oracle in %.1f s" % (done, shape.name, el)
+    if layers > 1:
+        sample += ", scaled to the %d-layer stack" % layers
+    return {"value": done / el / layers, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": sample}
 
 
 # ----------------------------------------------------------------- the timed runs
@@ -459,8 +473,7 @@ def run_moe(args, world, rank, local):
     import torch
     import int4_group_affine_b200 as moeq
     dev = torch.device("cuda", local)
-    shape = workloads.MOE_SHAPES[{"decode_k4": "decode_k4", "decode_k8": "decode_k8",
-                                  "multi_tenant": "multi_tenant", "prefill": "prefill"}[args.workload]]
+    shape = workloads.MOE_SHAPES[args.workload]
     stack = args.workload == "prefill"
     copies = args.copies or (shape.layers if stack else 40)
     K, W = args.steps, args.warmup
@@ -504,10 +517,10 @@ def run_moe(args, world, rank, local):
     clocks.stop()
     del g
     ms_step = ms / K
-    tokens_per_step = T * (copies if stack else 1)
+    tokens_per_step = T  # prefill: the prompt's tokens through the whole stack per step
 
     # per-kernel durations: the same steps captured again with library event timing on
-    kt = kernel_times(moeq, step, W, K)
+    kt = launch_times(kernel_times(moeq, step, W, K), ms)
     launches_per_step = sum(c for _, c in kt.values()) / K
 
     # routing of each timed step (for byte accounting), recomputed outside the timed region
@@ -521,11 +534,11 @@ def run_moe(args, world, rank, local):
 
     peaks, src = measured_peaks()
     hbm = float(peaks["hbm_gbs"])
-    dom = max(kt.items(), key=lambda kv: kv[1][0])[0] if kt else None
+    dom = max(kt.items(), key=lambda kv: kv[1][0] * kv[1][1])[0] if kt else None
     roof = None
     if dom is not None and dom in KIND_UNIT:
         unit = KIND_UNIT[dom]
-        roof = kernel_roofline(dom, kt[dom][0] / kt[dom][1], acc["kernel_bytes"][unit], acc["kernel_flops"][unit],
+        roof = kernel_roofline(dom, kt[dom][0], acc["kernel_bytes"][unit], acc["kernel_flops"][unit],
                                peaks, src, ms * 1e-3, args.workload)
     step_bytes = acc["weight_bytes"] + acc["act_bytes"]
     step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
@@ -535,7 +548,8 @@ def run_moe(args, world, rank, local):
         "ms_per_step": round(ms_step, 6), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4 weights, bf16 activations, fp32 accumulate", "data": "synthetic (seeded generator; no trained weights)",
         "config": {"workload": shape.name, "hidden": shape.H, "experts": shape.E, "top_k": shape.K,
-                   "inter": shape.I, "shared_inter": shape.Is, "tokens": T, "lora_rank": shape.rank,
+                   "inter": shape.I, "shared_inter": shape.Is, "tokens": T, "group": shape.group,
+                   "lora_rank": shape.rank,
                    "adapters": shape.n_adapters, "layer_copies": copies,
                    "l2": "inputs larger than L2: %d distinct layer copies (%.1f GB) rotated per step" %
                          (copies, sum(l.nbytes() for l in layers) / 1e9),
@@ -546,14 +560,17 @@ def run_moe(args, world, rank, local):
                           "frac": round(step_gbs / hbm, 4), "bytes_per_step": int(step_bytes),
                           "what": "touched expert + LoRA + router bytes per step / step time"},
         "tflops": round(acc["flops"] / (ms_step * 1e-3) / 1e12, 3),
-        "kernels": {k: {"ms_per_launch": round(v[0] / v[1], 6), "launches": v[1]} for k, v in kt.items()},
+        "kernels": {k: {"ms_per_launch": round(v[0], 6), "launches": v[1]} for k, v in kt.items()},
         "gpu_launches": int(round(launches_per_step * K)),
         "clocks": clocks.summary(t_wall0, t_wall1),
     }
+    if stack:
+        out["config"]["unit"] = "prompt tokens through the %d-layer stack" % copies
     if e2e is not None:
         out["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline_moe(shape, host0, args.seed, args.cpu_seconds, xs_host, aids_host)
+        out["cpu_baseline"] = cpu_baseline_moe(shape, host0, args.seed, args.cpu_seconds, xs_host, aids_host,
+                                               copies if stack else 1)
     return out
 
 
@@ -628,7 +645,7 @@ def run_e2e(moeq, shape, layers, xs_host, aids_host, K, W, copies, n_inputs, sta
     g = capture_steps(step, W, K)
     ms, _, _ = timed_replay(g, world)
     del g
-    toks = T * (len(layers) if stack else 1)
+    toks = T
     h2d = T * H * 2 + (0 if ha is None else T * 4)
     return {"value": round(job_throughput(toks, K, world, ms), 2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": T * H * 2, "ms_per_step": round(ms / K, 6)}
@@ -683,23 +700,24 @@ def run_mixed(args, world, rank, local):
     clocks.stop()
     del g
     ms_step = ms / K
-    kt = kernel_times(moeq, step, W, K)
+    kt = launch_times(kernel_times(moeq, step, W, K), ms)
     layer_bytes = sum(m.nbytes() for m in mats[0].values())
     peaks, src = measured_peaks()
     hbm = float(peaks["hbm_gbs"])
-    dom = max(kt.items(), key=lambda kv: kv[1][0])[0]
+    dom = max(kt.items(), key=lambda kv: kv[1][0] * kv[1][1])[0]
     per = {"mixed_gate_up": mats[0]["gate"].nbytes() + mats[0]["up"].nbytes(),
            "mixed_down": mats[0]["down"].nbytes()}.get(dom)
     roof = None
     if per:
-        dur = kt[dom][0] / kt[dom][1]
+        dur = kt[dom][0]
         gbs = per / (dur * 1e-3) / 1e9
         tr = NCU_TRAFFIC.get((args.workload, dom))
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(gbs / hbm, 4), "traffic": tr[0] if tr else None, "peak_source": "%s hbm_gbs" % src,
-                "launch_us": round(dur * 1e3, 3), "bytes_per_launch": per}
+                "frac": round(gbs / hbm, 4), "traffic": tr, "peak_source": "%s hbm_gbs" % src,
+                "launch_us": round(dur * 1e3, 3), "bytes_per_launch": per,
+                "launch_time": "CUDA events in a graph replay, less the event nodes' overhead"}
         if tr:
-            roof["traffic_source"] = "ncu capture, " + tr[1]
+            roof["traffic_source"] = "ncu capture of this kernel"
     step_gbs = L * layer_bytes / (ms_step * 1e-3) / 1e9
     out = {
         "metric": METRIC, "value": round(job_throughput(T, K, world, ms), 2), "unit": "tokens/s", "n_gpus": world,
@@ -714,7 +732,7 @@ def run_mixed(args, world, rank, local):
         "roofline": roof,
         "step_roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": hbm, "unit": "GB/s",
                           "frac": round(step_gbs / hbm, 4), "bytes_per_step": L * layer_bytes},
-        "kernels": {k: {"ms_per_launch": round(v[0] / v[1], 6), "launches": v[1]} for k, v in kt.items()},
+        "kernels": {k: {"ms_per_launch": round(v[0], 6), "launches": v[1]} for k, v in kt.items()},
         "gpu_launches": int(sum(c for _, c in kt.values())),
         "clocks": clocks.summary(t0, t1),
     }

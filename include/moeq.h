@@ -237,9 +237,11 @@ MOEQ_API moe_status moe_ffn_forward(const moe_layer* layer, const uint16_t* x, c
  * a fixed array of MOEQ_STATIC_WS_BYTES compiled into the library; every device
  * that loads the library holds that array until the process exits.  The caller
  * still passes x, adapter_id and y (device pointers, as for moe_ffn_forward).
- *  - Returns MOE_ERR_WORKSPACE, enqueuing nothing, when
- *    moe_ffn_workspace_bytes(layer, T) exceeds MOEQ_STATIC_WS_BYTES (16 MiB:
- *    e.g. up to about 300 tokens of the 2048-hidden, 256-expert, top-4 layer).
+ *  - The layer, T, x and y are checked first, with moe_ffn_forward's rules and
+ *    status codes; then MOE_ERR_WORKSPACE is returned when
+ *    moe_ffn_workspace_bytes(layer, T) exceeds MOEQ_STATIC_WS_BYTES (16 MiB: at
+ *    least 256 tokens of the 2048-hidden, 256-expert, top-4 layer with four
+ *    rank-16 adapter sets).  A rejected call enqueues nothing.
  *  - The first call on a device looks up the array's device address there
  *    (once per device, with that device current); make that first call before
  *    any stream capture.
@@ -251,6 +253,14 @@ MOEQ_API moe_status moe_ffn_forward(const moe_layer* layer, const uint16_t* x, c
 #define MOEQ_STATIC_WS_BYTES (16u * 1024u * 1024u)
 MOEQ_API moe_status moe_ffn_forward_static(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id,
                                            int32_t T, uint16_t* y, moe_stream stream);
+
+/* The sticky device status word of the fixed array above (what moe_get_device_status
+ * reads for a caller-owned workspace): the first problem the device saw during the
+ * most recent moe_ffn_forward_static call on this device (MOE_ERR_DEVICE_INDEX,
+ * MOE_ERR_TIMEOUT) or MOE_OK.  Read it after that call and before the next one,
+ * which clears it.  Writes the value into *status (host), clears the word, and
+ * synchronises `stream`. */
+MOEQ_API moe_status moe_ffn_static_device_status(moe_stream stream, int32_t* status);
 
 /* Pre-norm residual block for stacked layers:
  *   x_out = bf16(x + FFN(bf16(RMSNorm(x)))), RMSNorm with unit weight and eps.
@@ -264,6 +274,25 @@ MOEQ_API moe_status moe_rmsnorm(const uint16_t* x, int32_t T, int32_t H, float e
 /* Read the sticky device status word of a workspace into *status (host) and
  * clear it.  Synchronises `stream`. */
 MOEQ_API moe_status moe_get_device_status(void* workspace, moe_stream stream, int32_t* status);
+
+/* The routing a forward used: copies the expert indices [T][K] (int32) and the
+ * renormalised weights [T][K] (fp32) that the last moe_ffn_forward or
+ * moe_block_forward with this layer shape, T and workspace selected (whichever
+ * kernels ran it) into topk_idx / topk_w (device pointers; either may be NULL).
+ * Enqueued on `stream` after that call; the workspace must not have been used
+ * by another call in between.  Routing indices stay on the device ("Edge0 项目推荐"
+ * review, 亮点二); this is the record a caller or a test reads them from. */
+MOEQ_API moe_status moe_ffn_routing(const moe_layer* layer, int32_t T, const void* workspace, size_t ws_bytes,
+                                    int32_t* topk_idx, float* topk_w, moe_stream stream);
+
+/* Bound of every device-side wait (a grid-wide arrival, a ready flag, a bulk-copy
+ * or pipeline barrier), in nanoseconds of device time; 0 restores the default of
+ * one second.  A wait that runs out sets MOE_ERR_TIMEOUT in the status word and the
+ * kernel returns (its output is then incomplete).  The value is read when a call
+ * enqueues its kernels, so a captured CUDA graph keeps the value of its capture.
+ * Process-wide, not thread-safe. */
+MOEQ_API moe_status moe_set_wait_limit_ns(uint64_t ns);
+MOEQ_API uint64_t moe_wait_limit_ns(void);
 
 /* --------------------------------------------------------- a7 mixed layout
  * y[t][o] = s_o * sum_j q_oj x[t][j] (weight-only form of the EdgeRazor

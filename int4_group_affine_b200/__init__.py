@@ -20,7 +20,8 @@ __all__ = [
     "moe_index_workspace_bytes", "moe_index_build", "lora_set_adapters", "moe_ffn_workspace_bytes",
     "moe_workspace_init", "moe_ffn_forward", "moe_block_forward", "moe_rmsnorm", "moe_get_device_status",
     "moe_mixed_linear", "moe_mixed_mlp_workspace_bytes", "moe_mixed_mlp_forward",
-    "moe_timing_enable", "moe_timing_collect",
+    "moe_timing_enable", "moe_timing_collect", "moe_ffn_forward_static", "moe_ffn_static_device_status",
+    "moe_ffn_routing", "moe_set_wait_limit_ns", "moe_wait_limit_ns",
 ]
 
 
@@ -171,3 +172,25 @@ def moe_ffn_forward_static(layer: Layer, x, adapter_id, T, y, stream=None):
     _check("moe_ffn_forward_static", _lib.lib().moe_ffn_forward_static(ctypes.byref(layer), _ptr(x),
                                                                        _ptr(adapter_id), T, _ptr(y),
                                                                        _stream(stream)))
+
+
+def moe_ffn_static_device_status(stream=None) -> int:
+    """Read and clear the status word of the built-in workspace (synchronises)."""
+    v = ctypes.c_int32(0)
+    _check("moe_ffn_static_device_status", _lib.lib().moe_ffn_static_device_status(_stream(stream),
+                                                                                   ctypes.byref(v)))
+    return int(v.value)
+
+
+def moe_ffn_routing(layer: Layer, T, workspace, ws_bytes, topk_idx, topk_w, stream=None):
+    """Copy the routing (indices, weights) the last forward on this workspace used."""
+    _check("moe_ffn_routing", _lib.lib().moe_ffn_routing(ctypes.byref(layer), T, _ptr(workspace), ws_bytes,
+                                                         _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
+
+
+def moe_set_wait_limit_ns(ns: int):
+    _check("moe_set_wait_limit_ns", _lib.lib().moe_set_wait_limit_ns(int(ns)))
+
+
+def moe_wait_limit_ns() -> int:
+    return int(_lib.lib().moe_wait_limit_ns())

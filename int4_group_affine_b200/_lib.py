@@ -71,6 +71,10 @@ SIGNATURES = {
     "moe_mixed_linear": (ctypes.c_int, [PM, P, I32, P, P]),
     "moe_mixed_mlp_workspace_bytes": (SZ, [I32, I32, I32]),
     "moe_mixed_mlp_forward": (ctypes.c_int, [PM, PM, PM, P, I32, I32, F32, P, P, SZ, P]),
+    "moe_ffn_static_device_status": (ctypes.c_int, [P, ctypes.POINTER(I32)]),
+    "moe_ffn_routing": (ctypes.c_int, [PL, I32, P, SZ, P, P, P]),
+    "moe_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
+    "moe_wait_limit_ns": (ctypes.c_uint64, []),
     "moe_timing_kinds": (ctypes.c_int, []),
     "moe_timing_kind_name": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_timing_enable": (ctypes.c_int, [ctypes.c_int]),

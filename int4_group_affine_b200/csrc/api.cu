@@ -7,6 +7,13 @@
 #include "common.cuh"
 
 namespace moeq {
+
+namespace {
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;  // 1 s
+uint64_t g_wait_ns = kDefaultWaitNs;
+}  // namespace
+uint64_t wait_limit_ns() { return g_wait_ns; }
+
 cudaError_t launch_index_build_counts(const Work& wk, const int32_t* adapter_id, int n_adapters, int32_t* counts_out,
                                       cudaStream_t s);
 }
@@ -275,6 +282,8 @@ bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id
     sc.tdp = (float*)(b + p.dtdp);
     sc.bar = (unsigned long long*)(b + p.bar);
     sc.status = (int32_t*)(b + p.status);
+    sc.idx_out = (int32_t*)(b + p.idx);
+    sc.w_out = (float*)(b + p.w);
     const cudaError_t e = launch_decode(la, x, adapter_id, y, T, block, eps, sc, s);
     if (e == cudaErrorNotSupported || e == cudaErrorCooperativeLaunchTooLarge) {
         (void)cudaGetLastError();
@@ -297,7 +306,26 @@ int mixed_G(float rho) { return rho > 0.0f ? (int)floor(1.0 / (double)rho + 1e-6
 
 }  // namespace
 
+namespace moeq {
+// Everything moe_ffn_forward checks before it looks at the workspace: the layer, T,
+// and (for T > 0) the input and output pointers.
+moe_status ffn_precheck(const moe_layer* layer, const uint16_t* x, const uint16_t* y, int32_t T) {
+    moe_status st = validate_layer(layer);
+    if (st != MOE_OK) return st;
+    CHECK_ARG(T >= 0);
+    if (T > 0) CHECK_ARG(x && y && x != y && aligned(x, 16) && aligned(y, 2));
+    return MOE_OK;
+}
+}  // namespace moeq
+
 extern "C" {
+
+moe_status moe_set_wait_limit_ns(uint64_t ns) {
+    g_wait_ns = ns == 0 ? kDefaultWaitNs : ns;
+    return MOE_OK;
+}
+
+uint64_t moe_wait_limit_ns(void) { return g_wait_ns; }
 
 int moe_version(void) { return MOEQ_VERSION; }
 
@@ -451,15 +479,13 @@ moe_status moe_workspace_init(void* workspace, size_t ws_bytes, moe_stream strea
 
 moe_status moe_ffn_forward(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id, int32_t T,
                            uint16_t* y, void* workspace, size_t ws_bytes, moe_stream stream) {
-    moe_status st = validate_layer(layer);
+    moe_status st = ffn_precheck(layer, x, y, T);
     if (st != MOE_OK) return st;
-    CHECK_ARG(T >= 0);
     const Dims d = dims_of(layer, T);
     const WsPlan p = plan_of(d);
     st = ws_check(workspace, ws_bytes, p.total);
     if (st != MOE_OK) return st;
     if (T == 0) return MOE_OK;
-    CHECK_ARG(x && y && x != y && aligned(x, 16) && aligned(y, 2));
     cudaStream_t s = (cudaStream_t)stream;
     timing_begin(s);
     if (try_decode(layer, x, adapter_id, T, 0, 0.0f, y, d, p, workspace, s, &st)) return st;
@@ -492,6 +518,25 @@ moe_status moe_rmsnorm(const uint16_t* x, int32_t T, int32_t H, float eps, uint1
     cudaStream_t s = (cudaStream_t)stream;
     timing_begin(s);
     LAUNCH(kRmsnorm, launch_rmsnorm(x, T, H, eps, xn, s));
+    return MOE_OK;
+}
+
+moe_status moe_ffn_routing(const moe_layer* layer, int32_t T, const void* workspace, size_t ws_bytes,
+                           int32_t* topk_idx, float* topk_w, moe_stream stream) {
+    moe_status st = validate_layer(layer);
+    if (st != MOE_OK) return st;
+    CHECK_ARG(T >= 0);
+    const Dims d = dims_of(layer, T);
+    const WsPlan p = plan_of(d);
+    st = ws_check(const_cast<void*>(workspace), ws_bytes, p.total);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(topk_idx || topk_w);
+    cudaStream_t s = (cudaStream_t)stream;
+    const char* b = (const char*)workspace;
+    const size_t n = (size_t)T * d.K;
+    if (topk_idx) CHECK_CUDA(cudaMemcpyAsync(topk_idx, b + p.idx, n * 4, cudaMemcpyDeviceToDevice, s));
+    if (topk_w) CHECK_CUDA(cudaMemcpyAsync(topk_w, b + p.w, n * 4, cudaMemcpyDeviceToDevice, s));
     return MOE_OK;
 }
 

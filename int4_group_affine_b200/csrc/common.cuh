@@ -77,6 +77,13 @@ struct LayerArgs {
     moe_lora_ptrs lora[MOEQ_MAX_ADAPTERS];
 };
 
+// Bound (ns of device time) of every bounded device-side wait, passed to the kernels
+// with their arguments (moe_set_wait_limit_ns; 1 s by default).
+uint64_t wait_limit_ns();
+
+// The forward's checks that precede the workspace check (layer, T, x and y).
+moe_status ffn_precheck(const moe_layer* layer, const uint16_t* x, const uint16_t* y, int32_t T);
+
 // Raise a kernel's dynamic shared-memory limit to at least `bytes`, calling the
 // runtime only when the cached limit is too small (so repeated launches, and
 // launches during stream capture, do not call it again).  The cache assumes one
@@ -103,6 +110,8 @@ struct DecodeScratch {
     float* tdp;               // [MOEQ_DECODE_MAX_CTAS][3][T][rank] partial sums
     unsigned long long* bar;  // monotonic arrival counter: starts zeroed (workspace header)
     int32_t* status;          // workspace base (status word)
+    int32_t* idx_out;         // [T][K] routing record (the workspace's top-K region)
+    float* w_out;             // [T][K]
 };
 
 // ------------------------------------------------------------- timing

@@ -48,7 +48,6 @@ constexpr int kMaxOut = 32;                // output rows per CTA in phase D
 constexpr int kMaxUD = kMaxJ + 1;          // phase-D experts: the routed ones and the shared one
 constexpr int kFlagOffset = 16;            // byte offset of the LoRA-A ready flags in the workspace header
 constexpr int kMaxFlags = (256 - kFlagOffset) / 4;
-constexpr unsigned long long kWaitNs = 1000000000ull;  // bound of every wait (1 s)
 
 // Shared-memory plan of a launch: ranges per CTA and byte offsets into the dynamic
 // segment, computed on the host from the shape and the largest possible number of
@@ -83,6 +82,9 @@ struct DArgs {
     uint32_t* flags;   // [2 T K] launch epoch once tg of (slot, gate|up) is written
     unsigned long long* bar;  // monotonic arrival counter
     int32_t* status;
+    uint64_t wait_ns;  // bound of every wait
+    int32_t* idx_out;  // [T][K] routing written by CTA 0 (the forward's routing record)
+    float* w_out;      // [T][K]
     DPlan P;
 };
 
@@ -108,7 +110,7 @@ __device__ __forceinline__ void st_release32(uint32_t* p, uint32_t v) {
 // *abort set), after which the counter is out of step and the workspace must be
 // re-initialised.
 __device__ void grid_sync(unsigned long long* bar, unsigned long long& target, int32_t* status,
-                          volatile int* abort) {
+                          volatile int* abort, uint64_t limit_ns) {
     __syncthreads();
     if (threadIdx.x == 0) {
         const unsigned long long nb = gridDim.x;
@@ -118,7 +120,7 @@ __device__ void grid_sync(unsigned long long* bar, unsigned long long& target, i
         const uint64_t t0 = tc::globaltimer_ns();
         for (uint32_t i = 0; ld_acquire(bar) < target; ++i) {
             if ((i & 255) == 255) {
-                if (tc::globaltimer_ns() - t0 > kWaitNs) {
+                if (tc::globaltimer_ns() - t0 > limit_ns) {
                     raise_status(status, MOE_ERR_TIMEOUT);
                     *abort = 1;
                     break;
@@ -131,13 +133,13 @@ __device__ void grid_sync(unsigned long long* bar, unsigned long long& target, i
 }
 
 // Wait (bounded) for phase 0 of a bulk-copy mbarrier; gives up at once if *abort is set.
-__device__ bool copies_landed(uint64_t* bar, int32_t* status, volatile int* abort) {
+__device__ bool copies_landed(uint64_t* bar, int32_t* status, volatile int* abort, uint64_t limit_ns) {
     if (tc::mbar_try_wait(bar, 0)) return true;
     const uint64_t t0 = tc::globaltimer_ns();
     for (;;) {
         if (tc::mbar_try_wait(bar, 0)) return true;
         if (*abort) return false;
-        if (tc::globaltimer_ns() - t0 > kWaitNs) {
+        if (tc::globaltimer_ns() - t0 > limit_ns) {
             raise_status(status, MOE_ERR_TIMEOUT);
             *abort = 1;
             return false;
@@ -619,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         bool landed = false;
         for (int j = warp; j < nra + nsr + nla; j += kW) {
             if (j < nra + nsr + 2 && !landed) {
-                if (!copies_landed(&s_bar[0], a.status, &s_abort)) break;
+                if (!copies_landed(&s_bar[0], a.status, &s_abort, a.wait_ns)) break;
                 landed = true;
             }
             if (j < nra) {
@@ -680,13 +682,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
     }
     unsigned long long bar_target = 0;
-    grid_sync(a.bar, bar_target, a.status, &s_abort);
+    grid_sync(a.bar, bar_target, a.status, &s_abort, a.wait_ns);
 
     // ------------------------------------------------------------ phase B
     if (tid == 0) s_epoch = (uint32_t)(bar_target / (unsigned long long)NB);
     if (tid < T) s_sg[tid] = L.has_sgate ? 1.0f / (1.0f + expf(-__ldcg(a.gsl + tid))) : 1.0f;
     cta_topk(a.logits, T, E, K, reinterpret_cast<uint2*>(dsm + P.cand), s_idx, s_w);
     __syncthreads();
+    if (cta == 0 && tid < TK) {  // the routing this call used, for the caller's record
+        a.idx_out[tid] = s_idx[tid / K][tid % K];
+        a.w_out[tid] = s_w[tid / K][tid % K];
+    }
     if (warp == 0) {
         // routed jobs (lane = slot t*K+k) sorted by (expert, adapter, slot): the rank of a
         // lane's key among all keys is its position; experts ascending, each expert's jobs
@@ -893,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if (kk && ld) ad[m] = bf16f(ld->A[((int64_t)e * r + lane) * I + i]);
             }
             if (!landed) {
-                if (!copies_landed(&s_bar[1], a.status, &s_abort)) break;
+                if (!copies_landed(&s_bar[1], a.status, &s_abort, a.wait_ns)) break;
                 landed = true;
             }
             float ag[MT], au[MT];
@@ -917,7 +923,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         const uint32_t* fp = a.flags + slot * 2 + (lane & 1);
                         const uint64_t t0 = tc::globaltimer_ns();
                         for (uint32_t it = 0; ld_acquire32(fp) != epoch; ++it)
-                            if ((it & 63) == 63 && tc::globaltimer_ns() - t0 > kWaitNs) {
+                            if ((it & 63) == 63 && tc::globaltimer_ns() - t0 > a.wait_ns) {
                                 raise_status(a.status, MOE_ERR_TIMEOUT);
                                 s_abort = 1;
                                 ready = false;
@@ -969,7 +975,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         __syncthreads();
     }
     if (P.dalias && warp == 0) issue_down();  // the gate/up windows are no longer read
-    grid_sync(a.bar, bar_target, a.status, &s_abort);
+    grid_sync(a.bar, bar_target, a.status, &s_abort, a.wait_ns);
 
     // ------------------------------------------------------------ phase D
     const bool runD = s_abort == 0;
@@ -1053,7 +1059,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
     __syncthreads();
     // (output row, expert) tasks from the down windows; a task is a group of lpt lanes over one row
-    if (runD && no > 0 && copies_landed(&s_bar[2], a.status, &s_abort)) {
+    if (runD && no > 0 && copies_landed(&s_bar[2], a.status, &s_abort, a.wait_ns)) {
         int lpt = 1;
         while (lpt * 2 <= 32 && lpt * 2 <= Imax / 32) lpt *= 2;
         const int gpw = 32 / lpt, sub = lane / lpt, sl = lane % lpt;
@@ -1110,7 +1116,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // a CTA that gave up leaves no bulk copy in flight (bounded wait)
     if (tid == 0 && s_abort)
         for (int i = 0; i < 3; ++i)
-            if (s_issued[i]) tc::mbar_wait(&s_bar[i], 0, nullptr);
+            if (s_issued[i]) tc::mbar_wait(&s_bar[i], 0, nullptr, a.wait_ns);
 }
 
 }  // namespace
@@ -1310,6 +1316,9 @@ cudaError_t launch_decode(const LayerArgs& L, const uint16_t* x, const int32_t* 
     a.flags = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(sc.status) + kFlagOffset);
     a.bar = sc.bar;
     a.status = sc.status;
+    a.wait_ns = wait_limit_ns();
+    a.idx_out = sc.idx_out;
+    a.w_out = sc.w_out;
     if (T <= 1) return launch_mt<1>(a, s);
     if (T <= 2) return launch_mt<2>(a, s);
     if (T <= 4) return launch_mt<4>(a, s);

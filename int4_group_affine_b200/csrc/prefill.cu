@@ -99,6 +99,7 @@ struct TcArgs {
     float* logits;        // router: [T][E]
     int T;                // router: tokens
     int32_t* status;
+    uint64_t wait_ns;     // bound of every mbarrier wait
 };
 
 struct Geo {  // one expert group's geometry in the current mode
@@ -358,12 +359,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (opens(pl)) {
                 const int slot = cs % kRS;
                 if (cs >= (uint32_t)kRS) {
-                    if (!tc::mbar_wait_ok(&bar_rawfree[slot], ((cs / kRS) - 1) & 1u, a.status, &s_ok)) {
+                    if (!tc::mbar_wait_ok(&bar_rawfree[slot], ((cs / kRS) - 1) & 1u, a.status, &s_ok, a.wait_ns)) {
                         ok = false;
                         break;
                     }
                     const int tr = slot_mma[slot];
-                    if (tr >= 0 && !tc::mbar_wait_ok(&bar_tile[tr % kTiles], (tr / kTiles) & 1u, a.status, &s_ok)) {
+                    if (tr >= 0 && !tc::mbar_wait_ok(&bar_tile[tr % kTiles], (tr / kTiles) & 1u, a.status, &s_ok, a.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // ---- the step's activation slot (after the MMAs kRB steps back)
             const int bslot = t % kRB;
             if (t >= (uint32_t)kRB &&
-                !tc::mbar_wait_ok(&bar_tile[(t - kRB) % kTiles], ((t - kRB) / kTiles) & 1u, a.status, &s_ok)) {
+                !tc::mbar_wait_ok(&bar_tile[(t - kRB) % kTiles], ((t - kRB) / kTiles) & 1u, a.status, &s_ok, a.wait_ns)) {
                 ok = false;
                 break;
             }
@@ -459,10 +460,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         tc::cp_wait<0>();
         if (lane == 0) {
             for (uint32_t sq = issued > (uint32_t)kRS ? issued - kRS : 0; sq < issued; ++sq)
-                tc::mbar_wait(&bar_raw[sq % kRS], (sq / kRS) & 1u, a.status);
+                tc::mbar_wait(&bar_raw[sq % kRS], (sq / kRS) & 1u, a.status, a.wait_ns);
             if (tma_b)
                 for (uint32_t sq = t > (uint32_t)kRB ? t - kRB : 0; sq < t; ++sq)
-                    tc::mbar_wait(&bar_bfull[sq % kRB], (sq / kRB) & 1u, a.status);
+                    tc::mbar_wait(&bar_bfull[sq % kRB], (sq / kRB) & 1u, a.status, a.wait_ns);
             if (!ok) s_ok = 0;
         }
         __syncwarp();
@@ -485,9 +486,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             uint32_t idesc = tc::idesc_bf16(kBM, (tile_jobs(pc) + 15) / 16 * 16);
             while (pc.item < nitems) {
                 const bool wstep = pc.kt < pc.KW;
-                if (!tc::mbar_spin_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok) ||
-                    !tc::mbar_spin_ok(&bar_bfull[t % kRB], (t / kRB) & 1u, a.status, &s_ok) ||
-                    (!wstep && !tc::mbar_spin_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok))) {
+                if (!tc::mbar_spin_ok(&bar_full[t % kAS], (t / kAS) & 1u, a.status, &s_ok, a.wait_ns) ||
+                    !tc::mbar_spin_ok(&bar_bfull[t % kRB], (t / kRB) & 1u, a.status, &s_ok, a.wait_ns) ||
+                    (!wstep && !tc::mbar_spin_ok(&bar_raw[cs % kRS], (cs / kRS) & 1u, a.status, &s_ok, a.wait_ns))) {
                     ok = false;
                     break;
                 }
@@ -528,7 +529,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 if (pc.item < nitems && opens(pc)) ++cs;
             }
             // drain (bounded): the last MMAs
-            if (t > 0) tc::mbar_wait(&bar_tile[(t - 1) % kTiles], ((t - 1) / kTiles) & 1u, a.status);
+            if (t > 0) tc::mbar_wait(&bar_tile[(t - 1) % kTiles], ((t - 1) / kTiles) & 1u, a.status, a.wait_ns);
             if (!ok) s_ok = 0;
         }
         __syncwarp();
@@ -623,7 +624,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 
         // ---- epilogue of a finished item (accumulator buffer seq % 2)
         auto epilogue = [&](const Pos& p, uint32_t seq) -> bool {
-            if (!tc::mbar_wait_ok(&bar_acc[seq & 1u], (seq >> 1) & 1u, a.status, &s_ok)) return false;
+            if (!tc::mbar_wait_ok(&bar_acc[seq & 1u], (seq >> 1) & 1u, a.status, &s_ok, a.wait_ns)) return false;
             tc::tc_fence_after();
             const Geo q = geo(p);
             const int n_here = tile_jobs(p);
@@ -709,7 +710,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // the MMAs of step t - kAS must be done before TMEM stage t % kAS (and, for a LoRA-B
             // step, activation slot t % kRB) is rewritten
             if (t >= (uint32_t)kAS &&
-                !tc::mbar_wait_ok(&bar_tile[(t - kAS) % kTiles], ((t - kAS) / kTiles) & 1u, a.status, &s_ok)) {
+                !tc::mbar_wait_ok(&bar_tile[(t - kAS) % kTiles], ((t - kAS) / kTiles) & 1u, a.status, &s_ok, a.wait_ns)) {
                 good = false;
                 break;
             }
@@ -735,7 +736,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // inputs of the first LoRA-B step, fetched during the last weight step so their latency
             // overlaps it (later LoRA-B steps fetch theirs right after staging the previous one)
             if (NL > 0 && pc.kt + 1 == pc.KW) fetch_lora(pc, 0, lr);
-            if (span_start && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) {
+            if (span_start && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok, a.wait_ns)) {
                 good = false;
                 break;
             }
@@ -798,7 +799,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // A LoRA-B step's span (rows the MMAs read directly) is released only once it has
             // landed: the loader must have seen the slot's previous release complete before this
             // one completes, or its parity wait would alias two phases ahead.
-            if (!wstep && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok)) {
+            if (!wstep && !tc::mbar_wait_ok(&bar_raw[sseq % kRS], (sseq / kRS) & 1u, a.status, &s_ok, a.wait_ns)) {
                 good = false;
                 break;
             }
@@ -977,6 +978,7 @@ cudaError_t launch_tc_gemm(const LayerArgs& L, int mode, const uint16_t* act, in
     a.ypart = wk.ypart;
     a.t_in = mode == kTcGU ? wk.tgu : wk.td;
     a.status = wk.status;
+    a.wait_ns = wait_limit_ns();
     cudaError_t e = cudaSuccess;
     if (mode == kTcDown) e = encode_act(&a.tmb, act, wk.J, ld_act, ld_act, kNT);
     if (e != cudaSuccess) return e;
@@ -1008,6 +1010,7 @@ cudaError_t launch_tc_router(const moe_qtensor& router, const float* logit_bias,
     a.logits = logits;
     a.T = T;
     a.status = status;
+    a.wait_ns = wait_limit_ns();
     cudaError_t e = encode_words(&a.tm[0], router.packed, E, H / 4);
     if (e == cudaSuccess) e = encode_act(&a.tmb, x, T, H, H, kNT);
     if (e != cudaSuccess) return e;

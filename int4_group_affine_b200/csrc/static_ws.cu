@@ -44,16 +44,27 @@ moe_status static_ws_address(void** out) {
 
 extern "C" moe_status moe_ffn_forward_static(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id,
                                              int32_t T, uint16_t* y, moe_stream stream) {
-    if (T < 0) return MOE_ERR_INVALID_ARG;
+    // The same checks as moe_ffn_forward, with the same results, before anything is
+    // enqueued: a rejected call leaves the array (and the status it holds) untouched.
+    moe_status st = moeq::ffn_precheck(layer, x, y, T);
+    if (st != MOE_OK) return st;
     const size_t need = moe_ffn_workspace_bytes(layer, T);
-    if (need == 0) return MOE_ERR_INVALID_ARG;  // the layer itself was rejected
     if (need > (size_t)MOEQ_STATIC_WS_BYTES) return MOE_ERR_WORKSPACE;
+    if (T == 0) return MOE_OK;
     void* ws = nullptr;
-    moe_status st = static_ws_address(&ws);
+    st = static_ws_address(&ws);
     if (st != MOE_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     // The array keeps the previous call's contents: the status header must
     // start at zero (everything else is written before it is read).
     if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess) return MOE_ERR_CUDA;
     return moe_ffn_forward(layer, x, adapter_id, T, y, ws, need, stream);
+}
+
+extern "C" moe_status moe_ffn_static_device_status(moe_stream stream, int32_t* status) {
+    if (!status) return MOE_ERR_INVALID_ARG;
+    void* ws = nullptr;
+    moe_status st = static_ws_address(&ws);
+    if (st != MOE_OK) return st;
+    return moe_get_device_status(ws, stream, status);
 }

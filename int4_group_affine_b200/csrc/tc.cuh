@@ -34,14 +34,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up after
-// about two seconds of device time (a single try_wait may suspend the thread for a
-// while, so the bound is on time, not on polls), raising MOE_ERR_TIMEOUT.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+// `limit_ns` of device time (a single try_wait may suspend the thread for a while,
+// so the bound is on time, not on polls), raising MOE_ERR_TIMEOUT.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > 2000000000ull) break;
+        if (globaltimer_ns() - t0 > limit_ns) break;
     }
     raise_status(status, MOE_ERR_TIMEOUT);
     return false;
@@ -49,13 +49,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
 
 // As mbar_wait, but also gives up (without raising) as soon as *ok reads zero:
 // another thread of the CTA already failed and the pipeline is being abandoned.
-__device__ __forceinline__ bool mbar_wait_ok(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* ok) {
+__device__ __forceinline__ bool mbar_wait_ok(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* ok,
+                                             uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*ok == 0) return false;
-        if (globaltimer_ns() - t0 > 2000000000ull) break;
+        if (globaltimer_ns() - t0 > limit_ns) break;
     }
     raise_status(status, MOE_ERR_TIMEOUT);
     *ok = 0;
@@ -76,14 +77,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // As mbar_wait_ok, by polling without suspension.
-__device__ __forceinline__ bool mbar_spin_ok(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* ok) {
+__device__ __forceinline__ bool mbar_spin_ok(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* ok,
+                                             uint64_t limit_ns) {
     if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 0;; ++i) {
         if (mbar_test(bar, parity)) return true;
         if ((i & 63) == 63) {
             if (*ok == 0) return false;
-            if (globaltimer_ns() - t0 > 2000000000ull) break;
+            if (globaltimer_ns() - t0 > limit_ns) break;
         }
     }
     raise_status(status, MOE_ERR_TIMEOUT);

@@ -64,7 +64,12 @@ PREFILL = MoEShape("prefill", H=2048, E=256, K=4, I=512, Is=512, T=2048, layers=
 MIXED_B1 = MixedShape("mixed_b1", H=1024, I=3072, T=1, layers=28)
 MIXED_B16 = dataclasses.replace(MIXED_B1, name="mixed_b16", T=16)
 
-MOE_SHAPES = {s.name: s for s in (TINY, DECODE_K4, DECODE_K8, MULTI_TENANT, PREFILL)}
+# The same two workloads with the weights packed at group 32 (the d1a MLX port's group size).
+DECODE_K4_G32 = dataclasses.replace(DECODE_K4, name="decode_k4_g32", group=32)
+MULTI_TENANT_G32 = dataclasses.replace(MULTI_TENANT, name="multi_tenant_g32", group=32)
+
+MOE_SHAPES = {s.name: s for s in (TINY, DECODE_K4, DECODE_K8, MULTI_TENANT, PREFILL, DECODE_K4_G32,
+                                  MULTI_TENANT_G32)}
 MIXED_SHAPES = {s.name: s for s in (MIXED_B1, MIXED_B16)}
 
 

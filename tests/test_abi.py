@@ -144,3 +144,58 @@ def test_lora_set_adapters_host_rules():
         lora_set_adapters(L, 1, 16, 32.0, [half])
     lora_set_adapters(L, 0, 0, 0.0, [])
     assert L.n_adapters == 0
+
+
+def _edge0_fake_layer(n_adapters):
+    L = _fake_layer(H=2048, E=256, K=4, I=512, Is=512)
+    if n_adapters:
+        sets = [LoraPtrs() for _ in range(n_adapters)]
+        for st in sets:
+            for p in ("gate", "up", "down", "s_gate", "s_up", "s_down"):
+                lp = getattr(st, p)
+                lp.A, lp.B = 0x50000000, 0x51000000
+        lora_set_adapters(L, n_adapters, 16, 32.0, sets)
+    return L
+
+
+@pytest.mark.parametrize("n_adapters", [0, 1, 4])
+def test_static_array_holds_256_tokens_of_the_edge0_layer(n_adapters):
+    """The documented guarantee of moe_ffn_forward_static: 256 tokens of the Edge0-shaped
+    layer fit the built-in 16 MiB array."""
+    L = _edge0_fake_layer(n_adapters)
+    assert 0 < moe_ffn_workspace_bytes(L, 256) <= 16 * 1024 * 1024
+
+
+@pytest.mark.parametrize("mutate", [lambda L: setattr(L, "top_k", 17), lambda L: setattr(L, "n_experts", 513),
+                                    lambda L: setattr(L.gate, "group", 48), lambda L: setattr(L, "hidden", 250)])
+def test_static_forward_rejects_like_forward(mutate):
+    """The static entry point returns moe_ffn_forward's own status for a bad layer, before
+    it touches the device."""
+    from int4_group_affine_b200 import moe_ffn_forward_static
+    L = _fake_layer()
+    mutate(L)
+    with pytest.raises(MoeError) as e1:
+        moe_ffn_forward(L, 0x20000000, None, 4, 0x30000000, 0x40000000, 1 << 30, stream=0)
+    with pytest.raises(MoeError) as e2:
+        moe_ffn_forward_static(L, 0x20000000, None, 4, 0x30000000, stream=0)
+    assert e1.value.status == e2.value.status
+
+
+def test_static_forward_checks_x_and_y_first():
+    from int4_group_affine_b200 import moe_ffn_forward_static
+    L = _fake_layer()
+    for x, y in ((0x20000000, 0x20000000), (0x20000008, 0x30000000), (0, 0x30000000)):
+        with pytest.raises(MoeError) as ei:
+            moe_ffn_forward_static(L, x, None, 4, y, stream=0)
+        assert ei.value.status == 1
+
+
+def test_wait_limit_setting():
+    from int4_group_affine_b200 import moe_set_wait_limit_ns, moe_wait_limit_ns
+    assert moe_wait_limit_ns() == 1000000000
+    moe_set_wait_limit_ns(2000000)
+    try:
+        assert moe_wait_limit_ns() == 2000000
+    finally:
+        moe_set_wait_limit_ns(0)
+    assert moe_wait_limit_ns() == 1000000000

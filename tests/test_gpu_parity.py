@@ -11,8 +11,9 @@ import pytest
 import oracle
 import synth
 from synth import workloads
-from tests.gpu_helpers import (REL_L2, assert_close_output, bf16_dev_to_f64, check_routing, need_cuda,
-                               near_tie_tokens, oracle_for_gpu_routing)
+from tests.gpu_helpers import (PATH_KINDS, REL_L2, TIE_GAP, assert_close_output, bf16_dev_to_f64, check_routing,
+                               check_weights, forward_with_record, need_cuda, near_tie_tokens,
+                               oracle_for_gpu_routing)
 from tests.helpers import oracle_layer, quantize_layer, rel_l2
 
 torch = pytest.importorskip("torch")
@@ -202,16 +203,24 @@ def _ffn_case(shape, seed, T=None, n_adapters=None, lora_zero_B=False):
     return t, x, aid
 
 
-def _check_ffn(shape, t, x, aid, n_adapters=None, what=""):
-    _, ly = _mods()
+def _check_ffn(shape, t, x, aid, n_adapters=None, what="", path=None):
+    """The forward against the oracle: the routing the forward itself used (bit-exact
+    outside near ties, weights within fp32 rounding), then the output, with near ties
+    resolved by the forward's own choice.  `path` names the kernels the call must run."""
+    m, ly = _mods()
     L = oracle_layer(shape, t, n_adapters=n_adapters)
     d = ly.DeviceLayer.from_host(shape, t, n_adapters=n_adapters)
-    y = bf16_dev_to_f64(_gpu_ffn(d, x, aid))
-    y_ref, idx_r, _, _, logits_r = L.ffn(x, aid)
-    # the GPU's routing (from moe_router_topk, same kernels) decides which oracle output applies
-    ties = near_tie_tokens(logits_r, shape.K)
+    T = x.shape[0]
+    ws, nb = d.workspace(T)
+    yd, idx_g, w_g, kinds = forward_with_record(m, d, ly.to_device(x), None if aid is None else ly.to_device(aid),
+                                                T, ws, nb)
+    if path is not None:
+        assert PATH_KINDS[path] <= kinds, (what, path, kinds)
+    y = bf16_dev_to_f64(yd)
+    y_ref, idx_r, w_r, _, logits_r = L.ffn(x, aid)
+    ties = check_routing(idx_g, idx_r, logits_r, shape.K)
+    check_weights(idx_g, w_g, idx_r, w_r, ties)
     if ties.any():
-        idx_g = _gpu_router(t, shape, x, x.shape[0])[0]
         y_ref = oracle_for_gpu_routing(L, x, aid, idx_g, logits_r, y_ref)
     return assert_close_output(y, y_ref, what), y, y_ref
 
@@ -220,7 +229,21 @@ def _check_ffn(shape, t, x, aid, n_adapters=None, what=""):
 def test_ffn_tiny(T):
     shape = workloads.TINY
     t, x, aid = _ffn_case(shape, 400, T=T)
-    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T)
+    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T, path="decode" if T < 9 else "tensor_core")
+
+
+@pytest.mark.parametrize("variant,T", [("kE", 4), ("kE", 8), ("rank64", 3), ("rank64", 8)])
+def test_ffn_tiny_cuda_core_path(variant, T):
+    """Calls the fused decode kernel declines (more than 32 jobs, or a LoRA rank above
+    32) with fewer tokens than the tensor-core path takes: the multi-kernel CUDA-core
+    path (router, top-K, index build, LoRA-A, gate/up, down, combine kernels)."""
+    shape = workloads.TINY
+    if variant == "kE":
+        shape = dataclasses.replace(shape, K=shape.E)
+    else:
+        shape = dataclasses.replace(shape, rank=64, n_adapters=2, random_adapters=True)
+    t, x, aid = _ffn_case(shape, 415, T=T)
+    _check_ffn(shape, t, x, aid, what="%s T=%d" % (variant, T), path="cuda_core")
 
 
 @pytest.mark.parametrize("variant", ["k1", "kE", "no_lora", "no_shared", "no_sgate", "multi_adapter", "bias",
@@ -411,14 +434,63 @@ def test_full_size_pack_bit_exact(full_layer):
             assert np.array_equal(got.ravel(), t[name + suf].ravel()), name + suf
 
 
-@pytest.mark.parametrize("K,T", [(4, 1), (8, 1), (4, 3)])
+@pytest.mark.parametrize("K,T", [(4, 1), (8, 1), (4, 3), (4, 6)])
 def test_full_size_decode(full_layer, K, T):
     shape0, w, t = full_layer
     shape = dataclasses.replace(workloads.DECODE_K4, K=K)
     tt = dict(t)
     tt["logit_bias"] = None
     x, _ = workloads.moe_inputs(shape, seed=500 + K, T=T)
-    _check_ffn(shape, tt, x, None, n_adapters=1, what="decode K=%d T=%d" % (K, T))
+    _check_ffn(shape, tt, x, None, n_adapters=1, what="decode K=%d T=%d" % (K, T), path="decode")
+
+
+@pytest.mark.parametrize("T", [4, 5, 8])
+def test_full_size_cuda_core_top8(full_layer, T):
+    """Top-8 (the Edge0 config's K) at 4-8 tokens: 36-72 jobs, more than the fused decode
+    kernel takes and fewer tokens than the tensor-core path takes, so the CUDA-core
+    kernels run it; the routing comes from the CUDA-core router and top-K kernels."""
+    shape0, w, t = full_layer
+    shape = workloads.DECODE_K8
+    tt = dict(t)
+    tt["logit_bias"] = None
+    x, _ = workloads.moe_inputs(shape, seed=530 + T, T=T)
+    _check_ffn(shape, tt, x, None, n_adapters=1, what="top-8 T=%d" % T, path="cuda_core")
+
+
+@pytest.fixture(scope="module")
+def full_layer_rank64():
+    """The Edge0-shaped layer with one rank-64 adapter set (alpha 128)."""
+    shape = dataclasses.replace(workloads.DECODE_K4, rank=64, alpha=128.0)
+    w = workloads.moe_weights(shape, seed=3)
+    return shape, quantize_layer(w)
+
+
+@pytest.mark.parametrize("T", [1, 2, 8])
+def test_full_size_cuda_core_rank64(full_layer_rank64, T):
+    """A LoRA rank above the fused decode kernel's 32 at decode sizes: CUDA-core path."""
+    shape, t = full_layer_rank64
+    x, _ = workloads.moe_inputs(shape, seed=540 + T, T=T)
+    _check_ffn(shape, t, x, None, what="rank 64 T=%d" % T, path="cuda_core")
+
+
+@pytest.mark.parametrize("T", [5, 2048])
+def test_full_size_router_topk_entry(full_layer, T):
+    """moe_router_topk at the Edge0 shape: the CUDA-core router kernel (5 tokens) and the
+    tensor-core router (2048 tokens); indices bit-exact outside near ties."""
+    shape0, w, t = full_layer
+    shape = workloads.PREFILL
+    tt = dict(t)
+    tt["logit_bias"] = None
+    L = oracle_layer(shape, tt, n_adapters=1)
+    x, _ = workloads.moe_inputs(shape, seed=550 + T, T=T)
+    idx, wts, sg, logits = _gpu_router(tt, shape, x, T)
+    z_ref, gs_ref = L.router(x)
+    idx_r, w_r = oracle.topk(z_ref, shape.K)
+    # logit error well inside the near-tie margin, which is what makes the tie exclusion sound
+    assert np.max(np.abs(logits - z_ref)) < 0.5 * TIE_GAP
+    ties = check_routing(idx, idx_r, z_ref, shape.K)
+    check_weights(idx, wts, idx_r, w_r, ties)
+    assert np.allclose(sg, 1.0 / (1.0 + np.exp(-gs_ref)), rtol=1e-6, atol=1e-6)
 
 
 @pytest.mark.parametrize("case", ["decode", "multi_tenant"])
@@ -445,26 +517,104 @@ def test_full_size_multi_tenant(full_layer):
     _check_ffn(shape, t, x, aid, what="multi-tenant T=64")
 
 
-def test_full_size_prefill_layer_sampled(full_layer):
-    """All 2048 tokens on the GPU; the oracle recomputes a sample of them one by one."""
-    _, ly = _mods()
+def _chunk_sample(T, seed, extra):
+    """First and last token of every 32-token chunk plus `extra` random tokens."""
+    edges = np.concatenate([np.arange(0, T, 32), np.minimum(np.arange(31, T + 31, 32), T - 1)])
+    return np.unique(np.concatenate([edges, synth.randint(seed, "sample", (extra,), 0, T - 1)]))
+
+
+def test_full_size_prefill_layer(full_layer):
+    """All 2048 tokens on the GPU (tensor-core path).  The routing the forward used is
+    checked for every token against the oracle's router; the outputs of 256+ tokens (the
+    first and last of each 32-token chunk and a random sample) are recomputed one by one."""
+    m, ly = _mods()
     shape0, w, t = full_layer
     shape = workloads.PREFILL
     tt = dict(t)
     tt["logit_bias"] = None
     x, _ = workloads.moe_inputs(shape, seed=510)
     d = ly.DeviceLayer.from_host(shape, tt, n_adapters=1)
-    y = bf16_dev_to_f64(_gpu_ffn(d, x))
-    L = oracle_layer(shape, tt, n_adapters=1)
-    sample = np.unique(np.concatenate([[0, 1, 31, 32, 1023, 2046, 2047],
-                                       synth.randint(510, "sample", (17,), 0, shape.T - 1)]))
-    y_ref, idx_r, _, _, logits_r = L.ffn(x[sample])
-    ties = near_tie_tokens(logits_r, shape.K)
-    if ties.any():
-        idx_g = _gpu_router(tt, shape, x[sample], len(sample))[0]
-        y_ref = oracle_for_gpu_routing(L, x[sample], None, idx_g, logits_r, y_ref)
-    assert_close_output(y[sample], y_ref, "prefill sample")
+    ws, nb = d.workspace(shape.T)
+    yd, idx_g, w_g, kinds = forward_with_record(m, d, ly.to_device(x), None, shape.T, ws, nb)
+    assert PATH_KINDS["tensor_core"] <= kinds and "tc_router" in kinds, kinds
+    y = bf16_dev_to_f64(yd)
     assert np.all(np.isfinite(y))
+    L = oracle_layer(shape, tt, n_adapters=1)
+    z_ref, _ = L.router(x)
+    idx_r, w_r = oracle.topk(z_ref, shape.K)
+    ties = check_routing(idx_g, idx_r, z_ref, shape.K)
+    check_weights(idx_g, w_g, idx_r, w_r, ties)
+    sample = _chunk_sample(shape.T, 510, 128)
+    assert len(sample) >= 256
+    y_ref, _, _, _, logits_r = L.ffn(x[sample])
+    if ties[sample].any():
+        y_ref = oracle_for_gpu_routing(L, x[sample], None, idx_g[sample], logits_r, y_ref)
+    assert_close_output(y[sample], y_ref, "prefill sample")
+
+
+@pytest.fixture(scope="module")
+def stack_layers():
+    """Three distinct Edge0-shaped layers (one adapter set each), packed by the oracle."""
+    shape = workloads.PREFILL
+    out = []
+    for l in range(3):
+        t = quantize_layer(workloads.moe_weights(shape, seed=7, layer=l))
+        t["logit_bias"] = None
+        t["lora"] = t["lora"][:1]
+        out.append(t)
+    return shape, out
+
+
+def test_full_size_prefill_stack_teacher_forced(stack_layers):
+    """The 2048-token prefill stack, block by block (RMSNorm, FFN, residual): each GPU block
+    output is compared with the oracle's block run on that block's GPU input (teacher
+    forcing) for 256+ sampled tokens.  Then 40 blocks (the three layers in turn) run on the
+    GPU and 16 tokens go through the same 40 blocks in the oracle, free-running: the
+    end-to-end drift is printed, not gated."""
+    m, ly = _mods()
+    shape, ts = stack_layers
+    T = shape.T
+    x0, _ = workloads.moe_inputs(shape, seed=560)
+    devs = [ly.DeviceLayer.from_host(shape, t) for t in ts]
+    Ls = [oracle_layer(shape, t) for t in ts]
+    ws, nb = devs[0].workspace(T)
+    sample = _chunk_sample(T, 560, 128)
+    xd = ly.to_device(x0)
+    for l, (d, L) in enumerate(zip(devs, Ls)):
+        yd, idx_g, _, kinds = forward_with_record(m, d, xd, None, T, ws, nb, block_eps=1e-6)
+        assert "rmsnorm" in kinds and PATH_KINDS["tensor_core"] <= kinds, kinds
+        x_in = ly.to_host(xd, np.uint16)
+        out = bf16_dev_to_f64(yd)
+        ref = synth.bf16_to_f32(L.block(x_in[sample], eps=1e-6)).astype(np.float64)
+        # tokens whose normalised input sits at a routing near tie: the oracle block with
+        # the forward's own routing
+        xn = oracle.rmsnorm_bf16(x_in[sample], shape.H, 1e-6)
+        y_ref, _, _, _, logits_r = L.ffn(xn)
+        ties = near_tie_tokens(logits_r, shape.K)
+        if ties.any():
+            y_alt = oracle_for_gpu_routing(L, xn, None, idx_g[sample], logits_r, y_ref)
+            xs = synth.bf16_to_f32(x_in[sample]).astype(np.float64)
+            ref[ties] = synth.bf16_to_f32(synth.bf16((xs + y_alt)[ties])).astype(np.float64)
+        assert_close_block(out[sample], ref, synth.bf16_to_f32(x_in[sample]).astype(np.float64))
+        xd = yd
+    # free-running drift over 40 blocks
+    n_layers = shape.layers
+    xa = ly.to_device(x0)
+    xb = torch.empty_like(xa)
+    for l in range(n_layers):
+        m.moe_block_forward(devs[l % 3].L, xa, None, T, 1e-6, xb, ws, nb)
+        xa, xb = xb, xa
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status(ws) == 0
+    g = bf16_dev_to_f64(xa)
+    few = sample[:16]
+    xr = x0[few]
+    for l in range(n_layers):
+        xr = Ls[l % 3].block(xr, eps=1e-6)
+    r = synth.bf16_to_f32(xr).astype(np.float64)
+    assert np.all(np.isfinite(g))
+    print("40-block drift over %d tokens: rel-L2 %.3e, max-abs %.3e (max |x| %.2f)" % (
+        len(few), rel_l2(g[few], r), np.max(np.abs(g[few] - r)), np.max(np.abs(r))))
 
 
 # ------------------------------------------------------------------ mixed layout

@@ -74,6 +74,23 @@ def test_static_forward_follows_a_different_shape():
         assert_close_output(bf16_dev_to_f64(y), bf16_dev_to_f64(_reference(d, xd, None, T)), "T=%d" % T)
 
 
+def test_static_status_word_reports_device_errors():
+    """The built-in array's status word: MOE_OK after a clean call, MOE_ERR_DEVICE_INDEX
+    (5) after a call with an adapter id out of range, and cleared by the read."""
+    import int4_group_affine_b200 as m
+    from int4_group_affine_b200.layer import to_device
+    shape = dataclasses.replace(workloads.TINY, n_adapters=2)
+    d = _layer(shape, seed=930)
+    x, _ = workloads.moe_inputs(shape, seed=930, T=4)
+    xd = to_device(x)
+    y = torch.empty_like(xd)
+    m.moe_ffn_forward_static(d.L, xd, to_device(np.array([0, 1, -1, 0], np.int32)), 4, y)
+    assert m.moe_ffn_static_device_status() == 0
+    m.moe_ffn_forward_static(d.L, xd, to_device(np.array([0, 7, 1, -1], np.int32)), 4, y)
+    assert m.moe_ffn_static_device_status() == 5
+    assert m.moe_ffn_static_device_status() == 0  # read and cleared
+
+
 def test_static_forward_refuses_oversize():
     import int4_group_affine_b200 as m
     from int4_group_affine_b200 import MoeError
