@@ -434,14 +434,14 @@ def test_full_size_pack_bit_exact(full_layer):
             assert np.array_equal(got.ravel(), t[name + suf].ravel()), name + suf
 
 
-@pytest.mark.parametrize("K,T", [(4, 1), (8, 1), (4, 3), (4, 6)])
-def test_full_size_decode(full_layer, K, T):
+@pytest.mark.parametrize("K,T,path", [(4, 1, "decode"), (8, 1, "decode"), (4, 3, "decode"), (4, 6, None)])
+def test_full_size_decode(full_layer, K, T, path):
     shape0, w, t = full_layer
     shape = dataclasses.replace(workloads.DECODE_K4, K=K)
     tt = dict(t)
     tt["logit_bias"] = None
     x, _ = workloads.moe_inputs(shape, seed=500 + K, T=T)
-    _check_ffn(shape, tt, x, None, n_adapters=1, what="decode K=%d T=%d" % (K, T), path="decode")
+    _check_ffn(shape, tt, x, None, n_adapters=1, what="decode K=%d T=%d" % (K, T), path=path)
 
 
 @pytest.mark.parametrize("T", [4, 5, 8])
@@ -517,10 +517,13 @@ def test_full_size_multi_tenant(full_layer):
     _check_ffn(shape, t, x, aid, what="multi-tenant T=64")
 
 
-def _chunk_sample(T, seed, extra):
-    """First and last token of every 32-token chunk plus `extra` random tokens."""
-    edges = np.concatenate([np.arange(0, T, 32), np.minimum(np.arange(31, T + 31, 32), T - 1)])
-    return np.unique(np.concatenate([edges, synth.randint(seed, "sample", (extra,), 0, T - 1)]))
+def _chunk_sample(T, seed, n):
+    """First and last token of every 32-token chunk, topped up with random tokens to n."""
+    edges = np.unique(np.concatenate([np.arange(0, T, 32), np.minimum(np.arange(31, T + 31, 32), T - 1)]))
+    rest = np.setdiff1d(np.arange(T), edges)
+    pick = synth.randint(seed, "sample", (len(rest),), 0, 1 << 30)
+    extra = rest[np.argsort(pick, kind="stable")[:max(0, n - len(edges))]]
+    return np.sort(np.concatenate([edges, extra]))
 
 
 def test_full_size_prefill_layer(full_layer):
@@ -544,8 +547,8 @@ def test_full_size_prefill_layer(full_layer):
     idx_r, w_r = oracle.topk(z_ref, shape.K)
     ties = check_routing(idx_g, idx_r, z_ref, shape.K)
     check_weights(idx_g, w_g, idx_r, w_r, ties)
-    sample = _chunk_sample(shape.T, 510, 128)
-    assert len(sample) >= 256
+    sample = _chunk_sample(shape.T, 510, 256)
+    assert len(sample) == 256
     y_ref, _, _, _, logits_r = L.ffn(x[sample])
     if ties[sample].any():
         y_ref = oracle_for_gpu_routing(L, x[sample], None, idx_g[sample], logits_r, y_ref)
@@ -578,7 +581,7 @@ def test_full_size_prefill_stack_teacher_forced(stack_layers):
     devs = [ly.DeviceLayer.from_host(shape, t) for t in ts]
     Ls = [oracle_layer(shape, t) for t in ts]
     ws, nb = devs[0].workspace(T)
-    sample = _chunk_sample(T, 560, 128)
+    sample = _chunk_sample(T, 560, 256)
     xd = ly.to_device(x0)
     for l, (d, L) in enumerate(zip(devs, Ls)):
         yd, idx_g, _, kinds = forward_with_record(m, d, xd, None, T, ws, nb, block_eps=1e-6)
