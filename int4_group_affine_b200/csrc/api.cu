@@ -119,9 +119,12 @@ WsPlan plan_of(const Dims& d) {
         o = align_up(o + bytes);
         return at;
     };
-    p.status = take(16);  // status word, n_active and the decode barrier share the first 256 bytes
+    p.status = take(16);  // status word, n_active and the decode ticket counter share the first 256 bytes
     p.n_active = p.status + 4;
     p.bar = p.status + 8;
+    // the chain decode kernel's tagged words: first after the header and sized for the
+    // layer shape alone, so no other region of any T of this shape ever overlaps them
+    p.slots = take(chain_slot_words(d.E, d.K, d.I, d.Is, d.r) * 8);
     p.idx = take((size_t)d.T * d.K * 4);
     p.w = take((size_t)d.T * d.K * 4);
     p.sg = take((size_t)d.T * 4);
@@ -269,8 +272,25 @@ moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* ada
 // caller runs the multi-kernel path instead; otherwise *st is the launch result.
 bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, int T, int block, float eps,
                 uint16_t* y, const Dims& d, const WsPlan& p, void* ws, cudaStream_t s, moe_status* st) {
-    if (d.T > MOEQ_DECODE_MAX_TOKENS || d.J > MOEQ_DECODE_MAX_JOBS) return false;
+    if (d.T > MOEQ_DECODE_MAX_TOKENS) return false;
     const LayerArgs la = args_of(L);
+    if (chain_supported(la, T)) {  // one to four tokens: the chain kernel
+        char* b = (char*)ws;
+        ChainScratch cs;
+        cs.tick = (unsigned long long*)(b + p.bar);
+        cs.slots = (uint64_t*)(b + p.slots);
+        cs.status = (int32_t*)(b + p.status);
+        cs.idx_out = (int32_t*)(b + p.idx);
+        cs.w_out = (float*)(b + p.w);
+        const cudaError_t e = launch_chain(la, x, adapter_id, y, T, block, eps, cs, s);
+        if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) {
+            *st = e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+            if (e == cudaSuccess) timing_mark(kDecodeChain, s);
+            return true;
+        }
+        (void)cudaGetLastError();
+    }
+    if (d.J > MOEQ_DECODE_MAX_JOBS) return false;
     if (!decode_supported(la, T, nullptr)) return false;
     char* b = (char*)ws;
     DecodeScratch sc;
@@ -473,7 +493,7 @@ size_t moe_ffn_workspace_bytes(const moe_layer* layer, int32_t T) {
 
 moe_status moe_workspace_init(void* workspace, size_t ws_bytes, moe_stream stream) {
     if (!workspace || !aligned(workspace, kAlign) || ws_bytes < kAlign) return MOE_ERR_WORKSPACE;
-    CHECK_CUDA(cudaMemsetAsync(workspace, 0, kAlign, (cudaStream_t)stream));
+    CHECK_CUDA(cudaMemsetAsync(workspace, 0, ws_bytes, (cudaStream_t)stream));
     return MOE_OK;
 }
 

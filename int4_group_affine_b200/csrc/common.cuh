@@ -64,6 +64,7 @@ struct Work {
 struct WsPlan {
     size_t status, n_active, idx, w, sg, logits, gs, cnt, goff, active, perm, wperm, inv, tgu, td, h, ypart, xn, xp;
     size_t bar, dts, dtg, dtdp;  // fused decode scratch (sizes zero when T is too large for it)
+    size_t slots;                // chain decode tagged words (right after the header, for every T)
     size_t total;
 };
 
@@ -118,7 +119,7 @@ struct DecodeScratch {
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
     kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kTcLoraGUKind, kTcGUKind,
-    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kKindCount
+    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kDecodeChain, kKindCount
 };
 void timing_begin(cudaStream_t s);
 void timing_mark(int kind, cudaStream_t s);
@@ -171,6 +172,21 @@ cudaError_t launch_tc_router(const moe_qtensor& router, const float* logit_bias,
 bool decode_supported(const LayerArgs& L, int T, size_t* smem_out);
 cudaError_t launch_decode(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, uint16_t* y, int T,
                           int block, float eps, const DecodeScratch& sc, cudaStream_t s);
+
+// The chain decode kernel (csrc/decode_chain.cu): one to four tokens, cross-CTA
+// hand-offs through epoch-tagged 64-bit words in a workspace region of
+// chain_slot_words(...) words that sits at a fixed place for a layer shape.
+struct ChainScratch {
+    unsigned long long* tick;  // ticket counter in the workspace header (starts zeroed)
+    uint64_t* slots;           // the tagged-word region (starts zeroed)
+    int32_t* status;
+    int32_t* idx_out;          // [T][K] routing record
+    float* w_out;
+};
+size_t chain_slot_words(int E, int K, int I, int Is, int r);
+bool chain_supported(const LayerArgs& L, int T);
+cudaError_t launch_chain(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, uint16_t* y, int T,
+                         int block, float eps, const ChainScratch& sc, cudaStream_t s);
 
 cudaError_t launch_mixed_linear(const moe_mixed_tensor& W, int G, const uint16_t* x, int T, float* y,
                                 cudaStream_t s);

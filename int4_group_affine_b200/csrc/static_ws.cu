@@ -8,6 +8,8 @@
 // caller that cannot afford the implicit device synchronisation an allocation
 // may cause.  Those callers still pass the inputs and the output; only the
 // workspace comes from here.
+#include <string.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -22,6 +24,13 @@ static __device__ __align__(256) unsigned char g_static_ws[MOEQ_STATIC_WS_BYTES]
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_dev_ptr[kMaxDevices] = {};
+// The layer shape of the last call on each device: the fused decode kernels keep
+// epoch-tagged words and counters in the workspace that are laid out by shape, so
+// the array is cleared whenever the shape changes.
+struct ShapeKey {
+    int32_t H, E, K, I, Is, r, valid;
+};
+ShapeKey g_last[kMaxDevices] = {};
 
 // Device address of g_static_ws on the current device, looked up once per device.
 moe_status static_ws_address(void** out) {
@@ -55,9 +64,21 @@ extern "C" moe_status moe_ffn_forward_static(const moe_layer* layer, const uint1
     st = static_ws_address(&ws);
     if (st != MOE_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    // The array keeps the previous call's contents: the status header must
-    // start at zero (everything else is written before it is read).
-    if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess) return MOE_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    const ShapeKey key = {layer->hidden, layer->n_experts, layer->top_k, layer->inter,
+                          layer->s_gate.packed ? layer->shared_inter : 0, layer->n_adapters > 0 ? layer->rank : 0, 1};
+    bool same;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        same = memcmp(&g_last[dev], &key, sizeof(key)) == 0;
+        g_last[dev] = key;
+    }
+    // The array keeps the previous call's contents.  A call with the shape of the
+    // previous one needs only the status word cleared (the decode counters and tagged
+    // words carry over by design); a new shape starts from a cleared array.
+    if (cudaMemsetAsync(ws, 0, same ? sizeof(int32_t) : (size_t)MOEQ_STATIC_WS_BYTES, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
     return moe_ffn_forward(layer, x, adapter_id, T, y, ws, need, stream);
 }
 

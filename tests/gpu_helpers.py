@@ -120,8 +120,16 @@ def forward_with_record(m, d, xd, ad, T, ws, nb, block_eps=None):
     return y, idx.cpu().numpy(), w.cpu().numpy(), kinds
 
 
-# kernel kinds that identify each execution path of the forward
-PATH_KINDS = {"decode": {"decode_fused"}, "cuda_core": {"gate_up", "down"}, "tensor_core": {"tc_gate_up", "tc_down"}}
+# kernel kinds that identify each execution path of the forward: "chain" and "fused" are
+# the two single-kernel decode paths, "decode" either of them
+PATH_KINDS = {"chain": {"decode_chain"}, "fused": {"decode_fused"}, "cuda_core": {"gate_up", "down"},
+              "tensor_core": {"tc_gate_up", "tc_down"}}
+
+
+def path_ran(path, kinds):
+    if path == "decode":
+        return bool({"decode_chain", "decode_fused"} & kinds)
+    return PATH_KINDS[path] <= kinds
 
 
 def oracle_for_gpu_routing(L, x, aid, idx_gpu, logits_ref, y_ref):

@@ -11,7 +11,7 @@ import pytest
 import oracle
 import synth
 from synth import workloads
-from tests.gpu_helpers import (PATH_KINDS, REL_L2, TIE_GAP, assert_close_output, bf16_dev_to_f64, check_routing,
+from tests.gpu_helpers import (PATH_KINDS, REL_L2, TIE_GAP, path_ran, assert_close_output, bf16_dev_to_f64, check_routing,
                                check_weights, forward_with_record, need_cuda, near_tie_tokens,
                                oracle_for_gpu_routing)
 from tests.helpers import oracle_layer, quantize_layer, rel_l2
@@ -215,7 +215,7 @@ def _check_ffn(shape, t, x, aid, n_adapters=None, what="", path=None):
     yd, idx_g, w_g, kinds = forward_with_record(m, d, ly.to_device(x), None if aid is None else ly.to_device(aid),
                                                 T, ws, nb)
     if path is not None:
-        assert PATH_KINDS[path] <= kinds, (what, path, kinds)
+        assert path_ran(path, kinds), (what, path, kinds)
     y = bf16_dev_to_f64(yd)
     y_ref, idx_r, w_r, _, logits_r = L.ffn(x, aid)
     ties = check_routing(idx_g, idx_r, logits_r, shape.K)
@@ -229,7 +229,16 @@ def _check_ffn(shape, t, x, aid, n_adapters=None, what="", path=None):
 def test_ffn_tiny(T):
     shape = workloads.TINY
     t, x, aid = _ffn_case(shape, 400, T=T)
-    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T, path="decode" if T < 9 else "tensor_core")
+    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T, path="chain" if T <= 4 else "tensor_core")
+
+
+@pytest.mark.parametrize("T", [5, 8])
+def test_ffn_tiny_fused_decode_path(T):
+    """Five to eight tokens with at most 32 jobs: the older fused decode kernel (grid
+    barriers, dedicated LoRA-A CTAs), which takes what the chain kernel does not."""
+    shape = workloads.TINY
+    t, x, aid = _ffn_case(shape, 405, T=T)
+    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T, path="fused")
 
 
 @pytest.mark.parametrize("variant,T", [("kE", 4), ("kE", 8), ("rank64", 3), ("rank64", 8)])
@@ -247,8 +256,14 @@ def test_ffn_tiny_cuda_core_path(variant, T):
 
 
 @pytest.mark.parametrize("variant", ["k1", "kE", "no_lora", "no_shared", "no_sgate", "multi_adapter", "bias",
-                                     "group32", "group32_decode", "rank24", "rank64"])
+                                     "group32", "group32_decode", "rank24", "rank64", "k1_chain", "no_lora_chain",
+                                     "no_shared_chain", "no_sgate_chain", "multi_adapter_chain", "bias_chain",
+                                     "rank24_chain"])
 def test_ffn_tiny_variants(variant):
+    """Layer variants on the tensor-core path (19 tokens) and, for the _chain ones, on the
+    chain decode kernel (3 tokens)."""
+    chain = variant.endswith("_chain")
+    variant = variant[:-6] if chain else variant
     shape = workloads.TINY
     na = None
     if variant == "k1":
@@ -263,7 +278,7 @@ def test_ffn_tiny_variants(variant):
         shape = dataclasses.replace(shape, group=32)
     elif variant in ("rank24", "rank64"):  # LoRA-A products wider than one 32-column warp group
         shape = dataclasses.replace(shape, rank=int(variant[4:]), n_adapters=2, random_adapters=True)
-    t, x, aid = _ffn_case(shape, 410, T=3 if variant == "group32_decode" else 19)
+    t, x, aid = _ffn_case(shape, 410, T=3 if (variant == "group32_decode" or chain) else 19)
     if variant in ("group32", "group32_decode"):
         w = workloads.moe_weights(shape, seed=410)
         t = quantize_layer(w, group=32)
@@ -279,7 +294,8 @@ def test_ffn_tiny_variants(variant):
     if variant == "multi_adapter":
         aid = aid.copy()
         aid[::5] = -1  # some tokens with the base only
-    _check_ffn(shape, t, x, aid, n_adapters=na, what=variant)
+    _check_ffn(shape, t, x, aid, n_adapters=na, what=variant + (" (chain)" if chain else ""),
+               path="chain" if (chain or variant == "group32_decode") else None)
 
 
 def test_zero_B_equals_base_bitwise():
@@ -326,6 +342,54 @@ def test_bad_adapter_flags_status_and_falls_back_to_base():
     torch.cuda.synchronize()
     assert m.moe_get_device_status(ws) == 0
     assert torch.equal(y, y2)
+
+
+@pytest.mark.parametrize("T", [3, 1])
+def test_block_tiny_chain(T):
+    """The pre-norm residual block on the chain decode kernel (RMSNorm inside it)."""
+    m, ly = _mods()
+    shape = workloads.TINY
+    t, x, aid = _ffn_case(shape, 455, T=T)
+    L = oracle_layer(shape, t)
+    d = ly.DeviceLayer.from_host(shape, t)
+    ws, nb = d.workspace(T)
+    yd, idx_g, _, kinds = forward_with_record(m, d, ly.to_device(x), None, T, ws, nb, block_eps=1e-6)
+    assert path_ran("chain", kinds), kinds
+    ref = synth.bf16_to_f32(L.block(x, eps=1e-6)).astype(np.float64)
+    assert_close_block(bf16_dev_to_f64(yd), ref, synth.bf16_to_f32(x).astype(np.float64))
+
+
+def test_bounded_wait_runs_out_and_reports_timeout():
+    """A bounded device wait that cannot be satisfied gives up, reports MOE_ERR_TIMEOUT and
+    leaves the context usable.  The workspace's ticket counter (header bytes 8..15) is set
+    to 1 instead of a multiple of the grid, so one CTA of the chain decode kernel takes a
+    different epoch from the others and no CTA ever sees all the words it polls for; with a
+    2 ms wait limit every CTA gives up.  After re-initialising the workspace the same call
+    runs normally."""
+    m, ly = _mods()
+    shape = workloads.TINY
+    t, x, aid = _ffn_case(shape, 470, T=1)
+    d = ly.DeviceLayer.from_host(shape, t)
+    ws, nb = d.workspace(1)
+    xd = ly.to_device(x)
+    y = torch.zeros_like(xd)
+    ws.view(torch.int64)[1] = 1
+    m.moe_set_wait_limit_ns(2_000_000)
+    try:
+        m.moe_timing_enable(True)
+        m.moe_ffn_forward(d.L, xd, None, 1, y, ws, nb)
+        torch.cuda.synchronize()
+        kinds = set(m.moe_timing_collect())
+    finally:
+        m.moe_timing_enable(False)
+        m.moe_set_wait_limit_ns(0)
+    assert "decode_chain" in kinds
+    assert m.moe_get_device_status(ws) == 6
+    m.moe_workspace_init(ws, nb)
+    yd, _, _, kinds = forward_with_record(m, d, xd, None, 1, ws, nb)
+    assert path_ran("chain", kinds)
+    y_ref = oracle_layer(shape, t).ffn(x)[0]
+    assert_close_output(bf16_dev_to_f64(yd), y_ref, "after a timeout")
 
 
 def test_block_tiny():
@@ -434,7 +498,8 @@ def test_full_size_pack_bit_exact(full_layer):
             assert np.array_equal(got.ravel(), t[name + suf].ravel()), name + suf
 
 
-@pytest.mark.parametrize("K,T,path", [(4, 1, "decode"), (8, 1, "decode"), (4, 3, "decode"), (4, 6, None)])
+@pytest.mark.parametrize("K,T,path", [(4, 1, "chain"), (8, 1, "chain"), (4, 2, "chain"), (4, 3, "chain"),
+                                      (4, 6, None)])
 def test_full_size_decode(full_layer, K, T, path):
     shape0, w, t = full_layer
     shape = dataclasses.replace(workloads.DECODE_K4, K=K)
