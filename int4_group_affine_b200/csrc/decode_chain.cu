@@ -233,18 +233,24 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
         } else if (lane >= 1 && lane < 13) {
             const int w = lane - 1, k = w % 3, g = w / 3;  // g: router, shared gate, s_gate, s_up
             const moe_qtensor& q = g == 0 ? L.router : g == 1 ? L.shared_gate : g == 2 ? L.s_gate : L.s_up;
-            const int bits = g < 2 ? 8 : 4;
-            const int row0 = g == 0 ? ra0 : g == 1 ? 0 : s_lo;
-            const int n = g == 0 ? nra : g == 1 ? (L.has_sgate ? 1 : 0) : nsr;
-            const int ng = q.packed ? H / q.group : 0;
-            const void* src = nullptr;
-            uint32_t bytes = 0;
-            if (n > 0 && q.packed) {
-                src = k == 0 ? (const void*)(q.packed + (int64_t)row0 * (H * bits / 32))
-                             : (const void*)((k == 1 ? q.scales : q.biases) + (int64_t)row0 * ng);
-                bytes = k == 0 ? (uint32_t)(n * H * bits / 8) : (uint32_t)(n * ng * 2);
+            if (g == 1) {  // the shared-gate row is read by every CTA straight from global memory (L2)
+                s_aw[w] = !L.has_sgate ? nullptr
+                          : k == 0     ? reinterpret_cast<const unsigned char*>(q.packed)
+                                       : reinterpret_cast<const unsigned char*>(k == 1 ? q.scales : q.biases);
+            } else {
+                const int bits = g < 2 ? 8 : 4;
+                const int row0 = g == 0 ? ra0 : s_lo;
+                const int n = g == 0 ? nra : nsr;
+                const int ng = q.packed ? H / q.group : 0;
+                const void* src = nullptr;
+                uint32_t bytes = 0;
+                if (n > 0 && q.packed) {
+                    src = k == 0 ? (const void*)(q.packed + (int64_t)row0 * (H * bits / 32))
+                                 : (const void*)((k == 1 ? q.scales : q.biases) + (int64_t)row0 * ng);
+                    bytes = k == 0 ? (uint32_t)(n * H * bits / 8) : (uint32_t)(n * ng * 2);
+                }
+                s_aw[w] = win(wa + P.a_off[w], src, bytes, &s_bar[0], &tx);
             }
-            s_aw[w] = win(wa + P.a_off[w], src, bytes, &s_bar[0], &tx);
         }
         tx = warp_total(tx);
         if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[0], tx);
@@ -936,7 +942,7 @@ bool plan_chain(const LayerArgs& L, int T, int NB, CPlan* P) {
     if (T < 1 || T > kCMaxT || TK > kCMaxTK || r > kCMaxR || NB < 1 || NB > MOEQ_DECODE_MAX_CTAS) return false;
     if (E > MOEQ_MAX_EXPERTS || H % 32 || H > 4096 || I % 32 || I > 4096 || (sh && (Is % 32 || Is > 4096))) return false;
     if (!cwin_ok(L.router) || !cwin_ok(L.gate) || !cwin_ok(L.up) || !cwin_ok(L.down)) return false;
-    if (L.has_sgate && !cwin_ok(L.shared_gate)) return false;
+    if (L.has_sgate && (((uintptr_t)L.shared_gate.packed & 15) || L.shared_gate.bits != 8)) return false;
     if (sh && (!cwin_ok(L.s_gate) || !cwin_ok(L.s_up) || !cwin_ok(L.s_down))) return false;
     if (L.router.bits != 8 || L.gate.bits != 4 || L.up.bits != 4 || L.down.bits != 4) return false;
     if (lora) {  // LoRA rows move by bulk copies: 16-byte aligned factors, rows of whole 16-byte pieces
@@ -973,7 +979,7 @@ bool plan_chain(const LayerArgs& L, int T, int NB, CPlan* P) {
     {  // phase-R windows
         size_t wsz = 0;
         const moe_qtensor* qs[4] = {&L.router, &L.shared_gate, &L.s_gate, &L.s_up};
-        const int rows[4] = {P->perA, L.has_sgate ? 1 : 0, P->perS, P->perS};
+        const int rows[4] = {P->perA, 0, P->perS, P->perS};  // (the shared-gate row needs no window)
         for (int g = 0; g < 4; ++g) {
             const moe_qtensor& q = *qs[g];
             const int bits = g < 2 ? 8 : 4, ng = q.packed ? H / q.group : 0;

@@ -92,6 +92,9 @@ def _get():
             "orc_bf16_round_nearest": (ctypes.c_uint16, [D]),
             "orc_bf16_value": (D, [ctypes.c_uint16]),
             "orc_threads": (I, []),
+            "orc_fp16_value": (D, [ctypes.c_uint16]),
+            "orc_gelu_erf": (D, [D]),
+            "orc_prerouter": (I, [P, P, P, P, I, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -359,3 +362,34 @@ def rmsnorm_bf16(x_bf16, H: int, eps: float = 1e-6) -> np.ndarray:
     out = np.empty((T, H), dtype=np.uint16)
     _get().orc_rmsnorm_bf16(_p(x), T, H, float(eps), _p(out))
     return out
+
+
+class Prerouter(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("E", ctypes.c_int32), ("K", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
+                ("wl", ctypes.c_void_p), ("bl", ctypes.c_void_p)]
+
+
+def fp16_value(h: int) -> float:
+    return float(_get().orc_fp16_value(int(h)))
+
+
+def gelu_erf(v: float) -> float:
+    return float(_get().orc_gelu_erf(float(v)))
+
+
+def prerouter(H, E, K, D, w, h_bf16, exec_idx, prev_idx=None):
+    """Predicted next-layer logits [T, E] of one prerouter head.  `w` maps w1 [D, H+2E],
+    b1 [D], w2 [E, D], b2 [E], wl [E, H+2E], bl [E] to fp16 bit patterns (uint16); a
+    missing bias is zero."""
+    keep = {k: (None if w.get(k) is None else _c(w[k], np.uint16)) for k in ("w1", "b1", "w2", "b2", "wl", "bl")}
+    P = Prerouter(H, E, K, D, *[_p(keep[k]) for k in ("w1", "b1", "w2", "b2", "wl", "bl")])
+    h = _c(h_bf16, np.uint16)
+    T = h.size // H
+    ex = _c(exec_idx, np.int32)
+    pv = None if prev_idx is None else _c(prev_idx, np.int32)
+    z = np.empty((T, E), dtype=np.float64)
+    rc = _get().orc_prerouter(ctypes.byref(P), _p(h), _p(ex), _p(pv), T, _p(z))
+    if rc != 0:
+        raise ValueError("orc_prerouter rc=%d" % rc)
+    return z

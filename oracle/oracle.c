@@ -24,6 +24,8 @@
  *        _swiglu(up, gate) argument order).
  *  [ER]  "EDGERAZOR 深度解读", section 2.1 SQMP (super-group allocation, ternary
  *        and 4-bit quantisers, the matmul decomposition).
+ *  [PR]  "Edge0 项目推荐" review, 亮点一 (the prerouter head: features, fc1, exact
+ *        erf GELU, fc2, the linear_init skip, fp16 weights, the double shift).
  */
 #include "oracle.h"
 
@@ -645,5 +647,67 @@ int orc_moe_block(const orc_layer* L, const uint16_t* x, const int32_t* adapter_
         for (int64_t i = 0; i < (int64_t)T * H; ++i) x_out[i] = orc_bf16_round_nearest(orc_bf16_value(x[i]) + y[i]);
     free(xn);
     free(y);
+    return rc;
+}
+
+/* ------------------------------------------------------- prerouter head */
+
+/* IEEE 754 binary16 bit pattern -> value: sign, 5-bit exponent (bias 15), 10-bit
+ * fraction; exponent 0 is subnormal (fraction * 2^-24), exponent 31 is inf/NaN. */
+double orc_fp16_value(uint16_t h) {
+    const int sign = (h >> 15) & 1, ex = (h >> 10) & 31, fr = h & 1023;
+    double v;
+    if (ex == 0) v = ldexp((double)fr, -24);
+    else if (ex == 31) v = fr ? NAN : INFINITY;
+    else v = ldexp(1024.0 + fr, ex - 25);
+    return sign ? -v : v;
+}
+
+/* GELU in its exact form, x * Phi(x) with Phi the standard normal CDF written
+ * through erf ([PR]: "精确 erf 形式的 GELU"). */
+double orc_gelu_erf(double v) { return 0.5 * v * (1.0 + erf(v / sqrt(2.0))); }
+
+/* [PR]: layer N's head takes f = [h, onehot(executed top-K of this token),
+ * onehot(executed top-K of the previous token)] and predicts layer N+1's router
+ * logits, logits = linear_init(f) + fc2(gelu_erf(fc1(f))).  Every weight is fp16
+ * ([PR]: fp16 in training and in production); the sums here are fp64 in index
+ * order.  prev_idx NULL is an all-zero previous-token one-hot.  An expert listed
+ * twice in one top-K still sets a single one. */
+int orc_prerouter(const orc_prerouter_head* P, const uint16_t* h, const int32_t* exec_idx, const int32_t* prev_idx,
+                  int T, double* logits) {
+    const int H = P->H, E = P->E, K = P->K, D = P->D, F = H + 2 * E;
+    if (H <= 0 || E <= 0 || K <= 0 || K > E || D <= 0 || !P->w1 || !P->w2 || !P->wl) return -1;
+    double* f = (double*)malloc((size_t)F * sizeof(double));
+    double* g = (double*)malloc((size_t)D * sizeof(double));
+    int rc = 0;
+    for (int t = 0; t < T && rc == 0; ++t) {
+        for (int j = 0; j < H; ++j) f[j] = orc_bf16_value(h[(int64_t)t * H + j]);
+        for (int j = H; j < F; ++j) f[j] = 0.0;
+        for (int k = 0; k < K; ++k) {
+            const int e = exec_idx[(int64_t)t * K + k];
+            const int q = prev_idx ? prev_idx[(int64_t)t * K + k] : 0;
+            if (e < 0 || e >= E || (prev_idx && (q < 0 || q >= E))) rc = -2;
+            else {
+                f[H + e] = 1.0;
+                if (prev_idx) f[H + E + q] = 1.0;
+            }
+        }
+        if (rc) break;
+        #pragma omp parallel for schedule(static)
+        for (int d = 0; d < D; ++d) {
+            double a = P->b1 ? orc_fp16_value(P->b1[d]) : 0.0;
+            for (int j = 0; j < F; ++j) a += orc_fp16_value(P->w1[(int64_t)d * F + j]) * f[j];
+            g[d] = orc_gelu_erf(a);
+        }
+        #pragma omp parallel for schedule(static)
+        for (int e = 0; e < E; ++e) {
+            double z = (P->bl ? orc_fp16_value(P->bl[e]) : 0.0) + (P->b2 ? orc_fp16_value(P->b2[e]) : 0.0);
+            for (int j = 0; j < F; ++j) z += orc_fp16_value(P->wl[(int64_t)e * F + j]) * f[j];
+            for (int d = 0; d < D; ++d) z += orc_fp16_value(P->w2[(int64_t)e * D + d]) * g[d];
+            logits[(int64_t)t * E + e] = z;
+        }
+    }
+    free(f);
+    free(g);
     return rc;
 }

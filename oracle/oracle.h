@@ -94,6 +94,18 @@ void orc_rmsnorm_bf16(const uint16_t* x, int T, int H, double eps, uint16_t* xn)
 int orc_moe_block(const orc_layer* L, const uint16_t* x, const int32_t* adapter_id, int T,
                   double eps, uint16_t* x_out);
 
+/* Prerouter head of layer N ("Edge0 项目推荐" review, 亮点一): fp16 weights
+ * fc1 w1 [D][F], b1 [D]; fc2 w2 [E][D], b2 [E]; linear_init wl [E][F], bl [E];
+ * F = H + 2E (biases may be NULL). */
+typedef struct {
+    int32_t H, E, K, D;
+    const uint16_t *w1, *b1, *w2, *b2, *wl, *bl;
+} orc_prerouter_head;
+double orc_fp16_value(uint16_t h);
+double orc_gelu_erf(double v);
+int orc_prerouter(const orc_prerouter_head* P, const uint16_t* h, const int32_t* exec_idx, const int32_t* prev_idx,
+                  int T, double* logits);
+
 uint16_t orc_bf16_round_down(double v);
 uint16_t orc_bf16_round_up(double v);
 uint16_t orc_bf16_round_nearest(double v);

@@ -99,6 +99,11 @@ def bf16(a: np.ndarray) -> np.ndarray:
     return out
 
 
+def fp16(a: np.ndarray) -> np.ndarray:
+    """Round to IEEE binary16 (numpy's nearest-even conversion); returns the uint16 bit patterns."""
+    return np.ascontiguousarray(a, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
 def bf16_to_f32(h: np.ndarray) -> np.ndarray:
     """Widen bf16 bit patterns to fp32 (exact)."""
     return (np.ascontiguousarray(h, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)

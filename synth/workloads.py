@@ -14,7 +14,7 @@ import dataclasses
 
 import numpy as np
 
-from . import bf16, normal, randint
+from . import bf16, fp16, normal, randint, uniform
 
 
 @dataclasses.dataclass(frozen=True)
@@ -135,3 +135,46 @@ def mixed_weights(shape: MixedShape, seed: int = 0, layer: int = 0):
 def mixed_inputs(shape: MixedShape, seed: int = 0, T: int | None = None, tag: str = "mx"):
     T = shape.T if T is None else T
     return bf16(normal(seed, tag, (T, shape.H)))
+
+
+@dataclasses.dataclass(frozen=True)
+class PrerouterShape:
+    """One prerouter head: layer input width H, experts E, top-K, head hidden width D."""
+    name: str
+    H: int
+    E: int
+    K: int
+    D: int = 512
+    T: int = 1
+
+
+# The Edge0-35B heads: hidden 2048, 256 experts, top-4, head width 512, fp16.
+PREROUTER = PrerouterShape("prerouter", H=2048, E=256, K=4, D=512)
+PREROUTER_TINY = PrerouterShape("prerouter_tiny", H=64, E=8, K=2, D=16, T=5)
+
+
+def prerouter_weights(shape: PrerouterShape, seed: int = 0, layer: int = 0):
+    """fp16 bit patterns of one head: fc1 w1 [D, H+2E], b1 [D]; fc2 w2 [E, D], b2 [E];
+    linear_init wl [E, H+2E], bl [E].  Weights N(0, 1/fan_in), biases N(0, 0.1)."""
+    H, E, D = shape.H, shape.E, shape.D
+    F = H + 2 * E
+    p = "P%d/" % layer
+    return {
+        "w1": fp16(normal(seed, p + "w1", (D, F), std=F ** -0.5)),
+        "b1": fp16(normal(seed, p + "b1", (D,), std=0.1)),
+        "w2": fp16(normal(seed, p + "w2", (E, D), std=D ** -0.5)),
+        "b2": fp16(normal(seed, p + "b2", (E,), std=0.1)),
+        "wl": fp16(normal(seed, p + "wl", (E, F), std=F ** -0.5)),
+        "bl": fp16(normal(seed, p + "bl", (E,), std=0.1)),
+    }
+
+
+def prerouter_inputs(shape: PrerouterShape, seed: int = 0, T: int | None = None, tag: str = "pr"):
+    """The head's layer input h (bf16 N(0,1) [T, H]) and two top-K expert lists [T, K]
+    (K distinct experts per token, uniformly at random): the token's own executed
+    routing and the previous token's."""
+    T = shape.T if T is None else T
+    h = bf16(normal(seed, tag + "/h", (T, shape.H)))
+    ex = np.argsort(uniform(seed, tag + "/exec", (T, shape.E)), axis=1, kind="stable")[:, :shape.K].astype(np.int32)
+    pv = np.argsort(uniform(seed, tag + "/prev", (T, shape.E)), axis=1, kind="stable")[:, :shape.K].astype(np.int32)
+    return h, ex, pv
