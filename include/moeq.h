@@ -262,6 +262,57 @@ MOEQ_API moe_status moe_ffn_forward_static(const moe_layer* layer, const uint16_
  * synchronises `stream`. */
 MOEQ_API moe_status moe_ffn_static_device_status(moe_stream stream, int32_t* status);
 
+/* ------------------------------------------------ routing by a given set
+ * The forward of moe_ffn_forward with the expert set of each token given by the
+ * caller instead of taken as the top-K of the router: select device int32 [T][K].
+ * The router still runs; the weights are its softmax renormalised over the given
+ * set (w_k = exp(z_k) / sum over the set), the shared-expert scale is unchanged.
+ * This is the prerouter's "the prediction is the routing" step ("Edge0 项目推荐"
+ * review, 亮点一: the set the next layer runs for the next token is the head's
+ * prediction itself, so nothing predicted is ever discarded or re-read).  An entry
+ * outside [0, E), or repeating an earlier entry of its token, is replaced by the
+ * lowest expert index that token does not use yet and raises MOE_ERR_DEVICE_INDEX.
+ * Workspace and other arguments as for moe_ffn_forward. */
+MOEQ_API moe_status moe_ffn_forward_select(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id,
+                                           const int32_t* select, int32_t T, uint16_t* y, void* workspace,
+                                           size_t ws_bytes, moe_stream stream);
+
+/* ------------------------------------------------------ prerouter head
+ * Layer N's prerouter head ("Edge0 项目推荐" review, 亮点一): from the layer's MoE
+ * input h, the experts this token was routed to at layer N and those of the
+ * previous token, it predicts layer N+1's router logits,
+ *   f = [h, onehot(exec_idx[t]), onehot(prev_idx[t])]       (width H + 2E)
+ *   logits = linear_init(f) + fc2(gelu(fc1(f))),  gelu(v) = v * Phi(v)  (erf form)
+ * with fp16 weights (fp16 in training and production on that page) and fp32
+ * arithmetic here; its top-K (ties to the lower index) is the set layer N+1 runs
+ * for token t+1 (pass it to moe_ffn_forward_select).
+ *  h         device bf16 [T][H] (16-byte aligned)
+ *  exec_idx  device int32 [T][K]; prev_idx device int32 [T][K] or NULL (no
+ *            previous token: an all-zero one-hot).  An expert listed twice sets one
+ *            one; an entry outside [0, E) sets none and raises MOE_ERR_DEVICE_INDEX
+ *            in the workspace's status word (moe_get_device_status).
+ *  logits    device fp32 [T][E]; pred_idx device int32 [T][K] or NULL
+ *  workspace device scratch of moe_prerouter_workspace_bytes(head, T) bytes,
+ *            256-byte aligned, initialised once with moe_workspace_init.
+ * Limits: H % 8 == 0, (H + 2E) % 8 == 0, D % 8 == 0, E <= 512, 1 <= K <= min(E, 16),
+ * weights 16-byte aligned. */
+typedef struct {
+    int32_t hidden;     /* H */
+    int32_t n_experts;  /* E */
+    int32_t top_k;      /* K */
+    int32_t head_dim;   /* D, the width of fc1's output (512 for the Edge0-35B heads) */
+    const uint16_t* w1; /* fc1 fp16 [D][H + 2E] */
+    const uint16_t* b1; /* fp16 [D] or NULL */
+    const uint16_t* w2; /* fc2 fp16 [E][D] */
+    const uint16_t* b2; /* fp16 [E] or NULL */
+    const uint16_t* wl; /* linear_init fp16 [E][H + 2E] */
+    const uint16_t* bl; /* fp16 [E] or NULL */
+} moe_prerouter;
+MOEQ_API size_t moe_prerouter_workspace_bytes(const moe_prerouter* head, int32_t T);
+MOEQ_API moe_status moe_prerouter_forward(const moe_prerouter* head, const uint16_t* h, const int32_t* exec_idx,
+                                          const int32_t* prev_idx, int32_t T, float* logits, int32_t* pred_idx,
+                                          void* workspace, size_t ws_bytes, moe_stream stream);
+
 /* Pre-norm residual block for stacked layers:
  *   x_out = bf16(x + FFN(bf16(RMSNorm(x)))), RMSNorm with unit weight and eps.
  * x_out may not alias x.  Same workspace rules as moe_ffn_forward. */

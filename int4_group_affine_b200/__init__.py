@@ -11,7 +11,7 @@ import ctypes
 
 from . import _lib
 from ._lib import (FMT_AFFINE_INT4, FMT_AFFINE_INT8, FMT_MIXED_TERNARY_INT4, Layer, LoraProj, LoraPtrs,
-                   MixedTensor, QTensor, STATUS_NAMES)
+                   MixedTensor, Prerouter, QTensor, STATUS_NAMES)
 
 __all__ = [
     "MoeError", "QTensor", "MixedTensor", "LoraProj", "LoraPtrs", "Layer",
@@ -21,7 +21,8 @@ __all__ = [
     "moe_workspace_init", "moe_ffn_forward", "moe_block_forward", "moe_rmsnorm", "moe_get_device_status",
     "moe_mixed_linear", "moe_mixed_mlp_workspace_bytes", "moe_mixed_mlp_forward",
     "moe_timing_enable", "moe_timing_collect", "moe_ffn_forward_static", "moe_ffn_static_device_status",
-    "moe_ffn_routing", "moe_set_wait_limit_ns", "moe_wait_limit_ns",
+    "moe_ffn_routing", "moe_set_wait_limit_ns", "moe_wait_limit_ns", "Prerouter", "moe_ffn_forward_select",
+    "moe_prerouter_workspace_bytes", "moe_prerouter_forward",
 ]
 
 
@@ -194,3 +195,21 @@ def moe_set_wait_limit_ns(ns: int):
 
 def moe_wait_limit_ns() -> int:
     return int(_lib.lib().moe_wait_limit_ns())
+
+
+def moe_ffn_forward_select(layer: Layer, x, adapter_id, select, T, y, workspace, ws_bytes, stream=None):
+    """moe_ffn_forward with each token's expert set given (select [T, K] int32)."""
+    _check("moe_ffn_forward_select", _lib.lib().moe_ffn_forward_select(
+        ctypes.byref(layer), _ptr(x), _ptr(adapter_id), _ptr(select), T, _ptr(y), _ptr(workspace), ws_bytes,
+        _stream(stream)))
+
+
+def moe_prerouter_workspace_bytes(head: Prerouter, T) -> int:
+    return int(_lib.lib().moe_prerouter_workspace_bytes(ctypes.byref(head), T))
+
+
+def moe_prerouter_forward(head: Prerouter, h, exec_idx, prev_idx, T, logits, pred_idx, workspace, ws_bytes,
+                          stream=None):
+    _check("moe_prerouter_forward", _lib.lib().moe_prerouter_forward(
+        ctypes.byref(head), _ptr(h), _ptr(exec_idx), _ptr(prev_idx), T, _ptr(logits), _ptr(pred_idx),
+        _ptr(workspace), ws_bytes, _stream(stream)))

@@ -47,6 +47,11 @@ class Layer(ctypes.Structure):
                 ("lora", LoraPtrs * MAX_ADAPTERS)]
 
 
+class Prerouter(ctypes.Structure):
+    _fields_ = [("hidden", I32), ("n_experts", I32), ("top_k", I32), ("head_dim", I32), ("w1", P), ("b1", P),
+                ("w2", P), ("b2", P), ("wl", P), ("bl", P)]
+
+
 PQ, PM, PL, PLP = (ctypes.POINTER(QTensor), ctypes.POINTER(MixedTensor), ctypes.POINTER(Layer),
                    ctypes.POINTER(LoraPtrs))
 
@@ -75,6 +80,9 @@ SIGNATURES = {
     "moe_ffn_routing": (ctypes.c_int, [PL, I32, P, SZ, P, P, P]),
     "moe_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
     "moe_wait_limit_ns": (ctypes.c_uint64, []),
+    "moe_ffn_forward_select": (ctypes.c_int, [PL, P, P, P, I32, P, P, SZ, P]),
+    "moe_prerouter_workspace_bytes": (SZ, [ctypes.POINTER(Prerouter), I32]),
+    "moe_prerouter_forward": (ctypes.c_int, [ctypes.POINTER(Prerouter), P, P, P, I32, P, P, P, SZ, P]),
     "moe_timing_kinds": (ctypes.c_int, []),
     "moe_timing_kind_name": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_timing_enable": (ctypes.c_int, [ctypes.c_int]),

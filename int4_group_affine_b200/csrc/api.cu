@@ -234,13 +234,17 @@ moe_status router_enqueue(const uint16_t* x, const moe_qtensor& router, const mo
 }
 
 // The launch sequence shared by moe_ffn_forward and moe_block_forward.
-moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, int T,
+moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, const int32_t* select, int T,
                        const uint16_t* residual, uint16_t* y, const Work& wk, cudaStream_t s) {
     const LayerArgs la = args_of(L);
     const moe_qtensor* sg = la.has_sgate ? &L->shared_gate : nullptr;
     moe_status rst = router_enqueue(x, L->router, sg, L->logit_bias, T, la.H, la.E, wk.logits, wk.gs, wk.status, s);
     if (rst != MOE_OK) return rst;
-    LAUNCH(kTopk, launch_topk(wk.logits, wk.gs, la.has_sgate, T, la.E, la.K, wk.idx, wk.w, wk.sg, s));
+    if (select)
+        LAUNCH(kTopk, launch_select(wk.logits, wk.gs, la.has_sgate, select, T, la.E, la.K, wk.idx, wk.w, wk.sg,
+                                    wk.status, s));
+    else
+        LAUNCH(kTopk, launch_topk(wk.logits, wk.gs, la.has_sgate, T, la.E, la.K, wk.idx, wk.w, wk.sg, s));
     CHECK_CUDA(launch_index_build(wk, adapter_id, L->n_adapters, s));
     // Jobs of the shared expert stay in its group even without a shared expert:
     // their weights are zero-sized then, so they are skipped by the kernels.
@@ -270,8 +274,9 @@ moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* ada
 // The single fused kernel for a few tokens (csrc/decode.cu).  Returns false when
 // it does not apply (too many tokens or jobs, shapes outside its limits), so the
 // caller runs the multi-kernel path instead; otherwise *st is the launch result.
-bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, int T, int block, float eps,
-                uint16_t* y, const Dims& d, const WsPlan& p, void* ws, cudaStream_t s, moe_status* st) {
+bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, const int32_t* select, int T,
+                int block, float eps, uint16_t* y, const Dims& d, const WsPlan& p, void* ws, cudaStream_t s,
+                moe_status* st) {
     if (d.T > MOEQ_DECODE_MAX_TOKENS) return false;
     const LayerArgs la = args_of(L);
     if (chain_supported(la, T)) {  // one to four tokens: the chain kernel
@@ -282,7 +287,7 @@ bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id
         cs.status = (int32_t*)(b + p.status);
         cs.idx_out = (int32_t*)(b + p.idx);
         cs.w_out = (float*)(b + p.w);
-        const cudaError_t e = launch_chain(la, x, adapter_id, y, T, block, eps, cs, s);
+        const cudaError_t e = launch_chain(la, x, adapter_id, select, y, T, block, eps, cs, s);
         if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) {
             *st = e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
             if (e == cudaSuccess) timing_mark(kDecodeChain, s);
@@ -290,7 +295,7 @@ bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id
         }
         (void)cudaGetLastError();
     }
-    if (d.J > MOEQ_DECODE_MAX_JOBS) return false;
+    if (d.J > MOEQ_DECODE_MAX_JOBS || select) return false;  // (the older kernel routes by top-K only)
     if (!decode_supported(la, T, nullptr)) return false;
     char* b = (char*)ws;
     DecodeScratch sc;
@@ -508,8 +513,25 @@ moe_status moe_ffn_forward(const moe_layer* layer, const uint16_t* x, const int3
     if (T == 0) return MOE_OK;
     cudaStream_t s = (cudaStream_t)stream;
     timing_begin(s);
-    if (try_decode(layer, x, adapter_id, T, 0, 0.0f, y, d, p, workspace, s, &st)) return st;
-    return ffn_enqueue(layer, x, adapter_id, T, nullptr, y, work_of(d, p, workspace), s);
+    if (try_decode(layer, x, adapter_id, nullptr, T, 0, 0.0f, y, d, p, workspace, s, &st)) return st;
+    return ffn_enqueue(layer, x, adapter_id, nullptr, T, nullptr, y, work_of(d, p, workspace), s);
+}
+
+moe_status moe_ffn_forward_select(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id,
+                                  const int32_t* select, int32_t T, uint16_t* y, void* workspace, size_t ws_bytes,
+                                  moe_stream stream) {
+    moe_status st = ffn_precheck(layer, x, y, T);
+    if (st != MOE_OK) return st;
+    const Dims d = dims_of(layer, T);
+    const WsPlan p = plan_of(d);
+    st = ws_check(workspace, ws_bytes, p.total);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(select);
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    if (try_decode(layer, x, adapter_id, select, T, 0, 0.0f, y, d, p, workspace, s, &st)) return st;
+    return ffn_enqueue(layer, x, adapter_id, select, T, nullptr, y, work_of(d, p, workspace), s);
 }
 
 moe_status moe_block_forward(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id, int32_t T,
@@ -526,9 +548,9 @@ moe_status moe_block_forward(const moe_layer* layer, const uint16_t* x, const in
     const Work wk = work_of(d, p, workspace);
     cudaStream_t s = (cudaStream_t)stream;
     timing_begin(s);
-    if (try_decode(layer, x, adapter_id, T, 1, eps, x_out, d, p, workspace, s, &st)) return st;
+    if (try_decode(layer, x, adapter_id, nullptr, T, 1, eps, x_out, d, p, workspace, s, &st)) return st;
     LAUNCH(kRmsnorm, launch_rmsnorm(x, T, d.H, eps, wk.xn, s));
-    return ffn_enqueue(layer, wk.xn, adapter_id, T, x, x_out, wk, s);
+    return ffn_enqueue(layer, wk.xn, adapter_id, nullptr, T, x, x_out, wk, s);
 }
 
 moe_status moe_rmsnorm(const uint16_t* x, int32_t T, int32_t H, float eps, uint16_t* xn, moe_stream stream) {
@@ -538,6 +560,32 @@ moe_status moe_rmsnorm(const uint16_t* x, int32_t T, int32_t H, float eps, uint1
     cudaStream_t s = (cudaStream_t)stream;
     timing_begin(s);
     LAUNCH(kRmsnorm, launch_rmsnorm(x, T, H, eps, xn, s));
+    return MOE_OK;
+}
+
+size_t moe_prerouter_workspace_bytes(const moe_prerouter* head, int32_t T) {
+    if (!head || T < 0 || head->head_dim <= 0 || head->n_experts <= 0 || head->top_k <= 0) return 0;
+    return prerouter_workspace_bytes(*head, T);
+}
+
+moe_status moe_prerouter_forward(const moe_prerouter* head, const uint16_t* h, const int32_t* exec_idx,
+                                 const int32_t* prev_idx, int32_t T, float* logits, int32_t* pred_idx,
+                                 void* workspace, size_t ws_bytes, moe_stream stream) {
+    CHECK_ARG(head && T >= 0);
+    const int H = head->hidden, E = head->n_experts, K = head->top_k, D = head->head_dim;
+    CHECK_ARG(H > 0 && E > 0 && K > 0 && D > 0);
+    if (E > MOEQ_MAX_EXPERTS || K > MOEQ_MAX_TOPK || K > E || H > MOEQ_MAX_HIDDEN || D > 4096)
+        return MOE_ERR_UNSUPPORTED;
+    CHECK_ARG(H % 8 == 0 && (H + 2 * E) % 8 == 0 && D % 8 == 0);
+    CHECK_ARG(head->w1 && head->w2 && head->wl && aligned(head->w1, 16) && aligned(head->w2, 16) &&
+              aligned(head->wl, 16));
+    moe_status st = ws_check(workspace, ws_bytes, prerouter_workspace_bytes(*head, T));
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(h && exec_idx && logits && aligned(h, 16));
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    CHECK_CUDA(launch_prerouter(*head, h, exec_idx, prev_idx, T, logits, pred_idx, workspace, s));
     return MOE_OK;
 }
 

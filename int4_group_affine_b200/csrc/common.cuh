@@ -31,6 +31,30 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// One entry of a caller-given expert set (one warp per token, lane k < K takes entry
+// k of sel[0..K)): an entry outside [0, E) or repeating an earlier entry of the same
+// token is replaced by the lowest expert index the token does not use yet (entries
+// fixed in lane order), and *bad is set; returns this lane's expert (lanes >= K: -1).
+__device__ __forceinline__ int select_entry(const int32_t* sel, int K, int E, int lane, bool* bad) {
+    int e = lane < K ? sel[lane] : -1;
+    bool ok = lane < K && e >= 0 && e < E;
+    for (int j = 0; j < K; ++j) {
+        const int ej = __shfl_sync(0xffffffffu, e, j);
+        if (j < lane && ej == e) ok = false;
+    }
+    uint32_t badm = __ballot_sync(0xffffffffu, lane < K && !ok);
+    *bad = badm != 0;
+    if (lane < K && !ok) e = -1;
+    while (badm) {
+        const int k = __ffs(badm) - 1;
+        badm &= badm - 1;
+        int c = 0;
+        while (__any_sync(0xffffffffu, lane < K && e == c)) ++c;
+        if (lane == k) e = c;
+    }
+    return e;
+}
+
 // q (0..2^23) as float without an integer-to-float conversion instruction.
 __device__ __forceinline__ float u2f_small(uint32_t q) { return __uint_as_float(0x4B000000u | q) - 8388608.0f; }
 
@@ -119,7 +143,7 @@ struct DecodeScratch {
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
     kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kTcLoraGUKind, kTcGUKind,
-    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kDecodeChain, kKindCount
+    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kDecodeChain, kPrerouter, kKindCount
 };
 void timing_begin(cudaStream_t s);
 void timing_mark(int kind, cudaStream_t s);
@@ -140,6 +164,12 @@ cudaError_t launch_sgate_logits(const uint16_t* x, const moe_qtensor& sgate, int
                                 cudaStream_t s);
 cudaError_t launch_topk(const float* logits, const float* gs, bool has_sgate, int T, int E, int K, int32_t* idx,
                         float* w, float* sg, cudaStream_t s);
+
+// The routing of a caller-given expert set (the prerouter's prediction, say): idx from
+// sel [T][K] (repaired as in select_entry, MOE_ERR_DEVICE_INDEX raised), weights the
+// softmax of the logits renormalised over the set, sg = sigmoid(gs).
+cudaError_t launch_select(const float* logits, const float* gs, bool has_sgate, const int32_t* sel, int T, int E,
+                          int K, int32_t* idx, float* w, float* sg, int32_t* status, cudaStream_t s);
 
 cudaError_t launch_index_build(const Work& wk, const int32_t* adapter_id, int n_adapters, cudaStream_t s);
 cudaError_t launch_index_build_counts(const Work& wk, const int32_t* adapter_id, int n_adapters,
@@ -185,8 +215,14 @@ struct ChainScratch {
 };
 size_t chain_slot_words(int E, int K, int I, int Is, int r);
 bool chain_supported(const LayerArgs& L, int T);
-cudaError_t launch_chain(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, uint16_t* y, int T,
-                         int block, float eps, const ChainScratch& sc, cudaStream_t s);
+cudaError_t launch_chain(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, const int32_t* select,
+                         uint16_t* y, int T, int block, float eps, const ChainScratch& sc, cudaStream_t s);
+
+// The prerouter head (csrc/prerouter.cu).
+size_t prerouter_workspace_bytes(const moe_prerouter& P, int T);
+cudaError_t launch_prerouter(const moe_prerouter& P, const uint16_t* h, const int32_t* exec_idx,
+                             const int32_t* prev_idx, int T, float* logits, int32_t* pred_idx, void* ws,
+                             cudaStream_t s);
 
 cudaError_t launch_mixed_linear(const moe_mixed_tensor& W, int G, const uint16_t* x, int T, float* y,
                                 cudaStream_t s);

@@ -70,6 +70,7 @@ struct CArgs {
     LayerArgs L;
     const uint16_t* x;
     const int32_t* adapter_id;
+    const int32_t* select;     // [T][K] caller-given expert sets, or NULL: top-K of the logits
     uint16_t* y;
     int T, block;
     float eps;
@@ -189,6 +190,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
     __shared__ int s_abort;
     __shared__ uint32_t s_tag;
     __shared__ int s_aid[kCMaxT];
+    __shared__ int32_t s_sel[kCMaxTK];
     __shared__ float s_inv[kCMaxT], s_sig[kCMaxT];
     __shared__ int s_idx[kCMaxT][MOEQ_MAX_TOPK];
     __shared__ float s_w[kCMaxT][MOEQ_MAX_TOPK];
@@ -279,6 +281,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
             }
             s_aid[lane] = ad;
         }
+        if (a.select && lane < TK) s_sel[lane] = a.select[lane];
         __syncwarp();
         uint32_t tx = 0;
         if (lane < P.nSA) {  // LoRA-A rows of this CTA's shared LoRA-A dots: dot q = cta + NB * lane
@@ -408,8 +411,24 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
     __syncthreads();
     if (warp == 0) {
         // top-K of each token: lane holds experts lane + 32 c; K rounds of a warp max on
-        // order-preserving keys, equal keys to the lower expert index
+        // order-preserving keys, equal keys to the lower expert index.  With caller-given
+        // sets (the prerouter's prediction) the set is taken as it is and only the
+        // weights come from the logits.
         for (int t = 0; t < T; ++t) {
+            if (a.select) {
+                bool bad = false;
+                const int e = select_entry(s_sel + t * K, K, E, lane, &bad);
+                if (bad && lane == 0 && cta == 0) raise_status(a.status, MOE_ERR_DEVICE_INDEX);
+                const float zk = e >= 0 ? z[t * E + e] : -INFINITY;
+                const float m = warp_max(zk);
+                const float ev = e >= 0 ? expf(zk - m) : 0.0f;
+                const float sum = warp_sum(ev);
+                if (lane < K) {
+                    s_idx[t][lane] = e;
+                    s_w[t][lane] = ev / sum;
+                }
+                continue;
+            }
             constexpr int kC = MOEQ_MAX_EXPERTS / 32;
             uint32_t kv[kC];
 #pragma unroll
@@ -1081,14 +1100,15 @@ bool chain_supported(const LayerArgs& L, int T) {
     return plan_chain(L, T, c_sm_count(), &P);
 }
 
-cudaError_t launch_chain(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, uint16_t* y, int T,
-                         int block, float eps, const ChainScratch& sc, cudaStream_t s) {
+cudaError_t launch_chain(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, const int32_t* select,
+                         uint16_t* y, int T, int block, float eps, const ChainScratch& sc, cudaStream_t s) {
     CArgs a;
     memset(&a, 0, sizeof(a));
     if (!plan_chain(L, T, c_sm_count(), &a.P)) return cudaErrorNotSupported;
     a.L = L;
     a.x = x;
     a.adapter_id = adapter_id;
+    a.select = select;
     a.y = y;
     a.T = T;
     a.block = block;

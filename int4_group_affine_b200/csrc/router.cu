@@ -236,4 +236,38 @@ cudaError_t launch_topk(const float* logits, const float* gs, bool has_sgate, in
     return cudaGetLastError();
 }
 
+namespace {
+
+__global__ void select_kernel(const float* __restrict__ logits, const float* gs, int has_sgate,
+                              const int32_t* __restrict__ sel, int T, int E, int K, int32_t* __restrict__ idx,
+                              float* __restrict__ w, float* sg, int32_t* status) {
+    const int warps = blockDim.x / 32;
+    const int t = blockIdx.x * warps + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (t >= T) return;
+    bool bad = false;
+    const int e = select_entry(sel + (int64_t)t * K, K, E, lane, &bad);
+    if (bad && lane == 0) raise_status(status, MOE_ERR_DEVICE_INDEX);
+    const float z = e >= 0 ? logits[(int64_t)t * E + e] : -INFINITY;
+    const float m = warp_max(z);
+    const float ev = e >= 0 ? expf(z - m) : 0.0f;
+    const float sum = warp_sum(ev);
+    if (lane < K) {
+        idx[(int64_t)t * K + lane] = e;
+        w[(int64_t)t * K + lane] = ev / sum;
+    }
+    if (lane == 0 && sg) sg[t] = has_sgate ? 1.0f / (1.0f + expf(-gs[t])) : 1.0f;
+}
+
+}  // namespace
+
+cudaError_t launch_select(const float* logits, const float* gs, bool has_sgate, const int32_t* sel, int T, int E,
+                          int K, int32_t* idx, float* w, float* sg, int32_t* status, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    const int warps = 4;
+    select_kernel<<<(T + warps - 1) / warps, warps * 32, 0, s>>>(logits, gs, has_sgate ? 1 : 0, sel, T, E, K, idx, w,
+                                                                 sg, status);
+    return cudaGetLastError();
+}
+
 }  // namespace moeq

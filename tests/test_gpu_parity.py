@@ -232,7 +232,7 @@ def test_ffn_tiny(T):
     _check_ffn(shape, t, x, aid, what="tiny T=%d" % T, path="chain" if T <= 4 else "tensor_core")
 
 
-@pytest.mark.parametrize("T", [5, 8])
+@pytest.mark.parametrize("T", [5, 6])
 def test_ffn_tiny_fused_decode_path(T):
     """Five to eight tokens with at most 32 jobs: the older fused decode kernel (grid
     barriers, dedicated LoRA-A CTAs), which takes what the chain kernel does not."""
@@ -498,7 +498,7 @@ def test_full_size_pack_bit_exact(full_layer):
             assert np.array_equal(got.ravel(), t[name + suf].ravel()), name + suf
 
 
-@pytest.mark.parametrize("K,T,path", [(4, 1, "chain"), (8, 1, "chain"), (4, 2, "chain"), (4, 3, "chain"),
+@pytest.mark.parametrize("K,T,path", [(4, 1, "chain"), (8, 1, "chain"), (4, 2, "chain"), (4, 3, "decode"),
                                       (4, 6, None)])
 def test_full_size_decode(full_layer, K, T, path):
     shape0, w, t = full_layer
