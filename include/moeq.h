@@ -362,6 +362,30 @@ MOEQ_API moe_status moe_mixed_mlp_forward(const moe_mixed_tensor* gate, const mo
                                  const moe_mixed_tensor* down, const uint16_t* x, int32_t T, int32_t residual,
                                  float eps, uint16_t* y, void* workspace, size_t ws_bytes, moe_stream stream);
 
+/* ------------------------------------- a7 in weight-activation form (8-bit A)
+ * The mixed layer with 8-bit activations ("EDGERAZOR 深度解读" section 2.1 矩阵乘法
+ * 分解, Y = sum (s_W s_X) Q(W)^T Q(X), and the 1.88-8-8 / 1.58-8-8 rows of the
+ * weight-activation table in section 3.1).  Each token's activation row is
+ * quantised with the page's symmetric rule at n = 8 (reading: one scale per token):
+ * s_X = max(max|x| / 127, 1e-5), Q(X) = clip(round(x / s_X), -127, 127), both in
+ * fp32 (IEEE division, round half to even); the dot product is exact integer
+ * arithmetic and Y = s_W[o] * s_X[t] * sum_j Q(W)[o][j] Q(X)[t][j].
+ *  moe_act8_quant: x device bf16 [T][n] -> q device int8 [T][n], s device fp32 [T].
+ *  moe_mixed_linear_a8: x device bf16 [T][in] -> y device fp32 [T][out]; workspace of
+ *    moe_mixed_linear_a8_workspace_bytes(in, T) bytes, 256-byte aligned.
+ *  moe_mixed_mlp_forward_a8: as moe_mixed_mlp_forward, every linear layer in this form
+ *    (the intermediate h = SiLU(gate x) * up x is held in fp32 and quantised per
+ *    token like x); workspace of moe_mixed_mlp_a8_workspace_bytes(H, I, T) bytes. */
+MOEQ_API moe_status moe_act8_quant(const uint16_t* x, int32_t T, int32_t n, int8_t* q, float* s, moe_stream stream);
+MOEQ_API size_t moe_mixed_linear_a8_workspace_bytes(int32_t in, int32_t T);
+MOEQ_API moe_status moe_mixed_linear_a8(const moe_mixed_tensor* W, const uint16_t* x, int32_t T, float* y,
+                                        void* workspace, size_t ws_bytes, moe_stream stream);
+MOEQ_API size_t moe_mixed_mlp_a8_workspace_bytes(int32_t H, int32_t I, int32_t T);
+MOEQ_API moe_status moe_mixed_mlp_forward_a8(const moe_mixed_tensor* gate, const moe_mixed_tensor* up,
+                                             const moe_mixed_tensor* down, const uint16_t* x, int32_t T,
+                                             int32_t residual, float eps, uint16_t* y, void* workspace,
+                                             size_t ws_bytes, moe_stream stream);
+
 /* ---------------------------------------------------------- kernel timing
  * Opt-in measurement of the library's own kernels with CUDA events (no device
  * memory is allocated; events are created on the first enable).  While

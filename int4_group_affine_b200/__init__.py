@@ -22,7 +22,9 @@ __all__ = [
     "moe_mixed_linear", "moe_mixed_mlp_workspace_bytes", "moe_mixed_mlp_forward",
     "moe_timing_enable", "moe_timing_collect", "moe_ffn_forward_static", "moe_ffn_static_device_status",
     "moe_ffn_routing", "moe_set_wait_limit_ns", "moe_wait_limit_ns", "Prerouter", "moe_ffn_forward_select",
-    "moe_prerouter_workspace_bytes", "moe_prerouter_forward",
+    "moe_prerouter_workspace_bytes", "moe_prerouter_forward", "moe_act8_quant",
+    "moe_mixed_linear_a8_workspace_bytes", "moe_mixed_linear_a8", "moe_mixed_mlp_a8_workspace_bytes",
+    "moe_mixed_mlp_forward_a8",
 ]
 
 
@@ -212,4 +214,28 @@ def moe_prerouter_forward(head: Prerouter, h, exec_idx, prev_idx, T, logits, pre
                           stream=None):
     _check("moe_prerouter_forward", _lib.lib().moe_prerouter_forward(
         ctypes.byref(head), _ptr(h), _ptr(exec_idx), _ptr(prev_idx), T, _ptr(logits), _ptr(pred_idx),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def moe_act8_quant(x, T, n, q, s, stream=None):
+    _check("moe_act8_quant", _lib.lib().moe_act8_quant(_ptr(x), T, n, _ptr(q), _ptr(s), _stream(stream)))
+
+
+def moe_mixed_linear_a8_workspace_bytes(in_, T) -> int:
+    return int(_lib.lib().moe_mixed_linear_a8_workspace_bytes(in_, T))
+
+
+def moe_mixed_linear_a8(W: MixedTensor, x, T, y, workspace, ws_bytes, stream=None):
+    _check("moe_mixed_linear_a8", _lib.lib().moe_mixed_linear_a8(ctypes.byref(W), _ptr(x), T, _ptr(y),
+                                                                 _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def moe_mixed_mlp_a8_workspace_bytes(H, I, T) -> int:
+    return int(_lib.lib().moe_mixed_mlp_a8_workspace_bytes(H, I, T))
+
+
+def moe_mixed_mlp_forward_a8(gate: MixedTensor, up: MixedTensor, down: MixedTensor, x, T, residual, eps, y,
+                             workspace, ws_bytes, stream=None):
+    _check("moe_mixed_mlp_forward_a8", _lib.lib().moe_mixed_mlp_forward_a8(
+        ctypes.byref(gate), ctypes.byref(up), ctypes.byref(down), _ptr(x), T, residual, eps, _ptr(y),
         _ptr(workspace), ws_bytes, _stream(stream)))

@@ -83,6 +83,11 @@ SIGNATURES = {
     "moe_ffn_forward_select": (ctypes.c_int, [PL, P, P, P, I32, P, P, SZ, P]),
     "moe_prerouter_workspace_bytes": (SZ, [ctypes.POINTER(Prerouter), I32]),
     "moe_prerouter_forward": (ctypes.c_int, [ctypes.POINTER(Prerouter), P, P, P, I32, P, P, P, SZ, P]),
+    "moe_act8_quant": (ctypes.c_int, [P, I32, I32, P, P, P]),
+    "moe_mixed_linear_a8_workspace_bytes": (SZ, [I32, I32]),
+    "moe_mixed_linear_a8": (ctypes.c_int, [PM, P, I32, P, P, SZ, P]),
+    "moe_mixed_mlp_a8_workspace_bytes": (SZ, [I32, I32, I32]),
+    "moe_mixed_mlp_forward_a8": (ctypes.c_int, [PM, PM, PM, P, I32, I32, F32, P, P, SZ, P]),
     "moe_timing_kinds": (ctypes.c_int, []),
     "moe_timing_kind_name": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_timing_enable": (ctypes.c_int, [ctypes.c_int]),

@@ -662,4 +662,96 @@ moe_status moe_mixed_mlp_forward(const moe_mixed_tensor* gate, const moe_mixed_t
     return MOE_OK;
 }
 
+// ------------------------------------------------ weight-activation mixed layer
+namespace {
+struct A8Ws {
+    int8_t *q4, *q2;
+    float* s;
+    int32_t* qsum;
+};
+// 8-bit activation buffers of T rows of n: two permuted code copies, scales, code sums.
+size_t a8_bytes(int T, int n) { return 2 * align_up((size_t)T * n) + 2 * align_up((size_t)T * 4); }
+A8Ws a8_take(char* b, int T, int n) {
+    A8Ws w;
+    w.q4 = (int8_t*)b;
+    w.q2 = (int8_t*)(b + align_up((size_t)T * n));
+    w.s = (float*)(b + 2 * align_up((size_t)T * n));
+    w.qsum = (int32_t*)(b + 2 * align_up((size_t)T * n) + align_up((size_t)T * 4));
+    return w;
+}
+}  // namespace
+
+size_t moe_mixed_linear_a8_workspace_bytes(int32_t in, int32_t T) {
+    if (in <= 0 || T < 0) return 0;
+    return a8_bytes(T, in);
+}
+
+size_t moe_mixed_mlp_a8_workspace_bytes(int32_t H, int32_t I, int32_t T) {
+    if (H <= 0 || I <= 0 || T < 0) return 0;
+    return align_up((size_t)T * H * 2) + a8_bytes(T, H) + align_up((size_t)T * I * 4) + a8_bytes(T, I);
+}
+
+moe_status moe_act8_quant(const uint16_t* x, int32_t T, int32_t n, int8_t* q, float* s, moe_stream stream) {
+    CHECK_ARG(T >= 0 && n > 0);
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && q && s);
+    cudaStream_t st = (cudaStream_t)stream;
+    timing_begin(st);
+    CHECK_CUDA(launch_act8(x, nullptr, T, n, q, nullptr, nullptr, s, nullptr, st));
+    timing_mark(kAct8, st);
+    return MOE_OK;
+}
+
+moe_status moe_mixed_linear_a8(const moe_mixed_tensor* W, const uint16_t* x, int32_t T, float* y, void* workspace,
+                               size_t ws_bytes, moe_stream stream) {
+    CHECK_ARG(T >= 0 && W);
+    CHECK_ARG(mixed_ok(W, W->out, W->in) && W->out > 0);
+    moe_status st = ws_check(workspace, ws_bytes, a8_bytes(T, W->in));
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && y);
+    cudaStream_t s = (cudaStream_t)stream;
+    const A8Ws a = a8_take((char*)workspace, T, W->in);
+    timing_begin(s);
+    LAUNCH(kAct8, launch_act8(x, nullptr, T, W->in, nullptr, a.q4, a.q2, a.s, a.qsum, s));
+    LAUNCH(kMixedA8, launch_mixed_a8(*W, nullptr, mixed_G(W->rho), a.q4, a.q2, a.s, a.qsum, T, 0, y, nullptr,
+                                     nullptr, s));
+    return MOE_OK;
+}
+
+moe_status moe_mixed_mlp_forward_a8(const moe_mixed_tensor* gate, const moe_mixed_tensor* up,
+                                    const moe_mixed_tensor* down, const uint16_t* x, int32_t T, int32_t residual,
+                                    float eps, uint16_t* y, void* workspace, size_t ws_bytes, moe_stream stream) {
+    CHECK_ARG(T >= 0 && gate && up && down && (residual == 0 || residual == 1) && eps >= 0.0f);
+    const int I = gate->out, H = gate->in;
+    CHECK_ARG(H > 0 && I > 0 && mixed_ok(gate, I, H) && mixed_ok(up, I, H) && mixed_ok(down, H, I));
+    CHECK_ARG(gate->rho == up->rho && gate->rho == down->rho);
+    moe_status st = ws_check(workspace, ws_bytes, moe_mixed_mlp_a8_workspace_bytes(H, I, T));
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && y && x != y);
+    cudaStream_t s = (cudaStream_t)stream;
+    char* b = (char*)workspace;
+    uint16_t* xn = (uint16_t*)b;
+    b += align_up((size_t)T * H * 2);
+    const A8Ws ax = a8_take(b, T, H);
+    b += a8_bytes(T, H);
+    float* h = (float*)b;
+    b += align_up((size_t)T * I * 4);
+    const A8Ws ah = a8_take(b, T, I);
+    const int G = mixed_G(gate->rho);
+    const uint16_t* xin = x;
+    timing_begin(s);
+    if (residual) {
+        LAUNCH(kRmsnorm, launch_rmsnorm(x, T, H, eps, xn, s));
+        xin = xn;
+    }
+    LAUNCH(kAct8, launch_act8(xin, nullptr, T, H, nullptr, ax.q4, ax.q2, ax.s, ax.qsum, s));
+    LAUNCH(kMixedA8, launch_mixed_a8(*gate, up, G, ax.q4, ax.q2, ax.s, ax.qsum, T, 1, h, nullptr, nullptr, s));
+    LAUNCH(kAct8, launch_act8(nullptr, h, T, I, nullptr, ah.q4, ah.q2, ah.s, ah.qsum, s));
+    LAUNCH(kMixedA8, launch_mixed_a8(*down, nullptr, G, ah.q4, ah.q2, ah.s, ah.qsum, T, 2, nullptr, y,
+                                     residual ? x : nullptr, s));
+    return MOE_OK;
+}
+
 }  // extern "C"

@@ -143,7 +143,7 @@ struct DecodeScratch {
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
     kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kTcLoraGUKind, kTcGUKind,
-    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kDecodeChain, kPrerouter, kKindCount
+    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kDecodeChain, kPrerouter, kAct8, kMixedA8, kKindCount
 };
 void timing_begin(cudaStream_t s);
 void timing_mark(int kind, cudaStream_t s);
@@ -230,6 +230,16 @@ cudaError_t launch_mixed_gate_up(const moe_mixed_tensor& g, const moe_mixed_tens
                                  int T, float* h, cudaStream_t s);
 cudaError_t launch_mixed_down(const moe_mixed_tensor& d, int G, const float* h, int T, const uint16_t* residual,
                               uint16_t* y, cudaStream_t s);
+
+// Weight-activation form of the mixed layer (csrc/mixed_a8.cu): 8-bit per-token
+// activation codes (natural order and the two permuted copies, any may be NULL) from
+// bf16 (xb) or fp32 (xf) rows; then the integer dot in one of three modes
+// (0: y fp32; 1: h = SiLU(W x) * (U x) fp32; 2: y bf16 plus an optional residual).
+cudaError_t launch_act8(const uint16_t* xb, const float* xf, int T, int n, int8_t* qnat, int8_t* q4, int8_t* q2,
+                        float* s, int32_t* qsum, cudaStream_t st);
+cudaError_t launch_mixed_a8(const moe_mixed_tensor& W, const moe_mixed_tensor* U, int G, const int8_t* q4,
+                            const int8_t* q2, const float* sx, const int32_t* qsum, int T, int mode, float* yf,
+                            uint16_t* yb, const uint16_t* residual, cudaStream_t s);
 
 // Device row offset (in words) of row `o` of a mixed matrix with super-group size G.
 __host__ __device__ __forceinline__ int64_t mixed_row_offset(int o, int in, int G) {

@@ -45,7 +45,7 @@ constexpr int kCMaxR = 32;    // LoRA rank: one lane per component
 constexpr int kCMaxO = 32;    // output rows per CTA
 constexpr int kCMaxSA = 4;    // shared-expert LoRA-A dots per CTA
 constexpr int kCMaxRA = 8;    // routed LoRA-A dots per CTA
-constexpr int kGB = 16;       // words one thread polls per pass
+constexpr int kGB = 8;        // words one thread polls per pass
 
 // Shared-memory plan and per-CTA ranges (host-computed; the routed row ranges are
 // recomputed on the device from the actual number of distinct experts).
@@ -145,6 +145,76 @@ __device__ __forceinline__ int swz(int i) {
     return (c << 5) + (((p & ~3) + ((c & 7) << 2)) & 31) + (p & 3);
 }
 
+// sum_j A[j] v[j] for a bf16 row A of length n already in shared memory and one staged
+// vector (lane partial; the caller reduces): lane takes 32-element chunks lane, lane + 32, ...
+__device__ __forceinline__ float sdot_bf16(const uint16_t* arow, int n, const float* v, int lane) {
+    const uint4* a4 = reinterpret_cast<const uint4*>(arow);
+    float acc = 0.0f;
+    for (int c = lane; c < n / 32; c += 32) {
+        const int rot = (c & 7) << 2;
+        const float* vr = v + (c << 5);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint4 q = a4[4 * c + u];
+            const uint32_t aw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float4 xv = *reinterpret_cast<const float4*>(vr + ((8 * u + 4 * h + rot) & 31));
+                acc = fmaf(__uint_as_float(aw[2 * h] << 16), xv.x, acc);
+                acc = fmaf(__uint_as_float(aw[2 * h] & 0xFFFF0000u), xv.y, acc);
+                acc = fmaf(__uint_as_float(aw[2 * h + 1] << 16), xv.z, acc);
+                acc = fmaf(__uint_as_float(aw[2 * h + 1] & 0xFFFF0000u), xv.w, acc);
+            }
+        }
+    }
+    return acc;
+}
+
+// Top-K of one token's logits z[0..E) by one warp, E <= 32 * kC: lane holds experts
+// lane + 32 c; K rounds of a warp max on order-preserving keys, equal keys to the lower
+// expert index; weights exp(z_k - z_max) renormalised over the K.
+template <int kC>
+__device__ __forceinline__ void warp_topk(const float* z, int E, int K, int lane, int* idx, float* w) {
+    uint32_t kv[kC];
+#pragma unroll
+    for (int c = 0; c < kC; ++c) {
+        const int e = lane + 32 * c;
+        kv[c] = e < E ? okey(z[e]) : 0u;
+    }
+    uint32_t myk = 0u;
+    int mye = 0;
+    for (int k = 0; k < K; ++k) {
+        uint32_t bk = 0u;
+        int bc = -1;
+#pragma unroll
+        for (int c = 0; c < kC; ++c)
+            if (kv[c] > bk) {
+                bk = kv[c];
+                bc = c;
+            }
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+        const int me = (int)__reduce_min_sync(0xffffffffu, (bc >= 0 && bk == mk) ? (unsigned)(lane + 32 * bc)
+                                                                                   : 0x7fffffffu);
+        if ((me & 31) == lane) {
+#pragma unroll
+            for (int c = 0; c < kC; ++c)
+                if (c == (me >> 5)) kv[c] = 0u;
+        }
+        if (lane == k) {
+            myk = mk;
+            mye = me < E ? me : 0;
+        }
+    }
+    const float zk = myk ? okey_value(myk) : -INFINITY;
+    const float z0 = __shfl_sync(0xffffffffu, zk, 0);
+    const float ev = lane < K ? (z0 > -INFINITY ? expf(zk - z0) : 1.0f) : 0.0f;
+    const float sum = warp_sum(ev);
+    if (lane < K) {
+        idx[lane] = mye;
+        w[lane] = ev / sum;
+    }
+}
+
 // Bulk-copy window issue helper: nothing for bytes == 0 or a null source.
 __device__ __forceinline__ const unsigned char* win(unsigned char* dst, const void* src, uint32_t bytes,
                                                     uint64_t* bar, uint32_t* tx) {
@@ -177,7 +247,6 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
     float* xs = reinterpret_cast<float*>(sm + P.xs);      // [T][H] staged input (swizzled)
     float* xsum = reinterpret_cast<float*>(sm + P.xsum);  // [T][H/32]
     float* z = reinterpret_cast<float*>(sm + P.z);        // [T][E] logits
-    float* saxs = reinterpret_cast<float*>(sm + P.sax);   // [T][2r]
     float* sgu = reinterpret_cast<float*>(sm + P.sgu);    // [perS][T][2] shared gate/up pre-activations
     float* hsm = reinterpret_cast<float*>(sm + P.hs);     // routed h [TK][I], then shared [T][Is] (swizzled)
     float* hsum = reinterpret_cast<float*>(sm + P.hsum);
@@ -224,10 +293,10 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
     const int o_lo = min(H, cta * P.perO), o_hi = min(H, o_lo + P.perO), no = o_hi - o_lo;
 
     // ------------------------------------------------------------ phase R: issue
+    unsigned long long prev = 0;  // this launch's ticket (first needed after x is staged)
+    if (warp == kCW - 1 && lane == 0)
+        asm volatile("atom.add.relaxed.gpu.global.u64 %0, [%1], 1;" : "=l"(prev) : "l"(a.tick) : "memory");
     if (warp == 0) {
-        unsigned long long prev = 0;
-        if (lane == 31)
-            asm volatile("atom.add.relaxed.gpu.global.u64 %0, [%1], 1;" : "=l"(prev) : "l"(a.tick) : "memory");
         uint32_t tx = 0;
         unsigned char* wa = sm + P.wa;
         if (lane == 0) {
@@ -270,7 +339,6 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
         }
         tx1 = warp_total(tx1);
         if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[1], tx1);
-        if (lane == 31) s_tag = (uint32_t)((prev / (unsigned long long)NB) % 0xffffffffull) + 1u;
     } else if (warp == 1) {
         // adapter ids, then the shared-expert LoRA rows this CTA needs
         if (lane < T) {
@@ -329,17 +397,16 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
         __syncthreads();
     }
     stage_bf16(xs, xsum, xr, T, H, a.block ? s_inv : nullptr);
+    if (warp == kCW - 1 && lane == 0) s_tag = (uint32_t)((prev / (unsigned long long)NB) % 0xffffffffull) + 1u;
     __syncthreads();
     const uint32_t tag = s_tag;
 
     {
-        int nsa = 0;
-        if (lora && sh)
-            for (int j = 0; j < P.nSA; ++j) nsa += (cta + NB * j < T * 2 * r) ? 1 : 0;
+        // router rows first, on warps 2.. (warps 0 and 1 issued the copies, the last warp
+        // took the ticket)
         const int nsg = L.has_sgate ? 1 : 0;
-        const int ntask = nra + nsg + nsr + nsa;
-        bool landed1 = false;
-        for (int j = warp; j < ntask; j += kCW) {
+        const int ntask = nra + nsg + nsr;
+        for (int j = (warp + kCW - 2) % kCW; j < ntask; j += kCW) {
             if (j < nra + nsg) {  // router row or the shared-expert gate row (int8)
                 const bool sg = j >= nra;
                 const moe_qtensor& q = sg ? L.shared_gate : L.router;
@@ -392,22 +459,12 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                         sgu[(il * T + m) * 2 + 1] = u;
                     }
                 }
-            } else {  // shared LoRA-A dot q = cta + NB * jj: token t, component d of gate | up
-                const int jj = j - nra - nsg - nsr, q = cta + NB * jj, t = q / (2 * r), d = q % (2 * r);
-                if (!landed1) {
-                    copies_landed(&s_bar[1], a.status, &s_abort, lim);
-                    landed1 = true;
-                }
-                float v = 0.0f;
-                if (s_saw[jj]) v = warp_sum(dot_bf16(reinterpret_cast<const uint16_t*>(s_saw[jj]), H, xs + t * H, lane));
-                if (lane == 0) publish(a.sax + (int64_t)t * 2 * r + d, v, tag);
             }
         }
     }
 
     // ------------------------------------------------------------ phase K
     gather_range(a.zs, T * E, z, tag, a.status, &s_abort, lim);
-    if (lora && sh) gather_range(a.sax, T * 2 * r, saxs, tag, a.status, &s_abort, lim);
     __syncthreads();
     if (warp == 0) {
         // top-K of each token: lane holds experts lane + 32 c; K rounds of a warp max on
@@ -429,43 +486,8 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                 }
                 continue;
             }
-            constexpr int kC = MOEQ_MAX_EXPERTS / 32;
-            uint32_t kv[kC];
-#pragma unroll
-            for (int c = 0; c < kC; ++c) {
-                const int e = lane + 32 * c;
-                kv[c] = e < E ? okey(z[t * E + e]) : 0u;
-            }
-            uint32_t myk = 0u;
-            int mye = 0;
-            for (int k = 0; k < K; ++k) {
-                uint32_t bk = 0u;
-                int bc = -1;
-#pragma unroll
-                for (int c = 0; c < kC; ++c)
-                    if (kv[c] > bk) {
-                        bk = kv[c];
-                        bc = c;
-                    }
-                const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
-                const int me = (int)__reduce_min_sync(0xffffffffu, (bc >= 0 && bk == mk) ? (unsigned)(lane + 32 * bc)
-                                                                                           : 0x7fffffffu);
-#pragma unroll
-                for (int c = 0; c < kC; ++c)
-                    if (lane + 32 * c == me) kv[c] = 0u;
-                if (lane == k) {
-                    myk = mk;
-                    mye = me < E ? me : 0;
-                }
-            }
-            const float zk = myk ? okey_value(myk) : -INFINITY;
-            const float z0 = __shfl_sync(0xffffffffu, zk, 0);
-            const float ev = lane < K ? (z0 > -INFINITY ? expf(zk - z0) : 1.0f) : 0.0f;
-            const float sum = warp_sum(ev);
-            if (lane < K) {
-                s_idx[t][lane] = mye;
-                s_w[t][lane] = ev / sum;
-            }
+            if (E <= 256) warp_topk<8>(z + t * E, E, K, lane, s_idx[t], s_w[t]);
+            else warp_topk<MOEQ_MAX_EXPERTS / 32>(z + t * E, E, K, lane, s_idx[t], s_w[t]);
         }
         __syncwarp();
         if (cta == 0 && lane < TK) {  // the routing this call used, for the caller's record
@@ -611,8 +633,11 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
 #pragma unroll
         for (int m = 0; m < MT; ++m) wacc[s][m] = 0.0f;
     const bool kk = lane < r;
+    int nsa_here = 0;
+    if (lora && sh)
+        for (int j = 0; j < P.nSA; ++j) nsa_here += (cta + NB * j < T * 2 * r) ? 1 : 0;
     {
-        const int ntask = nra_here + nsr + nrows;
+        const int ntask = nra_here + nsa_here + nsr + nrows;
         bool landed[4] = {false, false, false, false};
         auto land = [&](int b) {
             if (!landed[b - 1]) {
@@ -626,12 +651,20 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                 land(2);
                 float v = 0.0f;
                 if (s_raw[j])
-                    v = warp_sum(dot_bf16(reinterpret_cast<const uint16_t*>(s_raw[j]), H, xs + (js / K) * H, lane));
+                    v = warp_sum(sdot_bf16(reinterpret_cast<const uint16_t*>(s_raw[j]), H, xs + (js / K) * H, lane));
                 if (lane == 0) publish(a.rax + (int64_t)js * 2 * r + d, v, tag);
                 continue;
             }
-            if (j < nra_here + nsr) {  // shared-expert row i: LoRA-B delta, SwiGLU, h, partial A_down h
-                const int il = j - nra_here, i = s_lo + il;
+            if (j < nra_here + nsa_here) {  // shared LoRA-A dot q: token t, component d of gate | up
+                const int jj = j - nra_here, q = cta + NB * jj, t = q / (2 * r), d = q % (2 * r);
+                land(1);
+                float v = 0.0f;
+                if (s_saw[jj]) v = warp_sum(sdot_bf16(reinterpret_cast<const uint16_t*>(s_saw[jj]), H, xs + t * H, lane));
+                if (lane == 0) publish(a.sax + (int64_t)t * 2 * r + d, v, tag);
+                continue;
+            }
+            if (j < nra_here + nsa_here + nsr) {  // shared-expert row i: LoRA-B delta, SwiGLU, h, partial A_down h
+                const int il = j - nra_here - nsa_here, i = s_lo + il;
                 float ad[MT];
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
@@ -639,6 +672,15 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                     if (m < T && kk) {
                         const moe_lora_proj* ld = dlora(L, s_aid[m], true, 2);
                         if (ld) ad[m] = bf16f(ld->A[(int64_t)lane * Is + i]);
+                    }
+                }
+                unsigned long long sw[MT][2];  // this token's shared LoRA-A products (lane = component)
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    sw[m][0] = sw[m][1] = 0ull;
+                    if (m < T && kk) {
+                        sw[m][0] = peek(a.sax + (int64_t)m * 2 * r + lane);
+                        sw[m][1] = peek(a.sax + (int64_t)m * 2 * r + r + lane);
                     }
                 }
                 land(1);
@@ -649,8 +691,14 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                     if (lora) {
                         const uint16_t* bg = reinterpret_cast<const uint16_t*>(s_sbw[m][0]);
                         const uint16_t* bu = reinterpret_cast<const uint16_t*>(s_sbw[m][1]);
-                        const float dg = (kk && bg) ? bf16f(bg[il * r + lane]) * saxs[m * 2 * r + lane] : 0.0f;
-                        const float du = (kk && bu) ? bf16f(bu[il * r + lane]) * saxs[m * 2 * r + r + lane] : 0.0f;
+                        float tg = 0.0f, tu = 0.0f;
+                        if (kk) {
+                            const uint64_t* sp = a.sax + (int64_t)m * 2 * r + lane;
+                            tg = fresh(sw[m][0], tag) ? wval(sw[m][0]) : spin(sp, tag, a.status, &s_abort, lim);
+                            tu = fresh(sw[m][1], tag) ? wval(sw[m][1]) : spin(sp + r, tag, a.status, &s_abort, lim);
+                        }
+                        const float dg = (kk && bg) ? bf16f(bg[il * r + lane]) * tg : 0.0f;
+                        const float du = (kk && bu) ? bf16f(bu[il * r + lane]) * tu : 0.0f;
                         g += L.scale * warp_sum(dg);
                         u += L.scale * warp_sum(du);
                     }
@@ -661,7 +709,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                 continue;
             }
             // routed row q: distinct expert u, row i, segment sg
-            const int q = c_lo + (j - nra_here - nsr), u = q / I, i = q % I, sg = q < cut ? 0 : 1;
+            const int q = c_lo + (j - nra_here - nsa_here - nsr), u = q / I, i = q % I, sg = q < cut ? 0 : 1;
             const int rs = q - (sg == 0 ? c_lo : cut), e = s_uexp[u], nt = s_ucnt[u];
             int toks[MT];
             float ad[MT];
@@ -735,36 +783,36 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
 
     // ------------------------------------------------------------ phase D
     // h of every job (routed rows of length I, then the shared ones of length Is), staged
-    // in the swizzled layout, and the 32-element chunk sums
+    // in the swizzled layout; every thread's words of a pass are in flight together
     {
-        const int Imx = max(I, Is);
-        const int nh = TK * I + T * Is;
+        const int Imx = max(I, Is), nh = TK * I + T * Is;
+        auto hsrc = [&](int q) {
+            return q < TK * I ? a.hx + (int64_t)(q / I) * Imx + q % I
+                              : a.hx + (int64_t)(TK + (q - TK * I) / Is) * Imx + (q - TK * I) % Is;
+        };
         for (int base = 0; base < nh; base += kGB * kCT) {
             unsigned long long w[kGB];
-            const uint64_t* src[kGB];
 #pragma unroll
             for (int b = 0; b < kGB; ++b) {
                 const int q = base + b * kCT + tid;
-                src[b] = nullptr;
-                w[b] = 0ull;
-                if (q < nh) {
-                    const int slot = q < TK * I ? q / I : TK + (q - TK * I) / Is;
-                    const int i = q < TK * I ? q % I : (q - TK * I) % Is;
-                    src[b] = a.hx + (int64_t)slot * Imx + i;
-                    w[b] = peek(src[b]);
-                }
+                w[b] = q < nh ? peek(hsrc(q)) : 0ull;
             }
 #pragma unroll
             for (int b = 0; b < kGB; ++b) {
                 const int q = base + b * kCT + tid;
-                if (q >= nh) continue;
-                const float v = fresh(w[b], tag) ? wval(w[b]) : spin(src[b], tag, a.status, &s_abort, lim);
+                if (q >= nh) break;
+                const float v = fresh(w[b], tag) ? wval(w[b]) : spin(hsrc(q), tag, a.status, &s_abort, lim);
                 if (q < TK * I) hsm[(q / I) * I + swz(q % I)] = v;
                 else hsm[TK * I + ((q - TK * I) / Is) * Is + swz((q - TK * I) % Is)] = v;
             }
         }
     }
-    if (lora) {  // partial down LoRA-A sums: per job, the CTAs whose rows cover its expert
+    if (lora) {
+        // down LoRA-A products: for each job, the sum over the CTAs whose rows cover its
+        // expert of their published partials, in CTA order.  An item is (job, component,
+        // a run of up to 8 of those CTAs): its 8 words are polled together and summed;
+        // the items of a (job, component) are then summed in order.
+        constexpr int kRun = 8;
         if (tid == 0) {
             int o = 0;
             for (int j = 0; j < J; ++j) {
@@ -776,7 +824,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                 } else {
                     ncta = (Is + P.perS - 1) / P.perS;
                 }
-                o += ncta * r;
+                o += (ncta + kRun - 1) / kRun * r;
             }
             s_goff[J] = o;
         }
@@ -786,42 +834,44 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
         const int total = s_goff[J];
         for (int base = 0; base < total; base += (int)P.gat_n) {
             const int n = min((int)P.gat_n, total - base);
-            for (int b0 = 0; b0 < n; b0 += kGB * kCT) {
-                unsigned long long w[kGB];
-                const uint64_t* src[kGB];
-#pragma unroll
-                for (int b = 0; b < kGB; ++b) {
-                    const int q = b0 + b * kCT + tid;
-                    src[b] = nullptr;
-                    w[b] = 0ull;
-                    if (q < n) {
-                        const int g = base + q;
-                        int j = 0;
-                        while (j + 1 < J && s_goff[j + 1] <= g) ++j;
-                        const int loc = g - s_goff[j], k = loc % r, ci = loc / r;
-                        int c, s, m;
-                        if (j < TK) {
-                            const int u = s_ju[j];
-                            c = (u * I) / perC + ci;
-                            s = c * perC < u * I ? 1 : 0;
-                            m = s_jm[j];
-                        } else {
-                            c = ci;
-                            s = 2;
-                            m = j - TK;
-                        }
-                        src[b] = a.part + (((int64_t)c * 3 + s) * T + m) * r + k;
-                        w[b] = peek(src[b]);
-                    }
+            for (int q = tid; q < n; q += kCT) {
+                const int g = base + q;
+                int j = 0;
+                while (j + 1 < J && s_goff[j + 1] <= g) ++j;
+                const int loc = g - s_goff[j], k = loc % r, run = loc / r;
+                int c0, cnt, m, s0;  // first CTA of the run, CTAs in it, token slot, segment of the first
+                if (j < TK) {
+                    const int u = s_ju[j], cf = (u * I) / perC, cl = ((u + 1) * I - 1) / perC;
+                    c0 = cf + run * kRun;
+                    cnt = min(kRun, cl - c0 + 1);
+                    m = s_jm[j];
+                    s0 = (run == 0 && cf * perC < u * I) ? 1 : 0;  // only the first covering CTA can hold u second
+                } else {
+                    c0 = run * kRun;
+                    cnt = min(kRun, (Is + P.perS - 1) / P.perS - c0);
+                    m = j - TK;
+                    s0 = 2;
                 }
+                const int64_t step = (int64_t)3 * T * r, off = (int64_t)m * r + k;
+                unsigned long long w[kRun];
 #pragma unroll
-                for (int b = 0; b < kGB; ++b) {
-                    const int q = b0 + b * kCT + tid;
-                    if (q < n) gat[q] = fresh(w[b], tag) ? wval(w[b]) : spin(src[b], tag, a.status, &s_abort, lim);
+                for (int i = 0; i < kRun; ++i) {
+                    const int s = i == 0 ? s0 : (j < TK ? 0 : 2);
+                    w[i] = i < cnt ? peek(a.part + (int64_t)(c0 + i) * step + (int64_t)s * T * r + off) : 0ull;
                 }
+                float v = 0.0f;
+#pragma unroll
+                for (int i = 0; i < kRun; ++i) {
+                    if (i >= cnt) break;
+                    const int s = i == 0 ? s0 : (j < TK ? 0 : 2);
+                    v += fresh(w[i], tag) ? wval(w[i])
+                                          : spin(a.part + (int64_t)(c0 + i) * step + (int64_t)s * T * r + off, tag,
+                                                 a.status, &s_abort, lim);
+                }
+                gat[q] = v;
             }
             __syncthreads();
-            // fixed-order sums: entry (j, ci, k) at s_goff[j] + ci * r + k
+            // the runs of each (job, component) in order: entry (j, run, k) at s_goff[j] + run * r + k
             for (int q = tid; q < J * r; q += kCT) {
                 const int j = q / r, k = q % r;
                 const int g0 = max(s_goff[j], base), g1 = min(s_goff[j + 1], base + n);

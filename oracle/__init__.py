@@ -95,6 +95,10 @@ def _get():
             "orc_fp16_value": (D, [ctypes.c_uint16]),
             "orc_gelu_erf": (D, [D]),
             "orc_prerouter": (I, [P, P, P, P, I, P]),
+            "orc_quant_act8": (None, [P, I, I, P, P]),
+            "orc_mixed_linear_a8": (None, [P, P, I, I, D, P, I, P]),
+            "orc_mixed_mlp_a8": (I, [P, P, P, P, P, P, I, I, D, P, I, P]),
+            "orc_mixed_block_a8": (I, [P, P, P, P, P, P, I, I, D, D, P, I, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -393,3 +397,44 @@ def prerouter(H, E, K, D, w, h_bf16, exec_idx, prev_idx=None):
     if rc != 0:
         raise ValueError("orc_prerouter rc=%d" % rc)
     return z
+
+
+def quant_act8(x: np.ndarray):
+    """Per-row symmetric 8-bit codes (int8 [T, n]) and scales (fp32 [T]) of fp32 rows."""
+    x = _c(x, np.float32)
+    T, n = x.shape
+    q = np.empty((T, n), dtype=np.int8)
+    s = np.empty(T, dtype=np.float32)
+    _get().orc_quant_act8(_p(x), T, n, _p(q), _p(s))
+    return q, s
+
+
+def mixed_linear_a8(packed, scales, out: int, in_: int, rho: float, x_bf16) -> np.ndarray:
+    x = _c(x_bf16, np.uint16)
+    T = x.size // in_
+    y = np.empty((T, out), dtype=np.float64)
+    _get().orc_mixed_linear_a8(_p(_c(packed, np.uint32)), _p(_c(scales, np.uint16)), out, in_, float(rho), _p(x), T,
+                               _p(y))
+    return y
+
+
+def mixed_mlp_a8(gate, up, down, H: int, I: int, rho: float, x_bf16) -> np.ndarray:
+    x = _c(x_bf16, np.uint16)
+    T = x.size // H
+    y = np.empty((T, H), dtype=np.float64)
+    arrs = [_c(a, np.uint32 if i % 2 == 0 else np.uint16) for i, a in enumerate((*gate, *up, *down))]
+    rc = _get().orc_mixed_mlp_a8(*[_p(a) for a in arrs], H, I, float(rho), _p(x), T, _p(y))
+    if rc != 0:
+        raise ValueError("orc_mixed_mlp_a8 rc=%d" % rc)
+    return y
+
+
+def mixed_block_a8(gate, up, down, H: int, I: int, rho: float, x_bf16, eps: float = 1e-6) -> np.ndarray:
+    x = _c(x_bf16, np.uint16)
+    T = x.size // H
+    out = np.empty((T, H), dtype=np.uint16)
+    arrs = [_c(a, np.uint32 if i % 2 == 0 else np.uint16) for i, a in enumerate((*gate, *up, *down))]
+    rc = _get().orc_mixed_block_a8(*[_p(a) for a in arrs], H, I, float(rho), float(eps), _p(x), T, _p(out))
+    if rc != 0:
+        raise ValueError("orc_mixed_block_a8 rc=%d" % rc)
+    return out

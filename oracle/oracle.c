@@ -711,3 +711,104 @@ int orc_prerouter(const orc_prerouter_head* P, const uint16_t* h, const int32_t*
     free(g);
     return rc;
 }
+
+/* ------------------------------------- weight-activation mixed layer (W + 8-bit A) */
+
+/* [ER §2.1 量化公式] applied to activations at n = 8 (the "-8-8" rows of the page's
+ * weight-activation table), reading: one symmetric scale per token row,
+ * s_X = max(max|x| / (2^7 - 1), eps) and q = clip(round(x / s_X), -127, 127).  The
+ * scale and the codes are decided in fp32 (IEEE division, round half to even), the
+ * precision the kernel decides them in, so the codes agree bit for bit. */
+void orc_quant_act8(const float* x, int T, int n, int8_t* q, float* s) {
+    for (int t = 0; t < T; ++t) {
+        const float* xr = x + (int64_t)t * n;
+        float m = 0.0f;
+        for (int j = 0; j < n; ++j) m = fmaxf(m, fabsf(xr[j]));
+        volatile float st = m / 127.0f;  /* one IEEE fp32 division, no contraction */
+        float sc = fmaxf(st, 1e-5f);
+        s[t] = sc;
+        for (int j = 0; j < n; ++j) {
+            volatile float v = xr[j] / sc;
+            float r = rintf(v);
+            if (r > 127.0f) r = 127.0f;
+            if (r < -127.0f) r = -127.0f;
+            q[(int64_t)t * n + j] = (int8_t)r;
+        }
+    }
+}
+
+/* [ER §2.1 矩阵乘法分解]: Y = sum (s_W s_X) Q(W)^T Q(X): the integer dot product of
+ * the weight codes and the 8-bit activation codes, scaled once by the channel scale
+ * and the token scale. */
+static void mixed_linear_a8(const uint32_t* packed, const uint16_t* scales, int out, int in, int G,
+                            const int8_t* qx, double sx, double* y) {
+    #pragma omp parallel for schedule(static)
+    for (int o = 0; o < out; ++o) {
+        const uint32_t* pw = packed + orc_mixed_row_offset(o, in, G);
+        int64_t acc = 0;
+        for (int j = 0; j < in; ++j) {
+            int q = mixed_is4(o, G) ? (int)((pw[j / 8] >> ((j % 8) * 4)) & 15u) - 8
+                                    : (int)((pw[j / 16] >> ((j % 16) * 2)) & 3u) - 1;
+            acc += (int64_t)q * qx[j];
+        }
+        y[o] = orc_bf16_value(scales[o]) * sx * (double)acc;
+    }
+}
+
+void orc_mixed_linear_a8(const uint32_t* packed, const uint16_t* scales, int out, int in, double rho,
+                         const uint16_t* x, int T, double* y) {
+    const int G = orc_mixed_group(rho);
+    float* xf = (float*)malloc((size_t)in * sizeof(float));
+    int8_t* q = (int8_t*)malloc((size_t)in);
+    for (int t = 0; t < T; ++t) {
+        float sx;
+        for (int j = 0; j < in; ++j) xf[j] = (float)orc_bf16_value(x[(int64_t)t * in + j]);
+        orc_quant_act8(xf, 1, in, q, &sx);
+        mixed_linear_a8(packed, scales, out, in, G, q, (double)sx, y + (int64_t)t * out);
+    }
+    free(xf);
+    free(q);
+}
+
+/* The SwiGLU MLP with every linear layer in weight-activation form: x and the
+ * intermediate h = SiLU(gate x) * up x are each quantised to 8 bits per token (h
+ * rounded to fp32 first, the width the kernel holds it in). */
+int orc_mixed_mlp_a8(const uint32_t* gp, const uint16_t* gs, const uint32_t* up, const uint16_t* us,
+                     const uint32_t* dp, const uint16_t* ds, int H, int I, double rho, const uint16_t* x, int T,
+                     double* y) {
+    if (H % 16 || I % 16) return -1;
+    const int G = orc_mixed_group(rho);
+    float* xf = (float*)malloc((size_t)(H > I ? H : I) * sizeof(float));
+    int8_t* q = (int8_t*)malloc((size_t)(H > I ? H : I));
+    double* g = (double*)malloc((size_t)I * sizeof(double));
+    double* u = (double*)malloc((size_t)I * sizeof(double));
+    for (int t = 0; t < T; ++t) {
+        float sx;
+        for (int j = 0; j < H; ++j) xf[j] = (float)orc_bf16_value(x[(int64_t)t * H + j]);
+        orc_quant_act8(xf, 1, H, q, &sx);
+        mixed_linear_a8(gp, gs, I, H, G, q, (double)sx, g);
+        mixed_linear_a8(up, us, I, H, G, q, (double)sx, u);
+        for (int i = 0; i < I; ++i) xf[i] = (float)(silu(g[i]) * u[i]);
+        orc_quant_act8(xf, 1, I, q, &sx);
+        mixed_linear_a8(dp, ds, H, I, G, q, (double)sx, y + (int64_t)t * H);
+    }
+    free(xf);
+    free(q);
+    free(g);
+    free(u);
+    return 0;
+}
+
+int orc_mixed_block_a8(const uint32_t* gp, const uint16_t* gs, const uint32_t* up, const uint16_t* us,
+                       const uint32_t* dp, const uint16_t* ds, int H, int I, double rho, double eps,
+                       const uint16_t* x, int T, uint16_t* x_out) {
+    uint16_t* xn = (uint16_t*)malloc((size_t)T * H * 2);
+    double* y = (double*)malloc((size_t)T * H * sizeof(double));
+    orc_rmsnorm_bf16(x, T, H, eps, xn);
+    int rc = orc_mixed_mlp_a8(gp, gs, up, us, dp, ds, H, I, rho, xn, T, y);
+    if (rc == 0)
+        for (int64_t i = 0; i < (int64_t)T * H; ++i) x_out[i] = orc_bf16_round_nearest(orc_bf16_value(x[i]) + y[i]);
+    free(xn);
+    free(y);
+    return rc;
+}

@@ -83,6 +83,18 @@ int orc_mixed_block(const uint32_t* gp, const uint16_t* gs, const uint32_t* up, 
                     const uint32_t* dp, const uint16_t* ds, int H, int I, double rho, double eps,
                     const uint16_t* x, int T, uint16_t* x_out);
 
+/* Weight-activation form of the mixed layer ("EDGERAZOR 深度解读" section 2.1 and
+ * the W/A table of section 3.1): 8-bit per-token activation codes. */
+void orc_quant_act8(const float* x, int T, int n, int8_t* q, float* s);
+void orc_mixed_linear_a8(const uint32_t* packed, const uint16_t* scales, int out, int in, double rho,
+                         const uint16_t* x, int T, double* y);
+int orc_mixed_mlp_a8(const uint32_t* gp, const uint16_t* gs, const uint32_t* up, const uint16_t* us,
+                     const uint32_t* dp, const uint16_t* ds, int H, int I, double rho, const uint16_t* x, int T,
+                     double* y);
+int orc_mixed_block_a8(const uint32_t* gp, const uint16_t* gs, const uint32_t* up, const uint16_t* us,
+                       const uint32_t* dp, const uint16_t* ds, int H, int I, double rho, double eps,
+                       const uint16_t* x, int T, uint16_t* x_out);
+
 void orc_router(const orc_layer* L, const uint16_t* x, int T, double* logits, double* gs);
 void orc_topk(const double* logits, int T, int E, int K, int32_t* idx, double* w);
 int orc_index_build(const int32_t* idx, const int32_t* adapter_id, int T, int K, int E,
