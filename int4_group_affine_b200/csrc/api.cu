@@ -282,7 +282,6 @@ bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id
     if (chain_supported(la, T)) {  // one to four tokens: the chain kernel
         char* b = (char*)ws;
         ChainScratch cs;
-        cs.tick = (unsigned long long*)(b + p.bar);
         cs.slots = (uint64_t*)(b + p.slots);
         cs.status = (int32_t*)(b + p.status);
         cs.idx_out = (int32_t*)(b + p.idx);

@@ -207,8 +207,7 @@ cudaError_t launch_decode(const LayerArgs& L, const uint16_t* x, const int32_t* 
 // hand-offs through epoch-tagged 64-bit words in a workspace region of
 // chain_slot_words(...) words that sits at a fixed place for a layer shape.
 struct ChainScratch {
-    unsigned long long* tick;  // ticket counter in the workspace header (starts zeroed)
-    uint64_t* slots;           // the tagged-word region (starts zeroed)
+    uint64_t* slots;           // the kernel's region: ticket, counters, tagged words (starts zeroed)
     int32_t* status;
     int32_t* idx_out;          // [T][K] routing record
     float* w_out;

@@ -74,12 +74,15 @@ struct CArgs {
     uint16_t* y;
     int T, block;
     float eps;
-    unsigned long long* tick;  // ticket counter (workspace header)
-    uint64_t* zs;              // [T][E] logits
-    uint64_t* sax;             // [T][2r] shared LoRA-A products (gate | up)
-    uint64_t* rax;             // [TK][2r] routed LoRA-A products, routed slot t*K+k
-    uint64_t* hx;              // [J][Imax] h: routed slot t*K+k, shared T*K+t
-    uint64_t* part;            // [NB][3][T][r] partial down LoRA-A sums: segment 0, 1, shared
+    unsigned long long* tick;  // ticket counter: a launch adds gridDim.x
+    unsigned long long* hcnt;  // arrivals after publishing h: a launch adds gridDim.x
+    unsigned long long* rflag; // tag of the last routing CTA 0 published
+    uint64_t* zs;              // [T][E] tagged logits (polled by CTA 0)
+    uint64_t* sax;             // [T][2r] tagged shared LoRA-A products (gate | up)
+    uint64_t* rax;             // [TK][2r] tagged routed LoRA-A products, routed slot t*K+k
+    uint64_t* route;           // [T][K] {expert, weight} published by CTA 0
+    float* hx;                 // [J][Imax] h: routed slot t*K+k, shared T*K+t
+    float* part;               // [NB][3][T][r] partial down LoRA-A sums: segment 0, 1, shared
     int32_t* status;
     int32_t* idx_out;          // [T][K] routing record
     float* w_out;
@@ -108,7 +111,7 @@ __device__ __noinline__ float spin(const uint64_t* p, uint32_t tag, int32_t* sta
     for (uint32_t i = 0;; ++i) {
         const unsigned long long w = peek(p);
         if (fresh(w, tag)) return wval(w);
-        if ((i & 15) == 15) {
+        if ((i & 7) == 7) {
             if (*abort) return 0.0f;
             if (tc::globaltimer_ns() - t0 > limit_ns) {
                 raise_status(status, MOE_ERR_TIMEOUT);
@@ -116,6 +119,31 @@ __device__ __noinline__ float spin(const uint64_t* p, uint32_t tag, int32_t* sta
                 return 0.0f;
             }
         }
+        __nanosleep(32);  // leave the issue slots to the warps that compute
+    }
+}
+
+__device__ __forceinline__ unsigned long long ld_acq64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// One thread: wait (bounded, with a short back-off between polls) until *p >= target
+// (ge) or *p == target; acquire semantics.  False on timeout (MOE_ERR_TIMEOUT, *abort).
+__device__ __noinline__ bool wait_word(const unsigned long long* p, unsigned long long target, bool ge,
+                                       int32_t* status, volatile int* abort, uint64_t limit_ns) {
+    const uint64_t t0 = tc::globaltimer_ns();
+    for (uint32_t i = 0;; ++i) {
+        const unsigned long long v = ld_acq64(p);
+        if (ge ? v >= target : v == target) return true;
+        if (*abort) return false;
+        if ((i & 7) == 7 && tc::globaltimer_ns() - t0 > limit_ns) {
+            raise_status(status, MOE_ERR_TIMEOUT);
+            *abort = 1;
+            return false;
+        }
+        __nanosleep(64);
     }
 }
 
@@ -143,6 +171,118 @@ __device__ void gather_range(const uint64_t* src, int n, float* dst, uint32_t ta
 __device__ __forceinline__ int swz(int i) {
     const int c = i >> 5, p = i & 31;
     return (c << 5) + (((p & ~3) + ((c & 7) << 2)) & 31) + (p & 3);
+}
+
+// Compact row dots for the chain kernel.  A launch runs most of its code once, so the
+// time of a step is set by the instructions it has to fetch, not by those it executes:
+// these loop over 32-element chunks with one chunk's body unrolled, instead of unrolling
+// several chunks.
+//
+// acc[m] += sum_j (s q_j + b) v_m[j] over one int4 row of length n, staged vectors
+// v_m = vbase + vid[m] * n, by lpt lanes (sl = lane in the group).  The nibble q goes
+// into the mantissa of 128.0f; the 128 is taken back through the bias term
+// (s sum (128 + q) v + (b - 128 s) sum v).
+template <int MT>
+__device__ __noinline__ void cdot_int4(const uint32_t* __restrict__ prow, const uint16_t* __restrict__ srow,
+                                       const uint16_t* __restrict__ brow, int group, int n, const float* vbase,
+                                       const float* vsum, const int* vid, int nv, float* acc, int sl, int lpt) {
+    const uint4* p4 = reinterpret_cast<const uint4*>(prow);
+    const int nc = n / 32;
+#pragma unroll 1
+    for (int c = sl; c < nc; c += lpt) {
+        const int g = (c * 32) / group;
+        const float s = bf16f(srow[g]), b128 = fmaf(-128.0f, s, bf16f(brow[g]));
+        const uint4 q4 = p4[c];
+        const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
+        const int rot = (c & 7) << 2;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            if (m >= nv) break;
+            const float* vr = vbase + vid[m] * n + (c << 5);
+            float a = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float4 x0 = *reinterpret_cast<const float4*>(vr + ((8 * w + rot) & 31));
+                const float4 x1 = *reinterpret_cast<const float4*>(vr + ((8 * w + 4 + rot) & 31));
+                const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                for (int f = 0; f < 8; ++f) {
+                    const uint32_t at16 = f <= 4 ? qw[w] << (16 - 4 * f) : qw[w] >> (4 * f - 16);
+                    a = fmaf(__uint_as_float((at16 & 0x000F0000u) | 0x43000000u), xv[f], a);
+                }
+            }
+            acc[m] = fmaf(s, a, fmaf(b128, vsum[vid[m] * nc + c], acc[m]));
+        }
+    }
+}
+
+// The same for an int8 row, full warp, vectors v_m = vbase + m * n.
+template <int MT>
+__device__ __noinline__ void cdot_int8(const uint32_t* __restrict__ prow, const uint16_t* __restrict__ srow,
+                                       const uint16_t* __restrict__ brow, int group, int n, const float* vbase,
+                                       const float* vsum, int nv, float* acc, int lane) {
+    const uint4* p4 = reinterpret_cast<const uint4*>(prow);
+    const int nc = n / 32;
+#pragma unroll 1
+    for (int c = lane; c < nc; c += 32) {
+        const int g = (c * 32) / group;
+        const float s = bf16f(srow[g]), b = bf16f(brow[g]);
+        const int rot = (c & 7) << 2;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            if (m >= nv) break;
+            const float* vr = vbase + m * n + (c << 5);
+            float a = 0.0f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 q4 = p4[2 * c + h];
+                const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const float4 xv = *reinterpret_cast<const float4*>(vr + ((16 * h + 4 * w + rot) & 31));
+                    a = fmaf(u2f_small(qw[w] & 255u), xv.x, a);
+                    a = fmaf(u2f_small((qw[w] >> 8) & 255u), xv.y, a);
+                    a = fmaf(u2f_small((qw[w] >> 16) & 255u), xv.z, a);
+                    a = fmaf(u2f_small(qw[w] >> 24), xv.w, a);
+                }
+            }
+            acc[m] = fmaf(s, a, fmaf(b, vsum[m * nc + c], acc[m]));
+        }
+    }
+}
+
+// bf16 rows (n elements, 16-byte aligned) into the swizzled fp32 layout with 32-element
+// chunk sums, optionally scaled (the normalised block input); a thread takes 8 elements.
+__device__ void cstage_bf16(float* dst, float* dsum, const uint16_t* src, int nv, int n, const float* scale) {
+    const int per = n / 8, total = nv * per, lim = (total + 31) / 32 * 32;
+#pragma unroll 1
+    for (int i = threadIdx.x; i < lim; i += kCT) {
+        const bool live = i < total;
+        const int v = live ? i / per : 0, q = live ? i % per : 0;
+        const uint4 raw = live ? reinterpret_cast<const uint4*>(src + (int64_t)v * n)[q] : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        float f[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            f[2 * k] = __uint_as_float(w[k] << 16);
+            f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+        }
+        if (scale && live)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) f[k] = bf16f(f2bf16(f[k] * scale[v]));
+        float sum = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) sum += f[k];
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        if (live) {
+            const int c = q / 4, o = (q % 4) * 8, rot = (c & 7) << 2;
+            float* d = dst + v * n + (c << 5);
+            *reinterpret_cast<float4*>(d + ((o + rot) & 31)) = make_float4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<float4*>(d + ((o + 4 + rot) & 31)) = make_float4(f[4], f[5], f[6], f[7]);
+            if ((q % 4) == 0) dsum[v * (n / 32) + c] = sum;
+        }
+    }
 }
 
 // sum_j A[j] v[j] for a bf16 row A of length n already in shared memory and one staged
@@ -229,8 +369,17 @@ __device__ __forceinline__ uint32_t warp_total(uint32_t v) {
 }
 
 template <int MT>
-__global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_constant__ CArgs a) {
+__global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_constant__ CArgs a_param) {
     extern __shared__ __align__(16) unsigned char sm[];
+    // The arguments (layer descriptor, adapter table, plan: about 2.3 KB) are read all over
+    // the kernel, most fields once; copied to shared memory by all threads at once, they
+    // cost one round trip here instead of a cold constant-cache miss at each first use.
+    __shared__ __align__(16) CArgs a_sm;
+    static_assert(sizeof(CArgs) % 4 == 0, "argument copy in words");
+    for (int i = threadIdx.x; i < (int)(sizeof(CArgs) / 4); i += kCT)
+        reinterpret_cast<uint32_t*>(&a_sm)[i] = reinterpret_cast<const uint32_t*>(&a_param)[i];
+    __syncthreads();
+    const CArgs& a = a_sm;
     const LayerArgs& L = a.L;
     const CPlan& P = a.P;
     const int T = a.T, H = L.H, E = L.E, K = L.K, I = L.I;
@@ -258,6 +407,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
     __shared__ __align__(8) uint64_t s_bar[5];
     __shared__ int s_abort;
     __shared__ uint32_t s_tag;
+    __shared__ unsigned long long s_hdone;
     __shared__ int s_aid[kCMaxT];
     __shared__ int32_t s_sel[kCMaxTK];
     __shared__ float s_inv[kCMaxT], s_sig[kCMaxT];
@@ -396,8 +546,11 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
         }
         __syncthreads();
     }
-    stage_bf16(xs, xsum, xr, T, H, a.block ? s_inv : nullptr);
-    if (warp == kCW - 1 && lane == 0) s_tag = (uint32_t)((prev / (unsigned long long)NB) % 0xffffffffull) + 1u;
+    cstage_bf16(xs, xsum, xr, T, H, a.block ? s_inv : nullptr);
+    if (warp == kCW - 1 && lane == 0) {
+        s_tag = (uint32_t)((prev / (unsigned long long)NB) % 0xffffffffull) + 1u;
+        s_hdone = (prev / (unsigned long long)NB + 1) * (unsigned long long)NB;  // h arrivals complete at this count
+    }
     __syncthreads();
     const uint32_t tag = s_tag;
 
@@ -416,7 +569,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
 #pragma unroll
                 for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
                 if (w[0])
-                    dot_int8<MT>(reinterpret_cast<const uint32_t*>(w[0] + (size_t)jj * H),
+                    cdot_int8<MT>(reinterpret_cast<const uint32_t*>(w[0] + (size_t)jj * H),
                                  reinterpret_cast<const uint16_t*>(w[1]) + jj * ng,
                                  reinterpret_cast<const uint16_t*>(w[2]) + jj * ng, q.group, H, xs, xsum, T, acc, lane);
 #pragma unroll
@@ -442,11 +595,11 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                     ag[m] = au[m] = 0.0f;
                     vid[m] = m;
                 }
-                dot_int4<MT>(reinterpret_cast<const uint32_t*>(s_aw[6] + (size_t)il * (H / 2)),
+                cdot_int4<MT>(reinterpret_cast<const uint32_t*>(s_aw[6] + (size_t)il * (H / 2)),
                              reinterpret_cast<const uint16_t*>(s_aw[7]) + il * ngg,
                              reinterpret_cast<const uint16_t*>(s_aw[8]) + il * ngg, L.s_gate.group, H, xs, xsum, vid, T,
                              ag, lane, 32);
-                dot_int4<MT>(reinterpret_cast<const uint32_t*>(s_aw[9] + (size_t)il * (H / 2)),
+                cdot_int4<MT>(reinterpret_cast<const uint32_t*>(s_aw[9] + (size_t)il * (H / 2)),
                              reinterpret_cast<const uint16_t*>(s_aw[10]) + il * ngu,
                              reinterpret_cast<const uint16_t*>(s_aw[11]) + il * ngu, L.s_up.group, H, xs, xsum, vid, T,
                              au, lane, 32);
@@ -464,18 +617,18 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
     }
 
     // ------------------------------------------------------------ phase K
-    gather_range(a.zs, T * E, z, tag, a.status, &s_abort, lim);
-    __syncthreads();
-    if (warp == 0) {
-        // top-K of each token: lane holds experts lane + 32 c; K rounds of a warp max on
-        // order-preserving keys, equal keys to the lower expert index.  With caller-given
-        // sets (the prerouter's prediction) the set is taken as it is and only the
-        // weights come from the logits.
-        for (int t = 0; t < T; ++t) {
-            if (a.select) {
+    // CTA 0 alone polls the logits, takes the top-K of each token (warp t for token t)
+    // and publishes the routing behind one release flag; every other CTA polls that
+    // flag with one thread, so no line is polled by the whole grid.
+    if (cta == 0) {
+        gather_range(a.zs, T * E, z, tag, a.status, &s_abort, lim);
+        __syncthreads();
+        if (warp < T) {
+            const int t = warp;
+            if (a.select) {  // caller-given sets (the prerouter's prediction): only the weights come from z
                 bool bad = false;
                 const int e = select_entry(s_sel + t * K, K, E, lane, &bad);
-                if (bad && lane == 0 && cta == 0) raise_status(a.status, MOE_ERR_DEVICE_INDEX);
+                if (bad && lane == 0) raise_status(a.status, MOE_ERR_DEVICE_INDEX);
                 const float zk = e >= 0 ? z[t * E + e] : -INFINITY;
                 const float m = warp_max(zk);
                 const float ev = e >= 0 ? expf(zk - m) : 0.0f;
@@ -484,16 +637,37 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                     s_idx[t][lane] = e;
                     s_w[t][lane] = ev / sum;
                 }
-                continue;
+            } else {
+                warp_topk<MOEQ_MAX_EXPERTS / 32>(z + t * E, E, K, lane, s_idx[t], s_w[t]);
             }
-            if (E <= 256) warp_topk<8>(z + t * E, E, K, lane, s_idx[t], s_w[t]);
-            else warp_topk<MOEQ_MAX_EXPERTS / 32>(z + t * E, E, K, lane, s_idx[t], s_w[t]);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            if (lane < TK) {
+                const int e = s_idx[lane / K][lane % K];
+                const float w = s_w[lane / K][lane % K];
+                a.route[lane] = ((unsigned long long)__float_as_uint(w) << 32) | (uint32_t)e;
+                a.idx_out[lane] = e;  // the routing this call used, for the caller's record
+                a.w_out[lane] = w;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence();
+                asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(a.rflag), "l"((unsigned long long)tag)
+                             : "memory");
+            }
+        }
+    } else if (warp == 0) {
+        if (lane == 0) wait_word(a.rflag, tag, false, a.status, &s_abort, lim);
+        __syncwarp();
+        if (lane < TK) {
+            const unsigned long long v = ld_acq64(reinterpret_cast<const unsigned long long*>(a.route) + lane);
+            s_idx[lane / K][lane % K] = (int)min((uint32_t)v, (uint32_t)(E - 1));  // (in range even after a timeout)
+            s_w[lane / K][lane % K] = __uint_as_float((uint32_t)(v >> 32));
         }
         __syncwarp();
-        if (cta == 0 && lane < TK) {  // the routing this call used, for the caller's record
-            a.idx_out[lane] = s_idx[lane / K][lane % K];
-            a.w_out[lane] = s_w[lane / K][lane % K];
-        }
+    }
+    if (warp == 0) {
         // routed jobs (lane = slot t*K+k) grouped by expert, ascending, then by slot
         const bool live = lane < TK;
         const int je = live ? s_idx[lane / K][lane % K] : 0x7fffffff;
@@ -703,7 +877,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                         u += L.scale * warp_sum(du);
                     }
                     const float hv = silu(g) * u;
-                    if (lane == 0) publish(a.hx + (int64_t)(TK + m) * max(I, Is) + i, hv, tag);
+                    if (lane == 0) a.hx[(int64_t)(TK + m) * max(I, Is) + i] = hv;
                     wacc[2][m] += ad[m] * hv;
                 }
                 continue;
@@ -733,11 +907,11 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
             for (int m = 0; m < MT; ++m) ag[m] = au[m] = 0.0f;
             const int ngg = H / L.gate.group, ngu = H / L.up.group;
             if (s_cw[sg][0] && s_cw[sg][3]) {  // (missing only when the CTA gave up before issuing them)
-                dot_int4<MT>(reinterpret_cast<const uint32_t*>(s_cw[sg][0] + (size_t)rs * (H / 2)),
+                cdot_int4<MT>(reinterpret_cast<const uint32_t*>(s_cw[sg][0] + (size_t)rs * (H / 2)),
                              reinterpret_cast<const uint16_t*>(s_cw[sg][1]) + rs * ngg,
                              reinterpret_cast<const uint16_t*>(s_cw[sg][2]) + rs * ngg, L.gate.group, H, xs, xsum, toks,
                              nt, ag, lane, 32);
-                dot_int4<MT>(reinterpret_cast<const uint32_t*>(s_cw[sg][3] + (size_t)rs * (H / 2)),
+                cdot_int4<MT>(reinterpret_cast<const uint32_t*>(s_cw[sg][3] + (size_t)rs * (H / 2)),
                              reinterpret_cast<const uint16_t*>(s_cw[sg][4]) + rs * ngu,
                              reinterpret_cast<const uint16_t*>(s_cw[sg][5]) + rs * ngu, L.up.group, H, xs, xsum, toks,
                              nt, au, lane, 32);
@@ -760,7 +934,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                     uu += L.scale * warp_sum((kk && bu) ? bf16f(bu[rs * r + lane]) * tu : 0.0f);
                 }
                 const float hv = silu(g) * uu;
-                if (lane == 0) publish(a.hx + (int64_t)slot * max(I, Is) + i, hv, tag);
+                if (lane == 0) a.hx[(int64_t)slot * max(I, Is) + i] = hv;
                 if (sg == 0) wacc[0][m] += ad[m] * hv;
                 else wacc[1][m] += ad[m] * hv;
             }
@@ -777,41 +951,52 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
             const int k = q % r, m = (q / r) % T, s = q / (r * T);
             float v = 0.0f;
             for (int w = 0; w < kCW; ++w) v += wpart[((w * 3 + s) * MT + m) * r + k];
-            publish(a.part + (((int64_t)cta * 3 + s) * T + m) * r + k, v, tag);
+            a.part[(((int64_t)cta * 3 + s) * T + m) * r + k] = v;
         }
+    }
+    // h and the partial sums of this CTA are written: one arrival (every CTA, every launch)
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(a.hcnt) : "memory");
     }
 
     // ------------------------------------------------------------ phase D
-    // h of every job (routed rows of length I, then the shared ones of length Is), staged
-    // in the swizzled layout; every thread's words of a pass are in flight together
+    // every CTA has written its h rows and partial sums once the arrival count is reached
+    if (tid == 0) wait_word(a.hcnt, s_hdone, true, a.status, &s_abort, lim);
+    __syncthreads();
+    // h of every job (routed rows of length I, then the shared ones of length Is), staged in
+    // the swizzled layout: 16-byte loads from L2, all of a thread's in flight together
     {
-        const int Imx = max(I, Is), nh = TK * I + T * Is;
-        auto hsrc = [&](int q) {
-            return q < TK * I ? a.hx + (int64_t)(q / I) * Imx + q % I
-                              : a.hx + (int64_t)(TK + (q - TK * I) / Is) * Imx + (q - TK * I) % Is;
-        };
-        for (int base = 0; base < nh; base += kGB * kCT) {
-            unsigned long long w[kGB];
+        const int Imx = max(I, Is);
+        const int nr4 = TK * (I / 4), nh4 = nr4 + T * (Is / 4);
+        for (int base = 0; base < nh4; base += 4 * kCT) {
+            float4 v[4];
 #pragma unroll
-            for (int b = 0; b < kGB; ++b) {
+            for (int b = 0; b < 4; ++b) {
                 const int q = base + b * kCT + tid;
-                w[b] = q < nh ? peek(hsrc(q)) : 0ull;
+                if (q < nh4) {
+                    const float* src = q < nr4 ? a.hx + (int64_t)(q / (I / 4)) * Imx + (q % (I / 4)) * 4
+                                               : a.hx + (int64_t)(TK + (q - nr4) / (Is / 4)) * Imx +
+                                                     ((q - nr4) % (Is / 4)) * 4;
+                    v[b] = __ldcg(reinterpret_cast<const float4*>(src));
+                }
             }
 #pragma unroll
-            for (int b = 0; b < kGB; ++b) {
+            for (int b = 0; b < 4; ++b) {
                 const int q = base + b * kCT + tid;
-                if (q >= nh) break;
-                const float v = fresh(w[b], tag) ? wval(w[b]) : spin(hsrc(q), tag, a.status, &s_abort, lim);
-                if (q < TK * I) hsm[(q / I) * I + swz(q % I)] = v;
-                else hsm[TK * I + ((q - TK * I) / Is) * Is + swz((q - TK * I) % Is)] = v;
+                if (q >= nh4) break;
+                float* dst = q < nr4 ? hsm + (q / (I / 4)) * I + swz((q % (I / 4)) * 4)
+                                     : hsm + TK * I + ((q - nr4) / (Is / 4)) * Is + swz(((q - nr4) % (Is / 4)) * 4);
+                *reinterpret_cast<float4*>(dst) = v[b];
             }
         }
     }
     if (lora) {
         // down LoRA-A products: for each job, the sum over the CTAs whose rows cover its
-        // expert of their published partials, in CTA order.  An item is (job, component,
-        // a run of up to 8 of those CTAs): its 8 words are polled together and summed;
-        // the items of a (job, component) are then summed in order.
+        // expert of their partial sums, in CTA order.  An item is (job, component, a run of
+        // up to 8 of those CTAs): its 8 loads are in flight together; the items of a (job,
+        // component) are then added in order.
         constexpr int kRun = 8;
         if (tid == 0) {
             int o = 0;
@@ -853,21 +1038,15 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                     s0 = 2;
                 }
                 const int64_t step = (int64_t)3 * T * r, off = (int64_t)m * r + k;
-                unsigned long long w[kRun];
+                float w[kRun];
 #pragma unroll
                 for (int i = 0; i < kRun; ++i) {
                     const int s = i == 0 ? s0 : (j < TK ? 0 : 2);
-                    w[i] = i < cnt ? peek(a.part + (int64_t)(c0 + i) * step + (int64_t)s * T * r + off) : 0ull;
+                    w[i] = i < cnt ? __ldcg(a.part + (int64_t)(c0 + i) * step + (int64_t)s * T * r + off) : 0.0f;
                 }
                 float v = 0.0f;
 #pragma unroll
-                for (int i = 0; i < kRun; ++i) {
-                    if (i >= cnt) break;
-                    const int s = i == 0 ? s0 : (j < TK ? 0 : 2);
-                    v += fresh(w[i], tag) ? wval(w[i])
-                                          : spin(a.part + (int64_t)(c0 + i) * step + (int64_t)s * T * r + off, tag,
-                                                 a.status, &s_abort, lim);
-                }
+                for (int i = 0; i < kRun; ++i) v += w[i];
                 gat[q] = v;
             }
             __syncthreads();
@@ -922,7 +1101,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
             for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
             const unsigned char* const* dw = shu ? s_sdw : s_dw[u];
             if (live && dw[0])
-                dot_int4<MT>(reinterpret_cast<const uint32_t*>(dw[0] + (size_t)ol * (n / 2)),
+                cdot_int4<MT>(reinterpret_cast<const uint32_t*>(dw[0] + (size_t)ol * (n / 2)),
                              reinterpret_cast<const uint16_t*>(dw[1]) + ol * ng,
                              reinterpret_cast<const uint16_t*>(dw[2]) + ol * ng, Wd.group, n,
                              shu ? hsm + TK * I - TK * n : hsm, shu ? hsum + TK * (I / 32) - TK * (n / 32) : hsum, sl_,
@@ -1135,14 +1314,16 @@ cudaError_t launch_chain_mt(const CArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-// Words of the tagged-slot region a layer shape needs (sized for the largest token
-// count the kernel takes with this top-K, so its place and size do not depend on T).
+// Words (8 bytes) of the chain kernel's region a layer shape needs: its ticket and
+// counters, the tagged words (logits, LoRA-A products), the routing CTA 0 publishes, h
+// and the partial down LoRA-A sums; sized for the largest token count the kernel takes
+// with this top-K, so that its place and size do not depend on T.
 size_t chain_slot_words(int E, int K, int I, int Is, int r) {
     const int Tm = std::min(kCMaxT, kCMaxTK / std::max(K, 1));
     if (Tm < 1) return 0;
-    const int rr = std::max(r, 1), Jm = Tm * (K + 1), Imx = std::max(I, Is);
-    return (size_t)Tm * E + (size_t)Tm * 2 * rr + (size_t)Tm * K * 2 * rr + (size_t)Jm * Imx +
-           (size_t)MOEQ_DECODE_MAX_CTAS * 3 * Tm * rr;
+    const size_t rr = std::max(r, 1), Jm = (size_t)Tm * (K + 1), Imx = std::max(I, Is);
+    return 8 + (size_t)Tm * E + (size_t)Tm * 2 * rr + (size_t)Tm * K * 2 * rr + (size_t)Tm * K +
+           (Jm * Imx + 1) / 2 + ((size_t)MOEQ_DECODE_MAX_CTAS * 3 * Tm * rr + 1) / 2 + 2;
 }
 
 bool chain_supported(const LayerArgs& L, int T) {
@@ -1163,20 +1344,26 @@ cudaError_t launch_chain(const LayerArgs& L, const uint16_t* x, const int32_t* a
     a.T = T;
     a.block = block;
     a.eps = eps;
-    a.tick = sc.tick;
     const int K = L.K, I = L.I, Is = L.has_shared ? L.Is : 0;
-    const int r = std::max(L.n_adapters > 0 ? L.rank : 0, 1);
-    const int Tm = std::min(kCMaxT, kCMaxTK / K), Jm = Tm * (K + 1), Imx = std::max(I, Is);
+    const size_t r = std::max(L.n_adapters > 0 ? L.rank : 0, 1);
+    const size_t Tm = std::min(kCMaxT, kCMaxTK / K), Jm = Tm * (K + 1), Imx = std::max(I, Is);
     uint64_t* p = sc.slots;
+    a.tick = reinterpret_cast<unsigned long long*>(p);
+    a.hcnt = reinterpret_cast<unsigned long long*>(p + 1);
+    a.rflag = reinterpret_cast<unsigned long long*>(p + 2);
+    p += 8;
     a.zs = p;
-    p += (size_t)Tm * L.E;
+    p += Tm * L.E;
     a.sax = p;
-    p += (size_t)Tm * 2 * r;
+    p += Tm * 2 * r;
     a.rax = p;
-    p += (size_t)Tm * K * 2 * r;
-    a.hx = p;
-    p += (size_t)Jm * Imx;
-    a.part = p;
+    p += Tm * K * 2 * r;
+    a.route = p;
+    p += Tm * K;
+    p += (reinterpret_cast<uintptr_t>(p) & 15) ? 1 : 0;  // 16-byte aligned float rows
+    a.hx = reinterpret_cast<float*>(p);
+    p += (Jm * Imx + 1) / 2;
+    a.part = reinterpret_cast<float*>(p);
     a.status = sc.status;
     a.idx_out = sc.idx_out;
     a.w_out = sc.w_out;

@@ -361,11 +361,11 @@ def test_block_tiny_chain(T):
 
 def test_bounded_wait_runs_out_and_reports_timeout():
     """A bounded device wait that cannot be satisfied gives up, reports MOE_ERR_TIMEOUT and
-    leaves the context usable.  The workspace's ticket counter (header bytes 8..15) is set
-    to 1 instead of a multiple of the grid, so one CTA of the chain decode kernel takes a
-    different epoch from the others and no CTA ever sees all the words it polls for; with a
-    2 ms wait limit every CTA gives up.  After re-initialising the workspace the same call
-    runs normally."""
+    leaves the context usable.  The chain decode kernel's ticket counter (the first word of
+    its region, right after the 256-byte workspace header) is set to 1 instead of a multiple
+    of the grid, so one CTA takes a different epoch from the others and waits for words and
+    counts that never come; with a 2 ms wait limit it gives up.  After re-initialising the
+    workspace the same call runs normally."""
     m, ly = _mods()
     shape = workloads.TINY
     t, x, aid = _ffn_case(shape, 470, T=1)
@@ -373,7 +373,7 @@ def test_bounded_wait_runs_out_and_reports_timeout():
     ws, nb = d.workspace(1)
     xd = ly.to_device(x)
     y = torch.zeros_like(xd)
-    ws.view(torch.int64)[1] = 1
+    ws.view(torch.int64)[32] = 1
     m.moe_set_wait_limit_ns(2_000_000)
     try:
         m.moe_timing_enable(True)
