@@ -380,6 +380,9 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
         reinterpret_cast<uint32_t*>(&a_sm)[i] = reinterpret_cast<const uint32_t*>(&a_param)[i];
     __syncthreads();
     const CArgs& a = a_sm;
+    // the next kernel on the stream may launch now; it waits for this grid before it
+    // reads anything this grid writes
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const LayerArgs& L = a.L;
     const CPlan& P = a.P;
     const int T = a.T, H = L.H, E = L.E, K = L.K, I = L.I;
@@ -443,15 +446,15 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
     const int o_lo = min(H, cta * P.perO), o_hi = min(H, o_lo + P.perO), no = o_hi - o_lo;
 
     // ------------------------------------------------------------ phase R: issue
+    // The weight rows of this phase depend on nothing the previous kernel on the stream
+    // writes: their copies start before the grid-dependency wait (launched as a
+    // programmatic dependent, this kernel's CTAs get here while that kernel finishes).
+    // Everything that reads the workspace, x or the adapter ids comes after the wait.
     unsigned long long prev = 0;  // this launch's ticket (first needed after x is staged)
-    if (warp == kCW - 1 && lane == 0)
-        asm volatile("atom.add.relaxed.gpu.global.u64 %0, [%1], 1;" : "=l"(prev) : "l"(a.tick) : "memory");
     if (warp == 0) {
         uint32_t tx = 0;
         unsigned char* wa = sm + P.wa;
-        if (lane == 0) {
-            win(sm + P.xraw, a.x, (uint32_t)(T * H * 2), &s_bar[0], &tx);
-        } else if (lane >= 1 && lane < 13) {
+        if (lane >= 1 && lane < 13) {
             const int w = lane - 1, k = w % 3, g = w / 3;  // g: router, shared gate, s_gate, s_up
             const moe_qtensor& q = g == 0 ? L.router : g == 1 ? L.shared_gate : g == 2 ? L.s_gate : L.s_up;
             if (g == 1) {  // the shared-gate row is read by every CTA straight from global memory (L2)
@@ -473,8 +476,6 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
                 s_aw[w] = win(wa + P.a_off[w], src, bytes, &s_bar[0], &tx);
             }
         }
-        tx = warp_total(tx);
-        if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[0], tx);
         uint32_t tx1 = 0;
         if (lane < 3) {  // the shared-expert down rows of this CTA's output range
             const int ngd = sh ? Is / L.s_down.group : 0;
@@ -489,8 +490,13 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
         }
         tx1 = warp_total(tx1);
         if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[1], tx1);
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (lane == 0) win(sm + P.xraw, a.x, (uint32_t)(T * H * 2), &s_bar[0], &tx);
+        tx = warp_total(tx);
+        if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[0], tx);
     } else if (warp == 1) {
         // adapter ids, then the shared-expert LoRA rows this CTA needs
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         if (lane < T) {
             int ad = a.adapter_id ? a.adapter_id[lane] : (L.n_adapters > 0 ? 0 : -1);
             if (ad < -1 || ad >= L.n_adapters) {
@@ -521,6 +527,12 @@ __global__ void __launch_bounds__(kCT, 1) decode_chain_kernel(const __grid_const
         }
         tx = warp_total(tx);
         if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[1], tx);
+    }
+
+    if (warp >= 2) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (warp == kCW - 1 && lane == 0)
+            asm volatile("atom.add.relaxed.gpu.global.u64 %0, [%1], 1;" : "=l"(prev) : "l"(a.tick) : "memory");
     }
 
     // ------------------------------------------------------------ phase R: compute
@@ -1304,11 +1316,13 @@ cudaError_t launch_chain_mt(const CArgs& a, cudaStream_t s) {
     cfg.blockDim = dim3(kCT);
     cfg.dynamicSmemBytes = a.P.total;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, decode_chain_kernel<MT>, a);
 }
 
