@@ -362,6 +362,46 @@ MOEQ_API moe_status moe_mixed_mlp_forward(const moe_mixed_tensor* gate, const mo
                                  const moe_mixed_tensor* down, const uint16_t* x, int32_t T, int32_t residual,
                                  float eps, uint16_t* y, void* workspace, size_t ws_bytes, moe_stream stream);
 
+/* ------------------------------------------------------ expert parallelism
+ * Building blocks of the expert-parallel forward over G ranks (one process per GPU),
+ * each owning E/G consecutive experts, with the router and the shared expert
+ * replicated: route locally (moe_router_topk), moe_ep_dispatch, an all-to-all of the
+ * rows (NCCL, by the caller), moe_experts_forward on the rows received, the reverse
+ * all-to-all, the shared expert on the local tokens, moe_ep_combine.  The sum over a
+ * token's experts is the forward's own sum (fixed order k = 0..K-1, then the shared
+ * expert); the expert outputs cross the all-to-all as bf16.
+ *
+ * moe_experts_forward: y[n] = E_{expert[n]}(x[n]) for N rows (no router, no shared
+ * expert, weight 1), adapter_id [N] or NULL as for moe_ffn_forward; an expert index
+ * outside [0, E) makes its row zero and raises MOE_ERR_DEVICE_INDEX.  x, y device bf16
+ * [N][H]; workspace of moe_experts_workspace_bytes(layer, N) bytes, 256-byte aligned,
+ * initialised once.  A layer whose expert tensors are views of E/G experts (n = E/G)
+ * is a rank's slice.
+ *
+ * moe_ep_dispatch: the routed jobs j = t*K + k of T local tokens (topk_idx device int32
+ * [T][K], experts of a layer with E experts) in send order: rank-major (owner =
+ * expert / (E/G)), job order within a rank.  Writes pos [T][K] (the send row of each
+ * job), counts [G] (rows per rank), send_x [T*K][H] bf16 (x[t] of each job) and
+ * send_meta [T*K][2] = {expert, adapter id}.  All device pointers; E % G == 0,
+ * G <= 64, H % 8 == 0.  An expert index out of range is clamped and raises
+ * MOE_ERR_DEVICE_INDEX in *status (a device int32 word).
+ *
+ * moe_ep_combine: y[t] = bf16(sum_k topk_w[t][k] ret[pos[t][k]] + shared_scale[t]
+ * shared[t]) (shared NULL: no shared term; shared_scale NULL: scale 1); ret device
+ * bf16 [T*K][H] in send order. */
+#define MOEQ_EP_MAX_RANKS 64
+MOEQ_API size_t moe_experts_workspace_bytes(const moe_layer* layer, int32_t N);
+MOEQ_API moe_status moe_experts_forward(const moe_layer* layer, const uint16_t* x, const int32_t* expert,
+                                        const int32_t* adapter_id, int32_t N, uint16_t* y, void* workspace,
+                                        size_t ws_bytes, moe_stream stream);
+MOEQ_API moe_status moe_ep_dispatch(const uint16_t* x, const int32_t* topk_idx, const int32_t* adapter_id,
+                                    int32_t n_adapters, int32_t T, int32_t K, int32_t H, int32_t E, int32_t G,
+                                    int32_t* pos, int32_t* counts, uint16_t* send_x, int32_t* send_meta,
+                                    int32_t* status, moe_stream stream);
+MOEQ_API moe_status moe_ep_combine(const uint16_t* ret, const int32_t* pos, const float* topk_w,
+                                   const uint16_t* shared, const float* shared_scale, int32_t T, int32_t K,
+                                   int32_t H, uint16_t* y, moe_stream stream);
+
 /* ------------------------------------- a7 in weight-activation form (8-bit A)
  * The mixed layer with 8-bit activations ("EDGERAZOR 深度解读" section 2.1 矩阵乘法
  * 分解, Y = sum (s_W s_X) Q(W)^T Q(X), and the 1.88-8-8 / 1.58-8-8 rows of the

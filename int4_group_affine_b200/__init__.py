@@ -24,7 +24,8 @@ __all__ = [
     "moe_ffn_routing", "moe_set_wait_limit_ns", "moe_wait_limit_ns", "Prerouter", "moe_ffn_forward_select",
     "moe_prerouter_workspace_bytes", "moe_prerouter_forward", "moe_act8_quant",
     "moe_mixed_linear_a8_workspace_bytes", "moe_mixed_linear_a8", "moe_mixed_mlp_a8_workspace_bytes",
-    "moe_mixed_mlp_forward_a8",
+    "moe_mixed_mlp_forward_a8", "moe_experts_workspace_bytes", "moe_experts_forward", "moe_ep_dispatch",
+    "moe_ep_combine",
 ]
 
 
@@ -239,3 +240,26 @@ def moe_mixed_mlp_forward_a8(gate: MixedTensor, up: MixedTensor, down: MixedTens
     _check("moe_mixed_mlp_forward_a8", _lib.lib().moe_mixed_mlp_forward_a8(
         ctypes.byref(gate), ctypes.byref(up), ctypes.byref(down), _ptr(x), T, residual, eps, _ptr(y),
         _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def moe_experts_workspace_bytes(layer: Layer, N) -> int:
+    return int(_lib.lib().moe_experts_workspace_bytes(ctypes.byref(layer), N))
+
+
+def moe_experts_forward(layer: Layer, x, expert, adapter_id, N, y, workspace, ws_bytes, stream=None):
+    """y[n] = expert[n]'s SwiGLU FFN (with its LoRA delta) of x[n]; no router, no shared expert."""
+    _check("moe_experts_forward", _lib.lib().moe_experts_forward(
+        ctypes.byref(layer), _ptr(x), _ptr(expert), _ptr(adapter_id), N, _ptr(y), _ptr(workspace), ws_bytes,
+        _stream(stream)))
+
+
+def moe_ep_dispatch(x, topk_idx, adapter_id, n_adapters, T, K, H, E, G, pos, counts, send_x, send_meta, status,
+                    stream=None):
+    _check("moe_ep_dispatch", _lib.lib().moe_ep_dispatch(
+        _ptr(x), _ptr(topk_idx), _ptr(adapter_id), n_adapters, T, K, H, E, G, _ptr(pos), _ptr(counts), _ptr(send_x),
+        _ptr(send_meta), _ptr(status), _stream(stream)))
+
+
+def moe_ep_combine(ret, pos, topk_w, shared, shared_scale, T, K, H, y, stream=None):
+    _check("moe_ep_combine", _lib.lib().moe_ep_combine(
+        _ptr(ret), _ptr(pos), _ptr(topk_w), _ptr(shared), _ptr(shared_scale), T, K, H, _ptr(y), _stream(stream)))

@@ -88,6 +88,10 @@ SIGNATURES = {
     "moe_mixed_linear_a8": (ctypes.c_int, [PM, P, I32, P, P, SZ, P]),
     "moe_mixed_mlp_a8_workspace_bytes": (SZ, [I32, I32, I32]),
     "moe_mixed_mlp_forward_a8": (ctypes.c_int, [PM, PM, PM, P, I32, I32, F32, P, P, SZ, P]),
+    "moe_experts_workspace_bytes": (SZ, [PL, I32]),
+    "moe_experts_forward": (ctypes.c_int, [PL, P, P, P, I32, P, P, SZ, P]),
+    "moe_ep_dispatch": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P]),
+    "moe_ep_combine": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, P, P]),
     "moe_timing_kinds": (ctypes.c_int, []),
     "moe_timing_kind_name": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_timing_enable": (ctypes.c_int, [ctypes.c_int]),

@@ -233,6 +233,9 @@ moe_status router_enqueue(const uint16_t* x, const moe_qtensor& router, const mo
     return MOE_OK;
 }
 
+moe_status experts_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, int T,
+                           const uint16_t* residual, uint16_t* y, const Work& wk, cudaStream_t s);
+
 // The launch sequence shared by moe_ffn_forward and moe_block_forward.
 moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, const int32_t* select, int T,
                        const uint16_t* residual, uint16_t* y, const Work& wk, cudaStream_t s) {
@@ -245,6 +248,14 @@ moe_status ffn_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* ada
                                     wk.status, s));
     else
         LAUNCH(kTopk, launch_topk(wk.logits, wk.gs, la.has_sgate, T, la.E, la.K, wk.idx, wk.w, wk.sg, s));
+    return experts_enqueue(L, x, adapter_id, T, residual, y, wk, s);
+}
+
+// From the routing in the workspace (idx, w, sg) on: index build, the expert GEMMs or
+// GEMVs (tensor cores from kTcMinTokens tokens on) and the fixed-order combine.
+moe_status experts_enqueue(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id, int T,
+                           const uint16_t* residual, uint16_t* y, const Work& wk, cudaStream_t s) {
+    const LayerArgs la = args_of(L);
     CHECK_CUDA(launch_index_build(wk, adapter_id, L->n_adapters, s));
     // Jobs of the shared expert stay in its group even without a shared expert:
     // their weights are zero-sized then, so they are skipped by the kernels.
@@ -750,6 +761,79 @@ moe_status moe_mixed_mlp_forward_a8(const moe_mixed_tensor* gate, const moe_mixe
     LAUNCH(kAct8, launch_act8(nullptr, h, T, I, nullptr, ah.q4, ah.q2, ah.s, ah.qsum, s));
     LAUNCH(kMixedA8, launch_mixed_a8(*down, nullptr, G, ah.q4, ah.q2, ah.s, ah.qsum, T, 2, nullptr, y,
                                      residual ? x : nullptr, s));
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------ expert parallelism
+namespace {
+// The layer as the experts-only forward sees it: one routed expert per row, no shared expert.
+moe_layer experts_only(const moe_layer* L) {
+    moe_layer c = *L;
+    c.top_k = 1;
+    memset(&c.s_gate, 0, sizeof(c.s_gate));
+    memset(&c.s_up, 0, sizeof(c.s_up));
+    memset(&c.s_down, 0, sizeof(c.s_down));
+    memset(&c.shared_gate, 0, sizeof(c.shared_gate));
+    for (int a = 0; a < MOEQ_MAX_ADAPTERS; ++a) {
+        memset(&c.lora[a].s_gate, 0, sizeof(moe_lora_proj));
+        memset(&c.lora[a].s_up, 0, sizeof(moe_lora_proj));
+        memset(&c.lora[a].s_down, 0, sizeof(moe_lora_proj));
+    }
+    return c;
+}
+}  // namespace
+
+size_t moe_experts_workspace_bytes(const moe_layer* layer, int32_t N) {
+    if (!layer || N < 0 || validate_layer(layer) != MOE_OK) return 0;
+    const moe_layer c = experts_only(layer);
+    return plan_of(dims_of(&c, N)).total;
+}
+
+moe_status moe_experts_forward(const moe_layer* layer, const uint16_t* x, const int32_t* expert,
+                               const int32_t* adapter_id, int32_t N, uint16_t* y, void* workspace, size_t ws_bytes,
+                               moe_stream stream) {
+    moe_status st = validate_layer(layer);
+    if (st != MOE_OK) return st;
+    CHECK_ARG(N >= 0);
+    const moe_layer c = experts_only(layer);
+    const Dims d = dims_of(&c, N);
+    const WsPlan p = plan_of(d);
+    st = ws_check(workspace, ws_bytes, p.total);
+    if (st != MOE_OK) return st;
+    if (N == 0) return MOE_OK;
+    CHECK_ARG(x && y && expert && x != y && aligned(x, 16) && aligned(y, 2));
+    cudaStream_t s = (cudaStream_t)stream;
+    const Work wk = work_of(d, p, workspace);
+    timing_begin(s);
+    LAUNCH(kTopk, launch_given_experts(expert, N, wk.idx, wk.w, wk.sg, s));
+    return experts_enqueue(&c, x, adapter_id, N, nullptr, y, wk, s);
+}
+
+moe_status moe_ep_dispatch(const uint16_t* x, const int32_t* topk_idx, const int32_t* adapter_id, int32_t n_adapters,
+                           int32_t T, int32_t K, int32_t H, int32_t E, int32_t G, int32_t* pos, int32_t* counts,
+                           uint16_t* send_x, int32_t* send_meta, int32_t* status, moe_stream stream) {
+    CHECK_ARG(T >= 0 && K > 0 && H > 0 && E > 0 && G > 0 && n_adapters >= 0);
+    if (G > MOEQ_EP_MAX_RANKS || E > MOEQ_MAX_EXPERTS || K > MOEQ_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    CHECK_ARG(E % G == 0 && H % 8 == 0);
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && topk_idx && pos && counts && send_x && send_meta && status && aligned(x, 16) &&
+              aligned(send_x, 16));
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    LAUNCH(kEpDispatch, launch_ep_dispatch(x, topk_idx, adapter_id, n_adapters, T, K, H, E, G, pos, counts, send_x,
+                                           send_meta, status, s));
+    return MOE_OK;
+}
+
+moe_status moe_ep_combine(const uint16_t* ret, const int32_t* pos, const float* topk_w, const uint16_t* shared,
+                          const float* shared_scale, int32_t T, int32_t K, int32_t H, uint16_t* y,
+                          moe_stream stream) {
+    CHECK_ARG(T >= 0 && K > 0 && H > 0 && H % 2 == 0);
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(ret && pos && topk_w && y && aligned(ret, 4) && aligned(y, 4) && (!shared || aligned(shared, 4)));
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    LAUNCH(kEpCombine, launch_ep_combine(ret, pos, topk_w, shared, shared_scale, T, K, H, y, s));
     return MOE_OK;
 }
 

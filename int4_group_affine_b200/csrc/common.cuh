@@ -143,7 +143,7 @@ struct DecodeScratch {
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
     kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kTcLoraGUKind, kTcGUKind,
-    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kDecodeChain, kPrerouter, kAct8, kMixedA8, kKindCount
+    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kDecodeChain, kPrerouter, kAct8, kMixedA8, kEpDispatch, kEpCombine, kKindCount
 };
 void timing_begin(cudaStream_t s);
 void timing_mark(int kind, cudaStream_t s);
@@ -239,6 +239,14 @@ cudaError_t launch_act8(const uint16_t* xb, const float* xf, int T, int n, int8_
 cudaError_t launch_mixed_a8(const moe_mixed_tensor& W, const moe_mixed_tensor* U, int G, const int8_t* q4,
                             const int8_t* q2, const float* sx, const int32_t* qsum, int T, int mode, float* yf,
                             uint16_t* yb, const uint16_t* residual, cudaStream_t s);
+
+// Expert parallelism (csrc/ep.cu); MOEQ_EP_MAX_RANKS comes from moeq.h.
+cudaError_t launch_given_experts(const int32_t* expert, int N, int32_t* idx, float* w, float* sg, cudaStream_t s);
+cudaError_t launch_ep_dispatch(const uint16_t* x, const int32_t* idx, const int32_t* adapter_id, int n_adapters, int T,
+                               int K, int H, int E, int G, int32_t* pos, int32_t* counts, uint16_t* send_x,
+                               int32_t* meta, int32_t* status, cudaStream_t s);
+cudaError_t launch_ep_combine(const uint16_t* ret, const int32_t* pos, const float* w, const uint16_t* shared,
+                              const float* sg, int T, int K, int H, uint16_t* y, cudaStream_t s);
 
 // Device row offset (in words) of row `o` of a mixed matrix with super-group size G.
 __host__ __device__ __forceinline__ int64_t mixed_row_offset(int o, int in, int G) {
