@@ -336,6 +336,19 @@ MOEQ_API moe_status moe_get_device_status(void* workspace, moe_stream stream, in
 MOEQ_API moe_status moe_ffn_routing(const moe_layer* layer, int32_t T, const void* workspace, size_t ws_bytes,
                                     int32_t* topk_idx, float* topk_w, moe_stream stream);
 
+/* Which single-kernel decode a forward of 1..8 tokens tries first.  AUTO: the barrier
+ * kernel (two grid-wide barriers, every CTA takes the top-K itself) for top-4 or less
+ * without a given expert set, the chain kernel (no grid barrier; CTA 0 routes and
+ * publishes, every hand-off an epoch-tagged word or an arrival count) otherwise, as
+ * measured faster for each; CHAIN or BARRIER: that kernel whenever it takes the call.
+ * A call neither kernel takes runs on the multi-kernel paths.  Process-wide, read when
+ * a call enqueues its kernels, not thread-safe. */
+#define MOE_DECODE_AUTO 0
+#define MOE_DECODE_CHAIN 1
+#define MOE_DECODE_BARRIER 2
+MOEQ_API moe_status moe_set_decode_path(int path);
+MOEQ_API int moe_decode_path(void);
+
 /* Bound of every device-side wait (a grid-wide arrival, a ready flag, a bulk-copy
  * or pipeline barrier), in nanoseconds of device time; 0 restores the default of
  * one second.  A wait that runs out sets MOE_ERR_TIMEOUT in the status word and the

@@ -25,8 +25,10 @@ __all__ = [
     "moe_prerouter_workspace_bytes", "moe_prerouter_forward", "moe_act8_quant",
     "moe_mixed_linear_a8_workspace_bytes", "moe_mixed_linear_a8", "moe_mixed_mlp_a8_workspace_bytes",
     "moe_mixed_mlp_forward_a8", "moe_experts_workspace_bytes", "moe_experts_forward", "moe_ep_dispatch",
-    "moe_ep_combine",
+    "moe_ep_combine", "moe_set_decode_path", "moe_decode_path", "DECODE_AUTO", "DECODE_CHAIN", "DECODE_BARRIER",
 ]
+
+DECODE_AUTO, DECODE_CHAIN, DECODE_BARRIER = 0, 1, 2
 
 
 class MoeError(RuntimeError):
@@ -263,3 +265,11 @@ def moe_ep_dispatch(x, topk_idx, adapter_id, n_adapters, T, K, H, E, G, pos, cou
 def moe_ep_combine(ret, pos, topk_w, shared, shared_scale, T, K, H, y, stream=None):
     _check("moe_ep_combine", _lib.lib().moe_ep_combine(
         _ptr(ret), _ptr(pos), _ptr(topk_w), _ptr(shared), _ptr(shared_scale), T, K, H, _ptr(y), _stream(stream)))
+
+
+def moe_set_decode_path(path: int):
+    _check("moe_set_decode_path", _lib.lib().moe_set_decode_path(int(path)))
+
+
+def moe_decode_path() -> int:
+    return int(_lib.lib().moe_decode_path())

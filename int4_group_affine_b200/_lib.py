@@ -79,6 +79,8 @@ SIGNATURES = {
     "moe_ffn_static_device_status": (ctypes.c_int, [P, ctypes.POINTER(I32)]),
     "moe_ffn_routing": (ctypes.c_int, [PL, I32, P, SZ, P, P, P]),
     "moe_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
+    "moe_set_decode_path": (ctypes.c_int, [ctypes.c_int]),
+    "moe_decode_path": (ctypes.c_int, []),
     "moe_wait_limit_ns": (ctypes.c_uint64, []),
     "moe_ffn_forward_select": (ctypes.c_int, [PL, P, P, P, I32, P, P, SZ, P]),
     "moe_prerouter_workspace_bytes": (SZ, [ctypes.POINTER(Prerouter), I32]),

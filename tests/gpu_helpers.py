@@ -1,6 +1,7 @@
 """Shared pieces of the GPU parity tests: device upload, tolerances, near-tie handling."""
 from __future__ import annotations
 
+import contextlib
 import itertools
 
 import numpy as np
@@ -98,15 +99,30 @@ def check_weights(idx_gpu, w_gpu, idx_ref, w_ref, ties, rtol=2e-5, atol=1e-6):
             assert abs(g[e] - r[e]) <= atol + rtol * abs(r[e]), (t, e, g[e], r[e])
 
 
-def forward_with_record(m, d, xd, ad, T, ws, nb, block_eps=None):
+@contextlib.contextmanager
+def decode_path(m, path):
+    """Runs the block with the single-kernel decode choice set to `path` (None: unchanged)."""
+    old = m.moe_decode_path()
+    if path is not None:
+        m.moe_set_decode_path(path)
+    try:
+        yield
+    finally:
+        m.moe_set_decode_path(old)
+
+
+def forward_with_record(m, d, xd, ad, T, ws, nb, block_eps=None, decode=None):
     """One forward through the C ABI with the library's launch record on: returns the
-    routing the call used (from moe_ffn_routing) and the kernel kinds it launched."""
+    routing the call used (from moe_ffn_routing) and the kernel kinds it launched.
+    `decode` forces one single-kernel decode (m.DECODE_CHAIN / m.DECODE_BARRIER)."""
     K = d.K
     idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
     w = torch.empty((T, K), dtype=torch.float32, device="cuda")
     y = torch.empty_like(xd)
     m.moe_timing_enable(True)
     try:
+        if decode is not None:
+            m.moe_set_decode_path(decode)
         if block_eps is None:
             m.moe_ffn_forward(d.L, xd, ad, T, y, ws, nb)
         else:
@@ -116,12 +132,13 @@ def forward_with_record(m, d, xd, ad, T, ws, nb, block_eps=None):
         kinds = set(m.moe_timing_collect())
     finally:
         m.moe_timing_enable(False)
+        m.moe_set_decode_path(m.DECODE_AUTO)
     assert m.moe_get_device_status(ws) == 0
     return y, idx.cpu().numpy(), w.cpu().numpy(), kinds
 
 
 # kernel kinds that identify each execution path of the forward: "chain" and "fused" are
-# the two single-kernel decode paths, "decode" either of them
+# the two single-kernel decode paths (chain kernel, barrier kernel), "decode" either of them
 PATH_KINDS = {"chain": {"decode_chain"}, "fused": {"decode_fused"}, "cuda_core": {"gate_up", "down"},
               "tensor_core": {"tc_gate_up", "tc_down"}}
 

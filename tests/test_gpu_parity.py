@@ -203,17 +203,18 @@ def _ffn_case(shape, seed, T=None, n_adapters=None, lora_zero_B=False):
     return t, x, aid
 
 
-def _check_ffn(shape, t, x, aid, n_adapters=None, what="", path=None):
+def _check_ffn(shape, t, x, aid, n_adapters=None, what="", path=None, decode=None):
     """The forward against the oracle: the routing the forward itself used (bit-exact
     outside near ties, weights within fp32 rounding), then the output, with near ties
-    resolved by the forward's own choice.  `path` names the kernels the call must run."""
+    resolved by the forward's own choice.  `path` names the kernels the call must run;
+    `decode` forces one of the single-kernel decodes."""
     m, ly = _mods()
     L = oracle_layer(shape, t, n_adapters=n_adapters)
     d = ly.DeviceLayer.from_host(shape, t, n_adapters=n_adapters)
     T = x.shape[0]
     ws, nb = d.workspace(T)
     yd, idx_g, w_g, kinds = forward_with_record(m, d, ly.to_device(x), None if aid is None else ly.to_device(aid),
-                                                T, ws, nb)
+                                                T, ws, nb, decode=decode)
     if path is not None:
         assert path_ran(path, kinds), (what, path, kinds)
     y = bf16_dev_to_f64(yd)
@@ -227,9 +228,14 @@ def _check_ffn(shape, t, x, aid, n_adapters=None, what="", path=None):
 
 @pytest.mark.parametrize("T", [4, 1, 12, 37, 70])
 def test_ffn_tiny(T):
+    """Up to four tokens at top-2: the barrier decode kernel by default, then the chain
+    kernel forced; more tokens: the tensor-core path."""
+    m, _ = _mods()
     shape = workloads.TINY
     t, x, aid = _ffn_case(shape, 400, T=T)
-    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T, path="chain" if T <= 4 else "tensor_core")
+    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T, path="fused" if T <= 4 else "tensor_core")
+    if T <= 4:
+        _check_ffn(shape, t, x, aid, what="tiny T=%d chain" % T, path="chain", decode=m.DECODE_CHAIN)
 
 
 @pytest.mark.parametrize("T", [5, 6])
@@ -294,8 +300,10 @@ def test_ffn_tiny_variants(variant):
     if variant == "multi_adapter":
         aid = aid.copy()
         aid[::5] = -1  # some tokens with the base only
+    m, _ = _mods()
     _check_ffn(shape, t, x, aid, n_adapters=na, what=variant + (" (chain)" if chain else ""),
-               path="chain" if (chain or variant == "group32_decode") else None)
+               path="chain" if chain else ("decode" if variant == "group32_decode" else None),
+               decode=m.DECODE_CHAIN if chain else None)
 
 
 def test_zero_B_equals_base_bitwise():
@@ -353,7 +361,8 @@ def test_block_tiny_chain(T):
     L = oracle_layer(shape, t)
     d = ly.DeviceLayer.from_host(shape, t)
     ws, nb = d.workspace(T)
-    yd, idx_g, _, kinds = forward_with_record(m, d, ly.to_device(x), None, T, ws, nb, block_eps=1e-6)
+    yd, idx_g, _, kinds = forward_with_record(m, d, ly.to_device(x), None, T, ws, nb, block_eps=1e-6,
+                                              decode=m.DECODE_CHAIN)
     assert path_ran("chain", kinds), kinds
     ref = synth.bf16_to_f32(L.block(x, eps=1e-6)).astype(np.float64)
     assert_close_block(bf16_dev_to_f64(yd), ref, synth.bf16_to_f32(x).astype(np.float64))
@@ -375,6 +384,7 @@ def test_bounded_wait_runs_out_and_reports_timeout():
     y = torch.zeros_like(xd)
     ws.view(torch.int64)[32] = 1
     m.moe_set_wait_limit_ns(2_000_000)
+    m.moe_set_decode_path(m.DECODE_CHAIN)
     try:
         m.moe_timing_enable(True)
         m.moe_ffn_forward(d.L, xd, None, 1, y, ws, nb)
@@ -383,10 +393,11 @@ def test_bounded_wait_runs_out_and_reports_timeout():
     finally:
         m.moe_timing_enable(False)
         m.moe_set_wait_limit_ns(0)
+        m.moe_set_decode_path(m.DECODE_AUTO)
     assert "decode_chain" in kinds
     assert m.moe_get_device_status(ws) == 6
     m.moe_workspace_init(ws, nb)
-    yd, _, _, kinds = forward_with_record(m, d, xd, None, 1, ws, nb)
+    yd, _, _, kinds = forward_with_record(m, d, xd, None, 1, ws, nb, decode=m.DECODE_CHAIN)
     assert path_ran("chain", kinds)
     y_ref = oracle_layer(shape, t).ffn(x)[0]
     assert_close_output(bf16_dev_to_f64(yd), y_ref, "after a timeout")
@@ -498,15 +509,22 @@ def test_full_size_pack_bit_exact(full_layer):
             assert np.array_equal(got.ravel(), t[name + suf].ravel()), name + suf
 
 
-@pytest.mark.parametrize("K,T,path", [(4, 1, "chain"), (8, 1, "chain"), (4, 2, "chain"), (4, 3, "decode"),
-                                      (4, 6, None)])
-def test_full_size_decode(full_layer, K, T, path):
+@pytest.mark.parametrize("K,T,kernel,path", [(4, 1, "auto", "fused"), (4, 1, "chain", "chain"),
+                                             (8, 1, "auto", "chain"), (8, 1, "barrier", "fused"),
+                                             (4, 2, "auto", "fused"), (4, 2, "chain", "chain"),
+                                             (4, 3, "auto", "decode"), (4, 6, "auto", None)])
+def test_full_size_decode(full_layer, K, T, kernel, path):
+    """The Edge0 layer at decode sizes: the default choice between the two single-kernel
+    decodes (barrier kernel at top-4, chain kernel at top-8) and each one forced."""
+    m, _ = _mods()
     shape0, w, t = full_layer
     shape = dataclasses.replace(workloads.DECODE_K4, K=K)
     tt = dict(t)
     tt["logit_bias"] = None
     x, _ = workloads.moe_inputs(shape, seed=500 + K, T=T)
-    _check_ffn(shape, tt, x, None, n_adapters=1, what="decode K=%d T=%d" % (K, T), path=path)
+    force = {"auto": None, "chain": m.DECODE_CHAIN, "barrier": m.DECODE_BARRIER}[kernel]
+    _check_ffn(shape, tt, x, None, n_adapters=1, what="decode K=%d T=%d %s" % (K, T, kernel), path=path,
+               decode=force)
 
 
 @pytest.mark.parametrize("T", [4, 5, 8])
