@@ -238,7 +238,8 @@ def step_accounting(shape, idx, aid):
 # library timing kind -> accounting unit
 KIND_UNIT = {"router_logits": "router", "tc_router": "router", "gate_up": "gate_up", "tc_gate_up": "gate_up",
              "down": "down", "tc_down": "down", "lora_a": "lora_a", "tc_lora_gate_up": "lora_gu",
-             "tc_lora_down": "lora_down", "decode_fused": "layer", "decode_chain": "layer"}
+             "tc_lora_down": "lora_down", "decode_fused": "layer", "decode_chain": "layer",
+             "decode_cluster": "layer"}
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the

@@ -336,16 +336,19 @@ MOEQ_API moe_status moe_get_device_status(void* workspace, moe_stream stream, in
 MOEQ_API moe_status moe_ffn_routing(const moe_layer* layer, int32_t T, const void* workspace, size_t ws_bytes,
                                     int32_t* topk_idx, float* topk_w, moe_stream stream);
 
-/* Which single-kernel decode a forward of 1..8 tokens tries first.  AUTO: the barrier
- * kernel (two grid-wide barriers, every CTA takes the top-K itself) for top-4 or less
- * without a given expert set, the chain kernel (no grid barrier; CTA 0 routes and
- * publishes, every hand-off an epoch-tagged word or an arrival count) otherwise, as
- * measured faster for each; CHAIN or BARRIER: that kernel whenever it takes the call.
- * A call neither kernel takes runs on the multi-kernel paths.  Process-wide, read when
- * a call enqueues its kernels, not thread-safe. */
+/* Which single-kernel decode a forward of 1..8 tokens tries first.  AUTO: the cluster
+ * kernel for one token (thread-block clusters; router, top-K and LoRA-A products per
+ * cluster through distributed shared memory, one grid-wide exchange of h), else the
+ * barrier kernel (two grid-wide barriers, every CTA takes the top-K itself) for top-4 or
+ * less without a given expert set, else the chain kernel (no grid barrier; CTA 0 routes
+ * and publishes, every hand-off an epoch-tagged word or an arrival count); CHAIN,
+ * BARRIER or CLUSTER: that kernel whenever it takes the call.  A call no single kernel
+ * takes runs on the multi-kernel paths.  Process-wide, read when a call enqueues its
+ * kernels, not thread-safe. */
 #define MOE_DECODE_AUTO 0
 #define MOE_DECODE_CHAIN 1
 #define MOE_DECODE_BARRIER 2
+#define MOE_DECODE_CLUSTER 3
 MOEQ_API moe_status moe_set_decode_path(int path);
 MOEQ_API int moe_decode_path(void);
 

@@ -25,10 +25,10 @@ __all__ = [
     "moe_prerouter_workspace_bytes", "moe_prerouter_forward", "moe_act8_quant",
     "moe_mixed_linear_a8_workspace_bytes", "moe_mixed_linear_a8", "moe_mixed_mlp_a8_workspace_bytes",
     "moe_mixed_mlp_forward_a8", "moe_experts_workspace_bytes", "moe_experts_forward", "moe_ep_dispatch",
-    "moe_ep_combine", "moe_set_decode_path", "moe_decode_path", "DECODE_AUTO", "DECODE_CHAIN", "DECODE_BARRIER",
+    "moe_ep_combine", "moe_set_decode_path", "moe_decode_path", "DECODE_AUTO", "DECODE_CHAIN", "DECODE_BARRIER", "DECODE_CLUSTER",
 ]
 
-DECODE_AUTO, DECODE_CHAIN, DECODE_BARRIER = 0, 1, 2
+DECODE_AUTO, DECODE_CHAIN, DECODE_BARRIER, DECODE_CLUSTER = 0, 1, 2, 3
 
 
 class MoeError(RuntimeError):

@@ -126,6 +126,7 @@ WsPlan plan_of(const Dims& d) {
     // the chain decode kernel's tagged words: first after the header and sized for the
     // layer shape alone, so no other region of any T of this shape ever overlaps them
     p.slots = take(chain_slot_words(d.E, d.K, d.I, d.Is, d.r) * 8);
+    p.cslots = take(cluster_slot_words(d.K, d.I, d.Is) * 8);
     p.idx = take((size_t)d.T * d.K * 4);
     p.w = take((size_t)d.T * d.K * 4);
     p.sg = take((size_t)d.T * 4);
@@ -311,6 +312,15 @@ bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id
         cs.w_out = (float*)(b + p.w);
         return finish(launch_chain(la, x, adapter_id, select, y, T, block, eps, cs, s), kDecodeChain);
     };
+    auto run_cluster = [&]() {
+        if (!cluster_supported(la, T)) return false;
+        ClusterScratch cs;
+        cs.slots = (uint64_t*)(b + p.cslots);
+        cs.status = (int32_t*)(b + p.status);
+        cs.idx_out = (int32_t*)(b + p.idx);
+        cs.w_out = (float*)(b + p.w);
+        return finish(launch_cluster(la, x, adapter_id, select, y, T, block, eps, cs, s), kDecodeCluster);
+    };
     auto run_barrier = [&]() {  // (routes by top-K only)
         if (d.J > MOEQ_DECODE_MAX_JOBS || select || !decode_supported(la, T, nullptr)) return false;
         DecodeScratch sc;
@@ -328,8 +338,10 @@ bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id
     };
     if (g_decode_path == MOE_DECODE_CHAIN) return run_chain();
     if (g_decode_path == MOE_DECODE_BARRIER) return run_barrier();
+    if (g_decode_path == MOE_DECODE_CLUSTER) return run_cluster();
     // Measured on one B200 (one token, the Edge0 layer): top-4 34.6 us on the barrier
     // kernel against 37.2 on the chain kernel, top-8 48.3 against 45.9.
+    if (run_cluster()) return true;
     if (la.K <= 4) return run_barrier() || run_chain();
     return run_chain() || run_barrier();
 }
@@ -361,7 +373,8 @@ moe_status ffn_precheck(const moe_layer* layer, const uint16_t* x, const uint16_
 extern "C" {
 
 moe_status moe_set_decode_path(int path) {
-    CHECK_ARG(path == MOE_DECODE_AUTO || path == MOE_DECODE_CHAIN || path == MOE_DECODE_BARRIER);
+    CHECK_ARG(path == MOE_DECODE_AUTO || path == MOE_DECODE_CHAIN || path == MOE_DECODE_BARRIER ||
+              path == MOE_DECODE_CLUSTER);
     g_decode_path = path;
     return MOE_OK;
 }

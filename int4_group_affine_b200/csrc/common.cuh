@@ -89,6 +89,7 @@ struct WsPlan {
     size_t status, n_active, idx, w, sg, logits, gs, cnt, goff, active, perm, wperm, inv, tgu, td, h, ypart, xn, xp;
     size_t bar, dts, dtg, dtdp;  // fused decode scratch (sizes zero when T is too large for it)
     size_t slots;                // chain decode tagged words (right after the header, for every T)
+    size_t cslots;               // cluster decode ticket and tagged words (after the chain's)
     size_t total;
 };
 
@@ -143,7 +144,7 @@ struct DecodeScratch {
 enum Kind {
     kPack, kDequant, kRouter, kTopk, kIndexCount, kIndexScan, kIndexScatter, kLoraA, kGateUp, kDown,
     kCombine, kRmsnorm, kMixedGateUp, kMixedDown, kMixedLinear, kDecode, kTcLoraGUKind, kTcGUKind,
-    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kDecodeChain, kPrerouter, kAct8, kMixedA8, kEpDispatch, kEpCombine, kKindCount
+    kTcLoraDownKind, kTcDownKind, kTcRouterKind, kKpermKind, kDecodeChain, kPrerouter, kAct8, kMixedA8, kEpDispatch, kEpCombine, kDecodeCluster, kKindCount
 };
 void timing_begin(cudaStream_t s);
 void timing_mark(int kind, cudaStream_t s);
@@ -216,6 +217,20 @@ size_t chain_slot_words(int E, int K, int I, int Is, int r);
 bool chain_supported(const LayerArgs& L, int T);
 cudaError_t launch_chain(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, const int32_t* select,
                          uint16_t* y, int T, int block, float eps, const ChainScratch& sc, cudaStream_t s);
+
+// The cluster decode kernel (csrc/decode_cluster.cu): one token; the per-cluster steps
+// exchange through distributed shared memory, h through epoch-tagged words in a
+// workspace region of cluster_slot_words(...) words at a fixed place for a layer shape.
+struct ClusterScratch {
+    uint64_t* slots;           // ticket counter, spares, tagged h words (starts zeroed)
+    int32_t* status;
+    int32_t* idx_out;          // [K] routing record
+    float* w_out;
+};
+size_t cluster_slot_words(int K, int I, int Is);
+bool cluster_supported(const LayerArgs& L, int T);
+cudaError_t launch_cluster(const LayerArgs& L, const uint16_t* x, const int32_t* adapter_id, const int32_t* select,
+                           uint16_t* y, int T, int block, float eps, const ClusterScratch& sc, cudaStream_t s);
 
 // The prerouter head (csrc/prerouter.cu).
 size_t prerouter_workspace_bytes(const moe_prerouter& P, int T);

@@ -11,7 +11,7 @@ constexpr int kMaxRecords = 1 << 16;
 const char* const kNames[kKindCount] = {
     "pack", "dequant", "router_logits", "topk", "index_count", "index_scan", "index_scatter",
     "lora_a", "gate_up", "down", "combine", "rmsnorm", "mixed_gate_up", "mixed_down", "mixed_linear",
-    "decode_fused", "tc_lora_gate_up", "tc_gate_up", "tc_lora_down", "tc_down", "tc_router", "kperm", "decode_chain", "prerouter", "act8", "mixed_a8", "ep_dispatch", "ep_combine",
+    "decode_fused", "tc_lora_gate_up", "tc_gate_up", "tc_lora_down", "tc_down", "tc_router", "kperm", "decode_chain", "prerouter", "act8", "mixed_a8", "ep_dispatch", "ep_combine", "decode_cluster",
 };
 
 struct Rec {

@@ -137,15 +137,17 @@ def forward_with_record(m, d, xd, ad, T, ws, nb, block_eps=None, decode=None):
     return y, idx.cpu().numpy(), w.cpu().numpy(), kinds
 
 
-# kernel kinds that identify each execution path of the forward: "chain" and "fused" are
-# the two single-kernel decode paths (chain kernel, barrier kernel), "decode" either of them
-PATH_KINDS = {"chain": {"decode_chain"}, "fused": {"decode_fused"}, "cuda_core": {"gate_up", "down"},
+# kernel kinds that identify each execution path of the forward: "chain", "fused" and
+# "cluster" are the single-kernel decode paths (chain, barrier and cluster kernels),
+# "decode" any of them
+PATH_KINDS = {"chain": {"decode_chain"}, "fused": {"decode_fused"}, "cluster": {"decode_cluster"},
+              "cuda_core": {"gate_up", "down"},
               "tensor_core": {"tc_gate_up", "tc_down"}}
 
 
 def path_ran(path, kinds):
     if path == "decode":
-        return bool({"decode_chain", "decode_fused"} & kinds)
+        return bool({"decode_chain", "decode_fused", "decode_cluster"} & kinds)
     return PATH_KINDS[path] <= kinds
 
 

@@ -202,15 +202,15 @@ def test_wait_limit_setting():
 
 
 def test_decode_path_setting():
-    from int4_group_affine_b200 import (DECODE_AUTO, DECODE_BARRIER, DECODE_CHAIN, MoeError, moe_decode_path,
-                                        moe_set_decode_path)
+    from int4_group_affine_b200 import (DECODE_AUTO, DECODE_BARRIER, DECODE_CHAIN, DECODE_CLUSTER, MoeError,
+                                        moe_decode_path, moe_set_decode_path)
     assert moe_decode_path() == DECODE_AUTO
     try:
-        for p in (DECODE_CHAIN, DECODE_BARRIER, DECODE_AUTO):
+        for p in (DECODE_CHAIN, DECODE_BARRIER, DECODE_CLUSTER, DECODE_AUTO):
             moe_set_decode_path(p)
             assert moe_decode_path() == p
         with pytest.raises(MoeError) as ei:
-            moe_set_decode_path(3)
+            moe_set_decode_path(4)
         assert ei.value.status == 1
         assert moe_decode_path() == DECODE_AUTO
     finally:

@@ -33,8 +33,8 @@ def test_group_32_bytes():
 
 def test_every_single_kernel_decode_kind_has_a_unit():
     """The fused decode kernels are a whole layer call each: their bytes are the layer's."""
-    for kind in ("decode_fused", "decode_chain"):
+    for kind in ("decode_fused", "decode_chain", "decode_cluster"):
         assert bench.KIND_UNIT[kind] == "layer"
     from int4_group_affine_b200 import _lib
     names = {_lib.lib().moe_timing_kind_name(k).decode() for k in range(_lib.lib().moe_timing_kinds())}
-    assert {"decode_fused", "decode_chain", "tc_gate_up", "gate_up"} <= names
+    assert {"decode_fused", "decode_chain", "decode_cluster", "tc_gate_up", "gate_up"} <= names

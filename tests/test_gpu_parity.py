@@ -228,14 +228,18 @@ def _check_ffn(shape, t, x, aid, n_adapters=None, what="", path=None, decode=Non
 
 @pytest.mark.parametrize("T", [4, 1, 12, 37, 70])
 def test_ffn_tiny(T):
-    """Up to four tokens at top-2: the barrier decode kernel by default, then the chain
+    """One token: the cluster decode kernel by default, then the barrier and chain kernels
+    forced; up to four tokens at top-2: the barrier kernel by default, then the chain
     kernel forced; more tokens: the tensor-core path."""
     m, _ = _mods()
     shape = workloads.TINY
     t, x, aid = _ffn_case(shape, 400, T=T)
-    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T, path="fused" if T <= 4 else "tensor_core")
+    auto = "cluster" if T == 1 else "fused" if T <= 4 else "tensor_core"
+    _check_ffn(shape, t, x, aid, what="tiny T=%d" % T, path=auto)
     if T <= 4:
         _check_ffn(shape, t, x, aid, what="tiny T=%d chain" % T, path="chain", decode=m.DECODE_CHAIN)
+    if T == 1:
+        _check_ffn(shape, t, x, aid, what="tiny T=1 barrier", path="fused", decode=m.DECODE_BARRIER)
 
 
 @pytest.mark.parametrize("T", [5, 6])
@@ -264,12 +268,17 @@ def test_ffn_tiny_cuda_core_path(variant, T):
 @pytest.mark.parametrize("variant", ["k1", "kE", "no_lora", "no_shared", "no_sgate", "multi_adapter", "bias",
                                      "group32", "group32_decode", "rank24", "rank64", "k1_chain", "no_lora_chain",
                                      "no_shared_chain", "no_sgate_chain", "multi_adapter_chain", "bias_chain",
-                                     "rank24_chain"])
+                                     "rank24_chain", "k1_cluster", "kE_cluster", "no_lora_cluster",
+                                     "no_shared_cluster", "no_sgate_cluster", "multi_adapter_cluster", "bias_cluster",
+                                     "rank24_cluster", "group32_cluster"])
 def test_ffn_tiny_variants(variant):
-    """Layer variants on the tensor-core path (19 tokens) and, for the _chain ones, on the
-    chain decode kernel (3 tokens)."""
+    """Layer variants on the tensor-core path (19 tokens), for the _chain ones on the
+    chain decode kernel (3 tokens) and for the _cluster ones on the cluster decode kernel
+    (one token)."""
+    m, _ = _mods()
     chain = variant.endswith("_chain")
-    variant = variant[:-6] if chain else variant
+    cluster = variant.endswith("_cluster")
+    variant = variant[:-6] if chain else variant[:-8] if cluster else variant
     shape = workloads.TINY
     na = None
     if variant == "k1":
@@ -284,7 +293,7 @@ def test_ffn_tiny_variants(variant):
         shape = dataclasses.replace(shape, group=32)
     elif variant in ("rank24", "rank64"):  # LoRA-A products wider than one 32-column warp group
         shape = dataclasses.replace(shape, rank=int(variant[4:]), n_adapters=2, random_adapters=True)
-    t, x, aid = _ffn_case(shape, 410, T=3 if (variant == "group32_decode" or chain) else 19)
+    t, x, aid = _ffn_case(shape, 410, T=1 if cluster else 3 if (variant == "group32_decode" or chain) else 19)
     if variant in ("group32", "group32_decode"):
         w = workloads.moe_weights(shape, seed=410)
         t = quantize_layer(w, group=32)
@@ -300,10 +309,12 @@ def test_ffn_tiny_variants(variant):
     if variant == "multi_adapter":
         aid = aid.copy()
         aid[::5] = -1  # some tokens with the base only
-    m, _ = _mods()
-    _check_ffn(shape, t, x, aid, n_adapters=na, what=variant + (" (chain)" if chain else ""),
-               path="chain" if chain else ("decode" if variant == "group32_decode" else None),
-               decode=m.DECODE_CHAIN if chain else None)
+    if variant == "multi_adapter" and cluster:
+        aid = np.array([2], np.int32)  # (one token: an adapter other than the first)
+    _check_ffn(shape, t, x, aid, n_adapters=na,
+               what=variant + (" (chain)" if chain else " (cluster)" if cluster else ""),
+               path="chain" if chain else "cluster" if cluster else ("decode" if variant == "group32_decode" else None),
+               decode=m.DECODE_CHAIN if chain else m.DECODE_CLUSTER if cluster else None)
 
 
 def test_zero_B_equals_base_bitwise():
@@ -352,9 +363,9 @@ def test_bad_adapter_flags_status_and_falls_back_to_base():
     assert torch.equal(y, y2)
 
 
-@pytest.mark.parametrize("T", [3, 1])
-def test_block_tiny_chain(T):
-    """The pre-norm residual block on the chain decode kernel (RMSNorm inside it)."""
+@pytest.mark.parametrize("T,kernel", [(3, "chain"), (1, "chain"), (1, "cluster")])
+def test_block_tiny_single_kernel(T, kernel):
+    """The pre-norm residual block on the chain and cluster decode kernels (RMSNorm inside)."""
     m, ly = _mods()
     shape = workloads.TINY
     t, x, aid = _ffn_case(shape, 455, T=T)
@@ -362,8 +373,8 @@ def test_block_tiny_chain(T):
     d = ly.DeviceLayer.from_host(shape, t)
     ws, nb = d.workspace(T)
     yd, idx_g, _, kinds = forward_with_record(m, d, ly.to_device(x), None, T, ws, nb, block_eps=1e-6,
-                                              decode=m.DECODE_CHAIN)
-    assert path_ran("chain", kinds), kinds
+                                              decode=m.DECODE_CHAIN if kernel == "chain" else m.DECODE_CLUSTER)
+    assert path_ran(kernel, kinds), kinds
     ref = synth.bf16_to_f32(L.block(x, eps=1e-6)).astype(np.float64)
     assert_close_block(bf16_dev_to_f64(yd), ref, synth.bf16_to_f32(x).astype(np.float64))
 
@@ -399,6 +410,49 @@ def test_bounded_wait_runs_out_and_reports_timeout():
     m.moe_workspace_init(ws, nb)
     yd, _, _, kinds = forward_with_record(m, d, xd, None, 1, ws, nb, decode=m.DECODE_CHAIN)
     assert path_ran("chain", kinds)
+    y_ref = oracle_layer(shape, t).ffn(x)[0]
+    assert_close_output(bf16_dev_to_f64(yd), y_ref, "after a timeout")
+
+
+def _cluster_ticket_word(E, K, I, Is, r):
+    """Index (in 8-byte words) of the cluster decode kernel's ticket counter in a forward
+    workspace: the 256-byte header, then the chain kernel's region (its size formula), each
+    rounded up to 256 bytes."""
+    Tm = min(4, 16 // K)
+    rr, Jm, Imx = max(r, 1), Tm * (K + 1), max(I, Is)
+    chain = 8 + Tm * E + Tm * 2 * rr + Tm * K * 2 * rr + Tm * K + (Jm * Imx + 1) // 2 + (256 * 3 * Tm * rr + 1) // 2 + 2
+    return (256 + (chain * 8 + 255) // 256 * 256) // 8
+
+
+def test_bounded_wait_runs_out_on_the_cluster_kernel():
+    """The cluster kernel's grid-wide exchange of h gives up as the chain kernel's does: its
+    ticket counter set to 1 puts one CTA in another epoch, whose h words the others never
+    see (nor it theirs); every CTA still passes every cluster barrier, the call reports
+    MOE_ERR_TIMEOUT and the next call on a re-initialised workspace is correct."""
+    m, ly = _mods()
+    shape = workloads.TINY
+    t, x, aid = _ffn_case(shape, 475, T=1)
+    d = ly.DeviceLayer.from_host(shape, t)
+    ws, nb = d.workspace(1)
+    xd = ly.to_device(x)
+    y = torch.zeros_like(xd)
+    ws.view(torch.int64)[_cluster_ticket_word(shape.E, shape.K, shape.I, shape.Is, shape.rank)] = 1
+    m.moe_set_wait_limit_ns(2_000_000)
+    m.moe_set_decode_path(m.DECODE_CLUSTER)
+    try:
+        m.moe_timing_enable(True)
+        m.moe_ffn_forward(d.L, xd, None, 1, y, ws, nb)
+        torch.cuda.synchronize()
+        kinds = set(m.moe_timing_collect())
+    finally:
+        m.moe_timing_enable(False)
+        m.moe_set_wait_limit_ns(0)
+        m.moe_set_decode_path(m.DECODE_AUTO)
+    assert "decode_cluster" in kinds
+    assert m.moe_get_device_status(ws) == 6
+    m.moe_workspace_init(ws, nb)
+    yd, _, _, kinds = forward_with_record(m, d, xd, None, 1, ws, nb, decode=m.DECODE_CLUSTER)
+    assert path_ran("cluster", kinds)
     y_ref = oracle_layer(shape, t).ffn(x)[0]
     assert_close_output(bf16_dev_to_f64(yd), y_ref, "after a timeout")
 
@@ -509,20 +563,22 @@ def test_full_size_pack_bit_exact(full_layer):
             assert np.array_equal(got.ravel(), t[name + suf].ravel()), name + suf
 
 
-@pytest.mark.parametrize("K,T,kernel,path", [(4, 1, "auto", "fused"), (4, 1, "chain", "chain"),
-                                             (8, 1, "auto", "chain"), (8, 1, "barrier", "fused"),
+@pytest.mark.parametrize("K,T,kernel,path", [(4, 1, "auto", "cluster"), (4, 1, "chain", "chain"),
+                                             (4, 1, "barrier", "fused"), (8, 1, "auto", "decode"),
+                                             (8, 1, "chain", "chain"), (8, 1, "barrier", "fused"),
                                              (4, 2, "auto", "fused"), (4, 2, "chain", "chain"),
                                              (4, 3, "auto", "decode"), (4, 6, "auto", None)])
 def test_full_size_decode(full_layer, K, T, kernel, path):
-    """The Edge0 layer at decode sizes: the default choice between the two single-kernel
-    decodes (barrier kernel at top-4, chain kernel at top-8) and each one forced."""
+    """The Edge0 layer at decode sizes: the default choice among the single-kernel decodes
+    (cluster kernel for one token, barrier kernel for more at top-4, chain kernel at
+    top-8) and each one forced."""
     m, _ = _mods()
     shape0, w, t = full_layer
     shape = dataclasses.replace(workloads.DECODE_K4, K=K)
     tt = dict(t)
     tt["logit_bias"] = None
     x, _ = workloads.moe_inputs(shape, seed=500 + K, T=T)
-    force = {"auto": None, "chain": m.DECODE_CHAIN, "barrier": m.DECODE_BARRIER}[kernel]
+    force = {"auto": None, "chain": m.DECODE_CHAIN, "barrier": m.DECODE_BARRIER, "cluster": m.DECODE_CLUSTER}[kernel]
     _check_ffn(shape, tt, x, None, n_adapters=1, what="decode K=%d T=%d %s" % (K, T, kernel), path=path,
                decode=force)
 
@@ -586,7 +642,7 @@ def test_full_size_group32(full_layer, case):
         shape = dataclasses.replace(workloads.DECODE_K4, group=32)
         t["logit_bias"] = None
         x, aid = workloads.moe_inputs(shape, seed=520, T=1)
-        _check_ffn(shape, t, x, None, n_adapters=1, what="group 32 decode")
+        _check_ffn(shape, t, x, None, n_adapters=1, what="group 32 decode", path="decode")
     else:
         shape = dataclasses.replace(shape0, group=32)
         x, aid = workloads.moe_inputs(shape, seed=521)

@@ -122,7 +122,7 @@ def _select_forward(shape, t, x, aid, sel):
     return bf16_dev_to_f64(y), idx.cpu().numpy(), wts.cpu().numpy(), kinds, m.moe_get_device_status(ws)
 
 
-@pytest.mark.parametrize("T,path", [(1, "chain"), (2, "chain"), (3, None), (6, "cuda_core"), (20, "tensor_core")])
+@pytest.mark.parametrize("T,path", [(1, "cluster"), (2, "chain"), (3, None), (6, "cuda_core"), (20, "tensor_core")])
 def test_select_forward_every_path(layer, T, path):
     shape, t = layer
     x, aid = workloads.moe_inputs(shape, seed=720 + T, T=T)
@@ -170,5 +170,5 @@ def test_double_shift_prediction_is_the_routing(layer, head):
     pred_ref, _ = oracle.topk(z_ref, hs.K)
     check_routing(pred, pred_ref, z_ref, hs.K)
     y1, idx1, _, kinds, st1 = _select_forward(shape, tN1, x[2:3], aid[2:3], pred)
-    assert st1 == 0 and np.array_equal(idx1, pred) and path_ran("chain", kinds)
+    assert st1 == 0 and np.array_equal(idx1, pred) and path_ran("cluster", kinds)
     assert_close_output(y1, oracle_layer(shape, tN1).ffn(x[2:3], aid[2:3], select=pred)[0], "layer N+1 on the prediction")
