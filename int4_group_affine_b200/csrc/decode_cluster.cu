@@ -51,10 +51,15 @@ constexpr int kQMaxRA = 16;   // routed LoRA-A rows per CTA
 constexpr int kQMaxDA = 16;   // down LoRA-A rows per CTA
 constexpr int kQMaxCS = 16;   // CTAs per cluster
 constexpr int kQIssue = 5;    // warps 0..4 take the top-K and issue the routed rows' copies
+constexpr int kQMaxGT = 8;    // gate/up tiles (8 h elements each) per CTA
 
 struct QPlan {
     int CS, perA, perS, perO, perC, nSA, nRA, nDA, imx_sh;
     int gu_ns, gu_spg, gu_gsh;    // routed gate/up tensor-core tiles: K slices, groups per slice, log2(group / 32)
+    int lean;                     // 1: the routed LoRA-A rows reuse the phase-R windows (copied once the
+                                  // shared-expert rows are read) and the packed down rows reuse the
+                                  // gate/up windows (copied once the gate/up dots are done)
+    uint32_t dp, dp_stride;       // packed down rows of slot k at dp + k * dp_stride
     uint32_t xraw, xs, xsum, z, sa, ra, da;
     uint32_t wr, r_off[3];        // router rows p/s/b
     uint32_t wsg, sg_off[9];      // shared gate rows p/s/b, shared up rows p/s/b, the shared-gate row p/s/b
@@ -242,7 +247,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     float* hsum = reinterpret_cast<float*>(sm + P.hsum);
     float* sv = reinterpret_cast<float*>(sm + P.sv);    // [perO][K+1] per-expert outputs of the CTA's rows
 
-    __shared__ __align__(8) uint64_t s_bar[5];
+    __shared__ __align__(8) uint64_t s_bar[6];
     __shared__ int s_abort, s_aid;
     __shared__ uint32_t s_tag;
     __shared__ float s_inv, s_sig;
@@ -269,7 +274,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
         s_abort = 0;
         s_sig = 1.0f;
         s_inv = 1.0f;
-        for (int i = 0; i < 5; ++i) tc::mbar_init(&s_bar[i], (i == 3 || i == 4) ? 2u : 1u);
+        for (int i = 0; i < 6; ++i) tc::mbar_init(&s_bar[i], (i == 3 || i == 4) ? 2u : 1u);
         tc::mbar_init_fence();
     }
     __syncthreads();
@@ -470,6 +475,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
             if (lane < CS) dsm_st(sa + q * P.nSA + jj, lane, v);
         }
     }
+    if (P.lean && warp >= kQIssue) asm volatile("bar.arrive 2, %0;" ::"n"((kCW - kQIssue + 1) * 32) : "memory");
     cl_wait();  // the logits of the whole cluster are here
 
     // ------------------------------------------------------------ phase K
@@ -500,20 +506,21 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     if (warp < kQIssue) asm volatile("bar.sync 1, %0;" ::"n"(kQIssue * 32) : "memory");
     const int ad = s_aid;
     if (warp < 2) {
-        // routed gate (warp 0) | up (warp 1) rows: lane j < nrows copies the row of h element
-        // c_lo + j to its own slot (stride rrs); lanes 24.. copy the scales and biases of the
-        // two segments (rows of one expert each); warp 1 lanes 28.. the LoRA-B rows
+        // routed gate (warp 0) | up (warp 1) rows: lane j copies the rows of h elements c_lo + j,
+        // c_lo + j + 32, .. to their own slots (stride rrs); lanes 0..3 copy the scales and
+        // biases of the two segments (rows of one expert each); warp 1 lanes 4..7 the LoRA-B rows
         uint32_t tx = 0;
         const int pj = warp;
         const moe_qtensor& qt = pj ? L.up : L.gate;
         const int ng = H / qt.group;
-        if (lane < nrows) {
-            const int qq = c_lo + lane;
+        for (int j = lane; j < nrows; j += 32) {
+            const int qq = c_lo + j;
             const int64_t row = (int64_t)s_idx[qq / I] * I + qq % I;
-            winp(pol, sm + P.wc + P.c_off[3 * pj] + lane * P.rrs, s_abort ? nullptr : qt.packed + row * (H / 8),
+            winp(pol, sm + P.wc + P.c_off[3 * pj] + j * P.rrs, s_abort ? nullptr : qt.packed + row * (H / 8),
                  (uint32_t)(H / 2), &s_bar[3], &tx);
-        } else if (lane >= 24 && lane < 28) {
-            const int sgi = (lane - 24) / 2, k = 1 + (lane - 24) % 2, part = 3 * pj + k;
+        }
+        if (lane < 4) {  // scales | biases of the two segments: lane 2 s + (k - 1)
+            const int sgi = lane / 2, k = 1 + lane % 2, part = 3 * pj + k;
             const int q0 = sgi == 0 ? c_lo : cut, q1 = sgi == 0 ? cut : c_hi;
             const void* src = nullptr;
             uint32_t off = P.wc + P.c_off[part];
@@ -526,12 +533,12 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
                 }
             }
             s_cw[sgi][part] = winp(pol, sm + off, src, (uint32_t)(q1 - q0) * ng * 2, &s_bar[3], &tx);
-        } else if (pj == 1 && lane >= 28) {  // LoRA-B rows of the routed gate/up rows: lane 28 + 2 s + p
-            const int sgi = (lane - 28) / 2, pb = (lane - 28) % 2;
+        } else if (pj == 1 && lane < 8) {  // LoRA-B rows of the routed gate/up rows: lane 4 + 2 s + p
+            const int sgi = (lane - 4) / 2, pb = (lane - 4) % 2;
             const int q0 = sgi == 0 ? c_lo : cut, q1 = sgi == 0 ? cut : c_hi;
             const moe_lora_proj* lp = (lora && q1 > q0 && s_abort == 0) ? dlora(L, ad, false, pb) : nullptr;
             const int64_t row = q1 > q0 ? (int64_t)s_idx[q0 / I] * I + q0 % I : 0;
-            s_rbw[sgi][pb] = winp(pol, sm + P.wrb + (lane - 28) * P.rb_stride, lp ? lp->B + row * r : nullptr,
+            s_rbw[sgi][pb] = winp(pol, sm + P.wrb + (lane - 4) * P.rb_stride, lp ? lp->B + row * r : nullptr,
                                   (uint32_t)((q1 - q0) * r * 2), &s_bar[3], &tx);
         }
         tx = warp_total(tx);
@@ -549,7 +556,9 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
                                 : (const void*)((part == 1 ? L.down.scales : L.down.biases) + row * ngd);
                 bytes = part == 0 ? (uint32_t)(no * I / 2) : (uint32_t)(no * ngd * 2);
             }
-            s_dw[k][part] = winp(pol, sm + P.wd + k * P.d_stride + P.d_off[part], src, bytes, &s_bar[4], &tx);
+            if (part > 0 || !P.lean)
+                s_dw[k][part] = winp(pol, sm + (part == 0 ? P.dp + k * P.dp_stride : P.wd + k * P.d_stride + P.d_off[part]),
+                                     src, bytes, &s_bar[4], &tx);
         }
         if (lane < K) {
             const moe_lora_proj* lp = (lora && no > 0 && s_abort == 0) ? dlora(L, ad, false, 2) : nullptr;
@@ -560,6 +569,10 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
         tx = warp_total(tx);
         if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[4], tx);
     } else if (warp == 3) {  // routed LoRA-A rows: row d = q nRA + lane of [slot k][gate A | up A]
+        if (P.lean) {  // (their slots are the phase-R windows: wait for warps kQIssue.. to be done with them)
+            asm volatile("bar.sync 2, %0;" ::"n"((kCW - kQIssue + 1) * 32) : "memory");
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
         uint32_t tx = 0;
         if (lane < kQMaxRA) {
             const int d = q * P.nRA + lane, k = d / max(2 * r, 1), c = d % max(2 * r, 1);
@@ -632,6 +645,16 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     }
     cl_wait();  // the LoRA-A products of the whole cluster are here
     __syncthreads();
+    if (P.lean && warp == 2) {  // the packed down rows into the gate/up windows, read by now
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        uint32_t tx = 0;
+        if (lane < K && no > 0 && s_abort == 0)
+            s_dw[lane][0] = winp(pol, sm + P.dp + lane * P.dp_stride,
+                                 L.down.packed + ((int64_t)s_idx[lane] * H + o_lo) * (I / 8), (uint32_t)(no * I / 2),
+                                 &s_bar[5], &tx);
+        tx = warp_total(tx);
+        if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[5], tx);
+    }
     {
         // LoRA-B deltas, SwiGLU; h published: one element per thread (shared rows first, then
         // routed elements), each LoRA-B dot a thread's own loop over the rank
@@ -772,6 +795,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     cl_arrive();  // (the last stores into other CTAs)
     copies_landed(&s_bar[4], a.status, &s_abort, lim);
     copies_landed(&s_bar[1], a.status, &s_abort, lim);
+    if (P.lean) copies_landed(&s_bar[5], a.status, &s_abort, lim);
     if (no > 0 && s_abort == 0) {
         // (output row, expert) tasks: lpt lanes over one row
         int lpt = 1;
@@ -829,7 +853,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     }
     // no bulk copy may be in flight when the CTA exits (bounded waits)
     if (tid == 0)
-        for (int i = 0; i < 5; ++i) tc::mbar_wait(&s_bar[i], 0, nullptr, lim);
+        for (int i = 0; i < (P.lean ? 6 : 5); ++i) tc::mbar_wait(&s_bar[i], 0, nullptr, lim);
 }
 
 }  // namespace
@@ -866,7 +890,7 @@ size_t q_static_smem() {
     return v;
 }
 
-bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P) {
+bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P, bool lean) {
     const bool sh = L.has_shared, lora = L.n_adapters > 0 && L.rank > 0;
     const int H = L.H, E = L.E, K = L.K, I = L.I, Is = sh ? L.Is : 0, r = lora ? L.rank : 0;
     const int Imx = std::max(I, Is), KS = K + (sh ? 1 : 0);
@@ -890,6 +914,7 @@ bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P) {
     }
     if (Imx & (Imx - 1)) return false;  // (h is gathered over a [K+1][Imx] layout by shifts)
     P->CS = CS;
+    P->lean = lean ? 1 : 0;
     P->imx_sh = 0;
     while ((1 << P->imx_sh) < Imx) ++P->imx_sh;
     P->perA = cdivq(E, CS);
@@ -899,7 +924,8 @@ bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P) {
     P->nSA = (lora && sh) ? cdivq(2 * r, CS) : 0;
     P->nRA = lora ? cdivq(K * 2 * r, CS) : 0;
     P->nDA = lora ? cdivq(KS * r, CS) : 0;
-    if (P->perO > kQMaxO || P->perC > I || P->perC > 24 || P->nSA > kQMaxSA || P->nRA > kQMaxRA || P->nDA > kQMaxDA)
+    if (P->perO > kQMaxO || P->perC > I || P->perC > 8 * kQMaxGT || P->nSA > kQMaxSA || P->nRA > kQMaxRA ||
+        P->nDA > kQMaxDA)
         return false;
     // the gate/up tiles: one group size for gate and up, 32, 64 or 128
     if (L.gate.group != L.up.group || (L.gate.group != 32 && L.gate.group != 64 && L.gate.group != 128)) return false;
@@ -944,10 +970,11 @@ bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P) {
                 wsz += L.has_sgate ? slack(gsz[k]) : 0;
             }
         }
-        P->wr = take(wsz);
-        P->wsg = P->wr;
         P->ra_stride = (uint32_t)slack((size_t)H * 2);
-        P->wra = take((size_t)P->nRA * P->ra_stride);
+        const size_t rasz = (size_t)P->nRA * P->ra_stride;
+        P->wr = take(lean ? std::max(wsz, rasz) : wsz);
+        P->wsg = P->wr;
+        P->wra = lean ? P->wr : take(rasz);
     }
     {
         const int ngd = sh ? Is / L.s_down.group : 0;
@@ -974,18 +1001,21 @@ bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P) {
             P->c_off[k] = (uint32_t)wsz;
             wsz += r16q(cpart[k]) + 64;
         }
-        const size_t hbytes = r16q((size_t)KS * Imx * 4), hsbytes = (size_t)KS * (Imx / 32) * 4;
-        P->wc = take(std::max(wsz, hbytes + hsbytes));
+        const size_t hbytes = r16q((size_t)KS * Imx * 4), hsbytes = r16q((size_t)KS * (Imx / 32) * 4);
+        P->dp_stride = (uint32_t)slack((size_t)P->perO * I / 2);
+        const size_t dpbytes = (size_t)K * P->dp_stride;
+        P->wc = take(std::max(wsz, hbytes + hsbytes + (lean ? dpbytes : 0)));
         P->hs = P->wc;
         P->hsum = P->wc + (uint32_t)hbytes;
+        P->dp = lean ? P->wc + (uint32_t)(hbytes + hsbytes) : take(dpbytes);
     }
     P->rb_stride = (uint32_t)slack((size_t)P->perC * std::max(r, 1) * 2);
     P->wrb = take(lora ? (size_t)4 * P->rb_stride : 0);
     {
-        const int ngd = I / L.down.group;
+        const int ngd = I / L.down.group;  // (scales and biases of slot k; its packed rows at dp)
         P->d_off[0] = 0;
-        P->d_off[1] = (uint32_t)slack((size_t)P->perO * I / 2);
-        P->d_off[2] = P->d_off[1] + (uint32_t)slack((size_t)P->perO * ngd * 2);
+        P->d_off[1] = 0;
+        P->d_off[2] = (uint32_t)slack((size_t)P->perO * ngd * 2);
         P->d_stride = P->d_off[2] + (uint32_t)slack((size_t)P->perO * ngd * 2);
         P->wd = take((size_t)K * P->d_stride);
     }
@@ -1060,7 +1090,9 @@ const QShape* q_shapes() {
 const QShape* q_pick(const LayerArgs& L, int T, QPlan* P) {
     const QShape* s = q_shapes();
     for (int i = 0; i < kQShapes; ++i)
-        if (s[i].NC >= 4 && plan_cluster(L, T, s[i].CS, s[i].CS * s[i].NC, P)) return &s[i];
+        if (s[i].NC >= 4 && (plan_cluster(L, T, s[i].CS, s[i].CS * s[i].NC, P, false) ||
+                             plan_cluster(L, T, s[i].CS, s[i].CS * s[i].NC, P, true)))
+            return &s[i];
     return nullptr;
 }
 

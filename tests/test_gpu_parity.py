@@ -564,14 +564,15 @@ def test_full_size_pack_bit_exact(full_layer):
 
 
 @pytest.mark.parametrize("K,T,kernel,path", [(4, 1, "auto", "cluster"), (4, 1, "chain", "chain"),
-                                             (4, 1, "barrier", "fused"), (8, 1, "auto", "decode"),
+                                             (4, 1, "barrier", "fused"), (8, 1, "auto", "cluster"),
+                                             (8, 1, "cluster", "cluster"),
                                              (8, 1, "chain", "chain"), (8, 1, "barrier", "fused"),
                                              (4, 2, "auto", "fused"), (4, 2, "chain", "chain"),
                                              (4, 3, "auto", "decode"), (4, 6, "auto", None)])
 def test_full_size_decode(full_layer, K, T, kernel, path):
     """The Edge0 layer at decode sizes: the default choice among the single-kernel decodes
-    (cluster kernel for one token, barrier kernel for more at top-4, chain kernel at
-    top-8) and each one forced."""
+    (cluster kernel for one token — at top-8 in its lean shared-memory layout —, barrier
+    kernel for more at top-4) and each one forced."""
     m, _ = _mods()
     shape0, w, t = full_layer
     shape = dataclasses.replace(workloads.DECODE_K4, K=K)
