@@ -52,6 +52,7 @@ constexpr int kQMaxDA = 16;   // down LoRA-A rows per CTA
 constexpr int kQMaxCS = 16;   // CTAs per cluster
 constexpr int kQIssue = 5;    // warps 0..4 take the top-K and issue the routed rows' copies
 constexpr int kQMaxGT = 8;    // gate/up tiles (8 h elements each) per CTA
+constexpr int kQGW = 12;      // h words per thread in the gather ((K+1) max(I, Is) <= 12 * 512)
 
 struct QPlan {
     int CS, perA, perS, perO, perC, nSA, nRA, nDA, imx_sh;
@@ -731,8 +732,18 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     // by now (the __syncthreads above): hs and hsum reuse them.
     {
         const uint32_t tag = s_tag;
-        // warp 0 waits for the ready words of all CTAs (one poll stream per CTA instead of
-        // one per h word), then every thread reads its h words once
+        // every thread reads its h words once at once (most are published by now), warp 0
+        // waits for the ready words of all CTAs (one poll stream per CTA instead of one per h
+        // word), then the words that were not yet published are read again.  Element i of the
+        // [K+1][Imx] layout: slot i >> imx_sh, place i & (Imx - 1); the places past a slot's
+        // length (Is < I or I < Is) are skipped.
+        const int nh = KS * Imx, Ish = P.imx_sh;
+        unsigned long long w[kQGW];
+#pragma unroll
+        for (int b = 0; b < kQGW; ++b) {
+            const int i = b * kCT + tid, slot = i >> Ish, e = i & (Imx - 1);
+            w[b] = (i < nh && e < (slot < K ? I : Is)) ? peek(a.hg + i) : 0ull;
+        }
         if (warp == 0) {
             uint32_t pend = 0;  // lane's ready words (CTAs lane + 32 m) without this launch's tag
             for (int m = 0; m < (NB + 31) / 32; ++m)
@@ -753,32 +764,25 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
                     }
                     pend = 0;
                 }
-                if (pend) __nanosleep(64);
+                if (pend) __nanosleep(32);
             }
         }
         __syncthreads();
-        // element i of the [K+1][Imx] layout: slot i >> imx_sh, place i & (Imx - 1); the
-        // places past a slot's length (Is < I or I < Is) are skipped
-        const int nh = KS * Imx, Ish = P.imx_sh;
-        for (int base = 0; base < nh; base += kGB * kCT) {
-            unsigned long long w[kGB];
 #pragma unroll
-            for (int b = 0; b < kGB; ++b) {
-                const int i = base + b * kCT + tid, slot = i >> Ish, e = i & (Imx - 1);
-                const bool live = i < nh && e < (slot < K ? I : Is);
-                w[b] = live ? peek(a.hg + i) : 0ull;
-            }
-            // (a warp's 32 elements of a pass are one 32-element chunk of one slot: I and Is
-            // are multiples of 32, so its chunk sum is one warp reduction)
+        for (int b = 0; b < kQGW; ++b) {
+            const int i = b * kCT + tid, slot = i >> Ish, e = i & (Imx - 1);
+            if (i < nh && e < (slot < K ? I : Is) && !fresh(w[b], tag)) w[b] = peek(a.hg + i);
+        }
+        // (a warp's 32 elements of a pass are one 32-element chunk of one slot: I and Is are
+        // multiples of 32, so its chunk sum is one warp reduction)
 #pragma unroll
-            for (int b = 0; b < kGB; ++b) {
-                const int i = base + b * kCT + tid, slot = i >> Ish, e = i & (Imx - 1);
-                if (i - lane >= nh || e - lane >= (slot < K ? I : Is)) continue;  // (uniform across the warp)
-                const float v = fresh(w[b], tag) ? wval(w[b]) : 0.0f;
-                hs[slot * Imx + swz(e)] = v;
-                const float cs = warp_sum(v);
-                if (lane == 0) hsum[slot * (Imx / 32) + (e >> 5)] = cs;
-            }
+        for (int b = 0; b < kQGW; ++b) {
+            const int i = b * kCT + tid, slot = i >> Ish, e = i & (Imx - 1);
+            if (i - lane >= nh || e - lane >= (slot < K ? I : Is)) continue;  // (uniform across the warp)
+            const float v = fresh(w[b], tag) ? wval(w[b]) : 0.0f;
+            hs[slot * Imx + swz(e)] = v;
+            const float cs = warp_sum(v);
+            if (lane == 0) hsum[slot * (Imx / 32) + (e >> 5)] = cs;
         }
         __syncthreads();
     }
@@ -912,7 +916,7 @@ bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P, bool lean
                 if ((p[k]->A && ((uintptr_t)p[k]->A & 15)) || (p[k]->B && ((uintptr_t)p[k]->B & 15))) return false;
         }
     }
-    if (Imx & (Imx - 1)) return false;  // (h is gathered over a [K+1][Imx] layout by shifts)
+    if (Imx & (Imx - 1) || KS * Imx > kQGW * kCT) return false;  // (h gathered over [K+1][Imx] by shifts)
     P->CS = CS;
     P->lean = lean ? 1 : 0;
     P->imx_sh = 0;
