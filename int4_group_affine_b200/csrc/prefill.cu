@@ -46,7 +46,7 @@
 //            into one accumulator, so the logits carry ~16 bits of each weight;
 //            epilogue adds the logit bias -> logits.
 //
-// Warp roles: 8 dequantisation warps (scales, dequant, LoRA-B operand, epilogue),
+// Warp roles: 8 dequantisation warps (16 in down mode: TcWarps) (scales, dequant, LoRA-B operand, epilogue),
 // one MMA warp and one loader warp (weight spans, activations, LoRA-B rows); they
 // hand steps over through mbarriers, so no CTA-wide barrier sits in the K loop.
 // Every wait is bounded in time and raises MOE_ERR_TIMEOUT when it gives up.
@@ -58,10 +58,6 @@
 namespace moeq {
 namespace {
 
-constexpr int kDeqWarps = 8;                      // dequantisation warps
-constexpr int kMmaWarp = kDeqWarps;               // MMA issue
-constexpr int kLoadWarp = kDeqWarps + 1;          // TMA spans, activation rows, LoRA rows
-constexpr int kTcThreads = (kDeqWarps + 2) * 32;
 constexpr int kBM = 128;                          // rows per MMA block
 constexpr int kNT = 64;                           // jobs per tile (MMA N <= 64)
 constexpr int kKS = 128;                          // K per pipeline step (two 64-wide operand sub-tiles)
@@ -80,6 +76,16 @@ constexpr uint32_t kTmemA = 256;
 static_assert(kTmemA + kAS * 128 <= 512, "TMEM columns");
 
 enum Mode { kGU = 0, kDown = 1, kRouterMode = 4 };
+
+// Dequantisation warps per mode: 16 for down (two threads per weight row, each half of a
+// step's words: measured 174 against 192 us per prefill layer), 8 elsewhere (gate/up ran
+// 318 against 268 us with 16: the step's TMEM stores and the per-thread state of the
+// LoRA-B operand then outweigh the shorter dequantisation chains).
+template <int kMode>
+struct TcWarps {
+    static constexpr int deq = kMode == kDown ? 16 : 8;
+    static constexpr int threads = (deq + 2) * 32;
+};
 
 struct TcArgs {
     CUtensorMap tm[4];    // weight words: gate/up {gate, up, s_gate, s_up}; down {down, s_down}; router {router}
@@ -210,14 +216,21 @@ struct BCtx {
     bool live[2];
 };
 
-// LoRA-B operand B of one step, fetched a step ahead: rows brow, brow + 32; chunk bch; sub-tiles 0, 1
+// LoRA-B operand B of one step, fetched a step ahead: the thread's job rows, chunk bch,
+// sub-tiles 0, 1
+template <int LJ>
 struct LoraRegs {
-    float4 t[2][2][2];  // [row][sub-tile][half], unscaled LoRA-A products
-    uint32_t live;      // bit (2 row + sub)
+    float4 t[LJ][2][2];  // [row][sub-tile][half], unscaled LoRA-A products
+    uint32_t live;       // bit (2 row + sub)
 };
 
 template <int kMode>
-__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcArgs a) {
+__global__ void __launch_bounds__(TcWarps<kMode>::threads, 1) tc_gemm_kernel(const __grid_constant__ TcArgs a) {
+    // warp roles of this mode: dequantisation warps, then the MMA warp and the loader warp
+    constexpr int kDeqW = TcWarps<kMode>::deq, kMmaW = kDeqW, kLoadW = kDeqW + 1, kThreads = TcWarps<kMode>::threads;
+    constexpr int NQ = kDeqW / 8;               // threads per (block, weight row)
+    constexpr int kLRows = kDeqW * 32 / 8;      // distinct LoRA-B operand job rows over the dequantisation threads
+    constexpr int kLJ = kNT / kLRows;           // job rows per thread
     extern __shared__ __align__(1024) unsigned char tsm_raw[];
     // 128-byte-swizzled tiles need 1024-byte aligned bases: align by hand (the
     // launch requests 1 KB of slack).
@@ -257,19 +270,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             s_goff[1] = a.T;
         }
     } else {
-        for (int g = tid; g <= ngroups; g += kTcThreads) s_goff[g] = a.goff[g];
+        for (int g = tid; g <= ngroups; g += kThreads) s_goff[g] = a.goff[g];
     }
-    if (warp == kMmaWarp) {
+    if (warp == kMmaW) {
         tc::tmem_alloc(&s_tmem, 512);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < kAS; ++i) tc::mbar_init(&bar_full[i], kDeqWarps);
+        for (int i = 0; i < kAS; ++i) tc::mbar_init(&bar_full[i], kDeqW);
         for (int i = 0; i < kRB; ++i) tc::mbar_init(&bar_bfull[i], 32);
         for (int i = 0; i < kTiles; ++i) tc::mbar_init(&bar_tile[i], 1);
         for (int i = 0; i < kRS; ++i) {
             tc::mbar_init(&bar_raw[i], 32);
-            tc::mbar_init(&bar_rawfree[i], kDeqWarps);
+            tc::mbar_init(&bar_rawfree[i], kDeqW);
         }
         tc::mbar_init(&bar_acc[0], 1);
         tc::mbar_init(&bar_acc[1], 1);
@@ -323,7 +336,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         if (++p.kt == p.KT) decode(p.item + NB, p);
     };
 
-    if (warp == kLoadWarp) {
+    if (warp == kLoadW) {
         // ====================================================== loader warp: TMA spans, activation rows,
         // LoRA-B rows.  It runs ahead of the MMAs by up to kRB steps (activation slots) and of the
         // dequantisation by up to kRS spans (weight ring).
@@ -467,7 +480,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (!ok) s_ok = 0;
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaW) {
         // ====================================================== MMA warp: lane 0 alone, so that
         // between two steps it does little more than wait and issue
         if (lane == 0) {
@@ -538,9 +551,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         // ---- weight rows.  int4: thread -> (block, row): the step's 16 words of the row;
         //      int8: thread -> (row, half of the step's 32 words).  Warp w writes TMEM
         //      lanes 32 (w % 4) .. +31, which are its rows.
+        static_assert(NQ == 1 || !int8_mode, "the int8 path takes one thread per (row, half)");
         const int wrow = tid % kBM;
-        const int wblk = int8_mode ? 0 : tid / kBM;
-        const int wh = tid / kBM;  // int8: half
+        const int wblk = int8_mode ? 0 : (tid / kBM) % 2;
+        const int wh = tid / kBM;       // int8: half
+        const int whs = NQ == 1 ? 0 : tid / (2 * kBM);  // int4: part of the step's chunks (of NQ)
         const uint32_t tlane = (uint32_t)((warp % 4) * 32) << 16;
         const int group = int8_mode ? L.router.group : L.gate.group;
         const int gshift = group == 64 ? 6 : 5;
@@ -577,16 +592,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         // sub-tiles): sub-tile k holds, for block k's matrix (gate/up: gate, up; down: down in
         // sub-tile 0), each job's scaled LoRA-A products in its adapter's K' columns
         const int brow = tid / 8, bch = tid % 8;
-        const uint32_t boff0 = tc::sw128_off(brow, bch), boff1 = tc::sw128_off(brow + 32, bch);
-        auto fetch_lora = [&](const Pos& p, int s, LoraRegs& R) {
+        const uint32_t boff0 = tc::sw128_off(brow, bch), boff1 = tc::sw128_off(brow + kLRows, bch);
+        auto fetch_lora = [&](const Pos& p, int s, LoraRegs<kLJ>& R) {
             const Geo q = geo(p);
             const int base = s_goff[p.g] + p.nt * kNT, end = s_goff[p.g + 1];
             const int cc = 64 * s + 8 * bch;
             const int tw = mode == kGU ? 2 * r : r;
             R.live = 0;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int job = base + brow + 32 * j;
+            for (int j = 0; j < kLJ; ++j) {
+                const int job = base + brow + kLRows * j;
                 if (job >= end || cc >= nar) continue;
                 const int ad = a.perm[job].z;
                 if (ad != cc / r) continue;
@@ -601,10 +616,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
             }
         };
-        auto stage_lora = [&](const LoraRegs& R, unsigned char* bslot) {
+        auto stage_lora = [&](const LoraRegs<kLJ>& R, unsigned char* bslot) {
             const float sc = L.scale;
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+            for (int j = 0; j < kLJ; ++j)
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {
                     if (mode == kDown && sub == 1) continue;
@@ -631,7 +646,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const int base = s_goff[p.g] + p.nt * kNT;
             const uint32_t dacc = tmem + tlane + (seq & 1u) * 128u;
             const int row = (warp % 4) * 32 + lane;  // TMEM lane of this thread
-            for (int ch = warp / 4; ch * 16 < n_here; ch += 2) {  // 16-column chunks
+            for (int ch = warp / 4; ch * 16 < n_here; ch += kDeqW / 4) {  // 16-column chunks
                 uint32_t d0[16], d1[16];
                 tc::tmem_ld16(dacc + ch * 16, d0);
                 if (int4_mode) tc::tmem_ld16(dacc + 64 + ch * 16, d1);
@@ -694,7 +709,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         };
         sb_next();
         uint32_t ss0[4] = {0, 0, 0, 0}, sb0[4] = {0, 0, 0, 0}, ss1[4] = {0, 0, 0, 0}, sb1[4] = {0, 0, 0, 0};
-        LoraRegs lr;
+        LoraRegs<kLJ> lr;
         // the epilogue of an item runs kAS steps after its last step, when its MMAs are done
         bool ep_pend = false;
         Pos ep_pos = pc;
@@ -745,17 +760,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (int4_mode && wstep) {
                 // the step's 16 words = 16-byte chunks 4kk .. 4kk+3 of the swizzled 128-byte row;
                 // word w = K elements 8w .. 8w+7 = TMEM columns 4w .. 4w+3 of this block
+                constexpr int CPT = 4 / NQ;  // chunks of the step's 4 per thread
                 const unsigned char* rowp = sR + (sseq % kRS) * kRawSlot + wblk * kSpanBytes + wrow * 128;
-                const uint32_t ta = astage + wblk * 64;
-                // all four chunks are read before any TMEM store (the stores are compiler
-                // barriers), so the 16 dequantisation chains overlap
-                uint4 w4[4];
+                const uint32_t ta = astage + wblk * 64 + whs * 16 * CPT;
+                // all the thread's chunks are read before any TMEM store (the stores are compiler
+                // barriers), so the dequantisation chains overlap
+                uint4 w4[CPT];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) w4[c] = *reinterpret_cast<const uint4*>(rowp + (((4 * kk + c) ^ (wrow & 7)) << 4));
-                uint32_t v[64];
+                for (int c = 0; c < CPT; ++c)
+                    w4[c] = *reinterpret_cast<const uint4*>(rowp + (((4 * kk + whs * CPT + c) ^ (wrow & 7)) << 4));
+                uint32_t v[16 * CPT];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const __nv_bfloat162 s2 = bf16x2_of(kk ? ss1[c] : ss0[c]), b2 = bf16x2_of(kk ? sb1[c] : sb0[c]);
+                for (int c = 0; c < CPT; ++c) {
+                    const int cc = whs * CPT + c;
+                    const __nv_bfloat162 s2 = bf16x2_of(kk ? ss1[cc] : ss0[cc]), b2 = bf16x2_of(kk ? sb1[cc] : sb0[cc]);
                     const uint4 o0 = dequant8p(w4[c].x, s2, b2), o1 = dequant8p(w4[c].y, s2, b2);
                     const uint4 o2 = dequant8p(w4[c].z, s2, b2), o3 = dequant8p(w4[c].w, s2, b2);
                     uint32_t* vc = v + 16 * c;
@@ -764,8 +782,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     vc[8] = o2.x; vc[9] = o2.y; vc[10] = o2.z; vc[11] = o2.w;
                     vc[12] = o3.x; vc[13] = o3.y; vc[14] = o3.z; vc[15] = o3.w;
                 }
-                tc::tmem_st32(ta, v);
-                tc::tmem_st32(ta + 32, v + 32);
+#pragma unroll
+                for (int i = 0; i < CPT / 2; ++i) tc::tmem_st32(ta + 32 * i, v + 32 * i);
                 tc::tmem_wait_st();
             } else if (int4_mode) {
                 stage_lora(lr, sB + (t % kRB) * kBSlot);
@@ -831,7 +849,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     }
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) tc::tmem_dealloc(tmem, 512);
+    if (warp == kMmaW) tc::tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------ host side
@@ -891,7 +909,7 @@ cudaError_t launch_mode(TcArgs& a, int nsm, cudaStream_t s) {
     const size_t smem = kRB * kBSlot + kRS * kRawSlot + 1024;
     cudaError_t e = ensure_smem((const void*)tc_gemm_kernel<kMode>, smem, cached);
     if (e != cudaSuccess) return e;
-    tc_gemm_kernel<kMode><<<nsm, kTcThreads, smem, s>>>(a);
+    tc_gemm_kernel<kMode><<<nsm, TcWarps<kMode>::threads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
