@@ -227,6 +227,20 @@ MOEQ_API moe_status moe_workspace_init(void* workspace, size_t ws_bytes, moe_str
 MOEQ_API moe_status moe_ffn_forward(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id, int32_t T,
                            uint16_t* y, void* workspace, size_t ws_bytes, moe_stream stream);
 
+/* The forward of moe_ffn_forward for a decode-sized call (1 to 8 tokens) whose input x and
+ * output y ([T][hidden] bf16, 16-byte aligned) are in page-locked host memory mapped into the
+ * device's address space (cudaHostAlloc / cudaMallocHost memory on a 64-bit system with
+ * unified addressing, or memory registered with cudaHostRegisterMapped).  The transfers are
+ * part of the call, on `stream`: with one token the cluster decode kernel reads x and writes y
+ * across the bus itself; otherwise x is copied into the workspace, the forward runs there and y
+ * is copied back.  adapter_id, if given, is device memory.  The workspace is
+ * moe_ffn_workspace_bytes(layer, T) bytes.  Errors: those of moe_ffn_forward;
+ * MOE_ERR_UNSUPPORTED for T above 8; MOE_ERR_INVALID_ARG when x or y is not mapped host
+ * memory.  Nothing is enqueued on an error. */
+MOEQ_API moe_status moe_ffn_forward_host(const moe_layer* layer, const uint16_t* x_host, const int32_t* adapter_id,
+                                         int32_t T, uint16_t* y_host, void* workspace, size_t ws_bytes,
+                                         moe_stream stream);
+
 /* ------------------------------------------ forward without device allocation
  * No counterpart on the pages: this entry point exists for callers that cannot
  * allocate device memory at the point where they run the layer (an engine's

@@ -25,7 +25,7 @@ __all__ = [
     "moe_prerouter_workspace_bytes", "moe_prerouter_forward", "moe_act8_quant",
     "moe_mixed_linear_a8_workspace_bytes", "moe_mixed_linear_a8", "moe_mixed_mlp_a8_workspace_bytes",
     "moe_mixed_mlp_forward_a8", "moe_experts_workspace_bytes", "moe_experts_forward", "moe_ep_dispatch",
-    "moe_ep_combine", "moe_set_decode_path", "moe_decode_path", "DECODE_AUTO", "DECODE_CHAIN", "DECODE_BARRIER", "DECODE_CLUSTER",
+    "moe_ep_combine", "moe_ffn_forward_host", "moe_set_decode_path", "moe_decode_path", "DECODE_AUTO", "DECODE_CHAIN", "DECODE_BARRIER", "DECODE_CLUSTER",
 ]
 
 DECODE_AUTO, DECODE_CHAIN, DECODE_BARRIER, DECODE_CLUSTER = 0, 1, 2, 3
@@ -124,6 +124,25 @@ def moe_workspace_init(workspace, ws_bytes, stream=None):
 def moe_ffn_forward(layer: Layer, x, adapter_id, T, y, workspace, ws_bytes, stream=None):
     _check("moe_ffn_forward", _lib.lib().moe_ffn_forward(ctypes.byref(layer), _ptr(x), _ptr(adapter_id), T,
                                                          _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def _hptr(t):
+    """Address of a page-locked host tensor (or a raw address)."""
+    if isinstance(t, int):
+        return t
+    if t.is_cuda or not t.is_pinned():
+        raise ValueError("expected a pinned host tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def moe_ffn_forward_host(layer: Layer, x_host, adapter_id, T, y_host, workspace, ws_bytes, stream=None):
+    """moe_ffn_forward with x and y in mapped page-locked host memory (pinned torch tensors or
+    raw host addresses); 1 to 8 tokens."""
+    _check("moe_ffn_forward_host", _lib.lib().moe_ffn_forward_host(ctypes.byref(layer), _hptr(x_host),
+                                                                   _ptr(adapter_id), T, _hptr(y_host),
+                                                                   _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def moe_block_forward(layer: Layer, x, adapter_id, T, eps, x_out, workspace, ws_bytes, stream=None):

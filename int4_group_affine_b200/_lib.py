@@ -69,6 +69,7 @@ SIGNATURES = {
     "moe_ffn_workspace_bytes": (SZ, [PL, I32]),
     "moe_workspace_init": (ctypes.c_int, [P, SZ, P]),
     "moe_ffn_forward": (ctypes.c_int, [PL, P, P, I32, P, P, SZ, P]),
+    "moe_ffn_forward_host": (ctypes.c_int, [PL, P, P, I32, P, P, SZ, P]),
     "moe_ffn_forward_static": (ctypes.c_int, [PL, P, P, I32, P, P]),
     "moe_block_forward": (ctypes.c_int, [PL, P, P, I32, F32, P, P, SZ, P]),
     "moe_rmsnorm": (ctypes.c_int, [P, I32, I32, F32, P, P]),

@@ -127,6 +127,8 @@ WsPlan plan_of(const Dims& d) {
     // layer shape alone, so no other region of any T of this shape ever overlaps them
     p.slots = take(chain_slot_words(d.E, d.K, d.I, d.Is, d.r) * 8);
     p.cslots = take(cluster_slot_words(d.K, d.I, d.Is) * 8);
+    p.hxin = take(d.T <= MOEQ_DECODE_MAX_TOKENS ? (size_t)d.T * d.H * 2 : 0);
+    p.hyout = take(d.T <= MOEQ_DECODE_MAX_TOKENS ? (size_t)d.T * d.H * 2 : 0);
     p.idx = take((size_t)d.T * d.K * 4);
     p.w = take((size_t)d.T * d.K * 4);
     p.sg = take((size_t)d.T * 4);
@@ -316,6 +318,7 @@ bool try_decode(const moe_layer* L, const uint16_t* x, const int32_t* adapter_id
         if (!cluster_supported(la, T)) return false;
         ClusterScratch cs;
         cs.slots = (uint64_t*)(b + p.cslots);
+        cs.x_host = 0;
         cs.status = (int32_t*)(b + p.status);
         cs.idx_out = (int32_t*)(b + p.idx);
         cs.w_out = (float*)(b + p.w);
@@ -551,6 +554,54 @@ moe_status moe_ffn_forward(const moe_layer* layer, const uint16_t* x, const int3
     timing_begin(s);
     if (try_decode(layer, x, adapter_id, nullptr, T, 0, 0.0f, y, d, p, workspace, s, &st)) return st;
     return ffn_enqueue(layer, x, adapter_id, nullptr, T, nullptr, y, work_of(d, p, workspace), s);
+}
+
+moe_status moe_ffn_forward_host(const moe_layer* layer, const uint16_t* x_host, const int32_t* adapter_id, int32_t T,
+                                uint16_t* y_host, void* workspace, size_t ws_bytes, moe_stream stream) {
+    moe_status st = ffn_precheck(layer, x_host, y_host, T);
+    if (st != MOE_OK) return st;
+    if (T > MOEQ_DECODE_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;
+    const Dims d = dims_of(layer, T);
+    const WsPlan p = plan_of(d);
+    st = ws_check(workspace, ws_bytes, p.total);
+    if (st != MOE_OK) return st;
+    void *xd = nullptr, *yd = nullptr;
+    if (T > 0 && (cudaHostGetDevicePointer(&xd, const_cast<uint16_t*>(x_host), 0) != cudaSuccess ||
+                  cudaHostGetDevicePointer(&yd, y_host, 0) != cudaSuccess || !xd || !yd)) {
+        (void)cudaGetLastError();
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (T == 0) return MOE_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(s);
+    const LayerArgs la = args_of(layer);
+    char* b = (char*)workspace;
+    if (T == 1 && (g_decode_path == MOE_DECODE_AUTO || g_decode_path == MOE_DECODE_CLUSTER) &&
+        cluster_supported(la, 1)) {  // the kernel reads x and writes y across the bus itself
+        ClusterScratch cs;
+        cs.slots = (uint64_t*)(b + p.cslots);
+        cs.x_host = 1;
+        cs.status = (int32_t*)(b + p.status);
+        cs.idx_out = (int32_t*)(b + p.idx);
+        cs.w_out = (float*)(b + p.w);
+        const cudaError_t e = launch_cluster(la, (const uint16_t*)xd, adapter_id, nullptr, (uint16_t*)yd, 1, 0, 0.0f,
+                                             cs, s);
+        if (e == cudaSuccess) {
+            timing_mark(kDecodeCluster, s);
+            return MOE_OK;
+        }
+        if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) return MOE_ERR_CUDA;
+        (void)cudaGetLastError();
+    }
+    // staged: x into the workspace, the forward there, y back
+    uint16_t* xs = (uint16_t*)(b + p.hxin);
+    uint16_t* ys = (uint16_t*)(b + p.hyout);
+    const size_t nb = (size_t)T * d.H * 2;
+    if (cudaMemcpyAsync(xs, xd, nb, cudaMemcpyDefault, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!try_decode(layer, xs, adapter_id, nullptr, T, 0, 0.0f, ys, d, p, workspace, s, &st))
+        st = ffn_enqueue(layer, xs, adapter_id, nullptr, T, nullptr, ys, work_of(d, p, workspace), s);
+    if (st != MOE_OK) return st;
+    return cudaMemcpyAsync(yd, ys, nb, cudaMemcpyDefault, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_ffn_forward_select(const moe_layer* layer, const uint16_t* x, const int32_t* adapter_id,

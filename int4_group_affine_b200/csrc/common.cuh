@@ -90,6 +90,7 @@ struct WsPlan {
     size_t bar, dts, dtg, dtdp;  // fused decode scratch (sizes zero when T is too large for it)
     size_t slots;                // chain decode tagged words (right after the header, for every T)
     size_t cslots;               // cluster decode ticket and tagged words (after the chain's)
+    size_t hxin, hyout;          // staging of host x and y (moe_ffn_forward_host, T <= 8)
     size_t total;
 };
 
@@ -223,6 +224,7 @@ cudaError_t launch_chain(const LayerArgs& L, const uint16_t* x, const int32_t* a
 // workspace region of cluster_slot_words(...) words at a fixed place for a layer shape.
 struct ClusterScratch {
     uint64_t* slots;           // ticket counter, spares, tagged h words (starts zeroed)
+    int x_host;                // x is mapped host memory: read with plain loads, not a bulk copy
     int32_t* status;
     int32_t* idx_out;          // [K] routing record
     float* w_out;

@@ -87,6 +87,7 @@ struct QArgs {
     uint16_t* y;
     int block;
     float eps;
+    int x_host;                // x (and y) in mapped host memory: x read with plain loads
     unsigned long long* tick;  // ticket counter: a launch adds gridDim.x
     uint64_t* hg;              // [K+1][max(I, Is)] tagged h: routed slot k, then the shared expert
     unsigned long long* ready; // [gridDim.x] per CTA: the tag of the last launch whose h it published
@@ -330,7 +331,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
             s_gw[k] = winp(pol, sm + P.wsg + P.sg_off[6 + k], src, bytes, &s_bar[0], &tx);
         }
         asm volatile("griddepcontrol.wait;" ::: "memory");
-        if (lane == 0) win(sm + P.xraw, a.x, (uint32_t)(H * 2), &s_bar[0], &tx);
+        if (lane == 0 && !a.x_host) win(sm + P.xraw, a.x, (uint32_t)(H * 2), &s_bar[0], &tx);
         tx = warp_total(tx);
         if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[0], tx);
     } else if (warp == 1) {
@@ -377,6 +378,29 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     }
 
     // ------------------------------------------------------------ phase R: compute
+    if (a.x_host) {
+        // x across the bus once per cluster: CTA q reads its 1/CS of x (16-byte pieces) and
+        // stores each piece into every CTA of its cluster; after one cluster barrier every CTA
+        // holds all of x.  (A bulk copy does not read host memory here, and a read of all of x
+        // by every CTA would cross the bus 112 times.)
+        cl_wait();  // (every CTA of the cluster has started)
+        const int npc = H / 8, per = (npc + CS - 1) / CS;
+        if (tid < per && q * per + tid < npc) {
+            const int pi = q * per + tid;
+            const uint4 v = reinterpret_cast<const uint4*>(a.x)[pi];
+            uint32_t ra;
+            for (int rk = 0; rk < CS; ++rk) {
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                             : "=r"(ra)
+                             : "r"(tc::smem_u32(sm + P.xraw + 16 * pi)), "r"(rk));
+                asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ra), "r"(v.x), "r"(v.y), "r"(v.z),
+                             "r"(v.w)
+                             : "memory");
+            }
+        }
+        cl_arrive();
+        cl_wait();  // all of x is here
+    }
     copies_landed(&s_bar[0], a.status, &s_abort, lim);
     const uint16_t* xr = reinterpret_cast<const uint16_t*>(sm + P.xraw);
     if (a.block) {  // RMSNorm scale of the token
@@ -417,7 +441,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
         }
     }
     __syncthreads();
-    cl_wait();  // (every CTA of the cluster has started)
+    if (!a.x_host) cl_wait();  // (every CTA of the cluster has started; with x from host memory, above)
     // router rows (int8): row j of the CTA's range, or the shared-gate row (j == nra)
     auto row8 = [&](int j) {
         const bool sg = j == nra;
@@ -1126,6 +1150,7 @@ cudaError_t launch_cluster(const LayerArgs& L, const uint16_t* x, const int32_t*
     a.y = y;
     a.block = block;
     a.eps = eps;
+    a.x_host = sc.x_host;
     a.tick = reinterpret_cast<unsigned long long*>(sc.slots);
     a.hg = sc.slots + 8;
     a.ready = reinterpret_cast<unsigned long long*>(sc.slots + 8 + (size_t)(L.K + 1) * std::max(L.I, L.has_shared ? L.Is : 0));

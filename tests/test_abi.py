@@ -215,3 +215,15 @@ def test_decode_path_setting():
         assert moe_decode_path() == DECODE_AUTO
     finally:
         moe_set_decode_path(DECODE_AUTO)
+
+
+def test_host_forward_takes_decode_sizes_only():
+    """moe_ffn_forward_host: the forward's own checks first (x == y, misaligned), then more
+    than 8 tokens is UNSUPPORTED; all before any CUDA call."""
+    from int4_group_affine_b200 import moe_ffn_forward_host
+    L = _fake_layer()
+    for x, y, T, code in ((0x20000000, 0x20000000, 4, 1), (0x20000008, 0x30000000, 4, 1),
+                          (0x20000000, 0x30000000, 9, 2)):
+        with pytest.raises(MoeError) as ei:
+            moe_ffn_forward_host(L, x, None, T, y, 0x40000000, 1 << 30, stream=0)
+        assert ei.value.status == code

@@ -803,3 +803,56 @@ def test_mixed_mlp_full_size(mixed_layer, T, residual):
     else:
         ref = oracle.mixed_mlp(q["gate"], q["up"], q["down"], s.H, s.I, s.rho, x)
         assert_close_output(out, ref, "mixed mlp")
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_host_buffers_forward_matches_device_forward(T):
+    """moe_ffn_forward_host with x and y in pinned host memory: one token through the cluster
+    kernel reading and writing across the bus, four tokens staged through the workspace; each
+    bit-for-bit the device forward's output, and the oracle's within tolerance."""
+    m, ly = _mods()
+    shape = workloads.TINY
+    t, x, aid = _ffn_case(shape, 480 + T, T=T)
+    d = ly.DeviceLayer.from_host(shape, t)
+    ws, nb = d.workspace(T)
+    xd = ly.to_device(x)
+    yd = torch.empty_like(xd)
+    m.moe_ffn_forward(d.L, xd, None, T, yd, ws, nb)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status(ws) == 0
+    hx = torch.from_numpy(x.view(np.int16).copy()).pin_memory()
+    hy = torch.zeros((T, shape.H), dtype=torch.int16).pin_memory()
+    m.moe_workspace_init(ws, nb)
+    m.moe_timing_enable(True)
+    try:
+        m.moe_ffn_forward_host(d.L, hx, None, T, hy, ws, nb)
+        torch.cuda.synchronize()
+        kinds = set(m.moe_timing_collect())
+    finally:
+        m.moe_timing_enable(False)
+    assert m.moe_get_device_status(ws) == 0
+    assert path_ran("cluster" if T == 1 else "decode", kinds), kinds
+    assert np.array_equal(hy.numpy(), yd.cpu().numpy())
+    y_ref = oracle_layer(shape, t).ffn(x)[0]
+    assert_close_output(synth.bf16_to_f32(hy.numpy().view(np.uint16)).astype(np.float64), y_ref, "host buffers")
+
+
+def test_full_size_host_buffers_forward(full_layer):
+    """The Edge0 layer, one token, x and y in pinned host memory: the device forward's output."""
+    m, ly = _mods()
+    shape0, w, t = full_layer
+    shape = workloads.DECODE_K4
+    tt = dict(t)
+    tt["logit_bias"] = None
+    x, _ = workloads.moe_inputs(shape, seed=530, T=1)
+    d = ly.DeviceLayer.from_host(shape, tt, n_adapters=1)
+    ws, nb = d.workspace(1)
+    xd = ly.to_device(x)
+    yd = torch.empty_like(xd)
+    m.moe_ffn_forward(d.L, xd, None, 1, yd, ws, nb)
+    hx = torch.from_numpy(x.view(np.int16).copy()).pin_memory()
+    hy = torch.zeros((1, shape.H), dtype=torch.int16).pin_memory()
+    m.moe_ffn_forward_host(d.L, hx, None, 1, hy, ws, nb)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status(ws) == 0
+    assert np.array_equal(hy.numpy(), yd.cpu().numpy())
