@@ -110,10 +110,10 @@ __device__ __noinline__ void cdot_int4(const uint32_t* __restrict__ prow, const 
                                        const uint16_t* __restrict__ brow, int group, int n, const float* vbase,
                                        const float* vsum, const int* vid, int nv, float* acc, int sl, int lpt) {
     const uint4* p4 = reinterpret_cast<const uint4*>(prow);
-    const int nc = n / 32;
+    const int nc = n / 32, gsh = 31 - __clz(group >> 5);  // (group: a power of two, 32 or more)
 #pragma unroll 1
     for (int c = sl; c < nc; c += lpt) {
-        const int g = (c * 32) / group;
+        const int g = c >> gsh;
         const float s = bf16f(srow[g]), b128 = fmaf(-128.0f, s, bf16f(brow[g]));
         const uint4 q4 = p4[c];
         const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
@@ -145,10 +145,10 @@ __device__ __noinline__ void cdot_int8(const uint32_t* __restrict__ prow, const 
                                        const uint16_t* __restrict__ brow, int group, int n, const float* vbase,
                                        const float* vsum, int nv, float* acc, int lane) {
     const uint4* p4 = reinterpret_cast<const uint4*>(prow);
-    const int nc = n / 32;
+    const int nc = n / 32, gsh = 31 - __clz(group >> 5);  // (group: a power of two, 32 or more)
 #pragma unroll 1
     for (int c = lane; c < nc; c += 32) {
-        const int g = (c * 32) / group;
+        const int g = c >> gsh;
         const float s = bf16f(srow[g]), b = bf16f(brow[g]);
         const int rot = (c & 7) << 2;
 #pragma unroll

@@ -877,7 +877,8 @@ bool cwin_ok(const moe_qtensor& q) {
     const size_t rows = (size_t)q.n * q.out;
     const size_t pb = rows * (size_t)q.in * q.bits / 8, sb = rows * (size_t)(q.in / q.group) * 2;
     return ((uintptr_t)q.packed & 15) == 0 && ((uintptr_t)q.scales & 15) == 0 && ((uintptr_t)q.biases & 15) == 0 &&
-           pb % 16 == 0 && sb % 16 == 0 && q.group % 32 == 0;
+           pb % 16 == 0 && sb % 16 == 0 && q.group % 32 == 0 &&
+           (q.group & (q.group - 1)) == 0;
 }
 
 int c_sm_count() {
@@ -920,7 +921,9 @@ bool plan_chain(const LayerArgs& L, int T, int NB, CPlan* P) {
     if (T < 1 || T > kCMaxT || TK > kCMaxTK || r > kCMaxR || NB < 1 || NB > MOEQ_DECODE_MAX_CTAS) return false;
     if (E > MOEQ_MAX_EXPERTS || H % 32 || H > 4096 || I % 32 || I > 4096 || (sh && (Is % 32 || Is > 4096))) return false;
     if (!cwin_ok(L.router) || !cwin_ok(L.gate) || !cwin_ok(L.up) || !cwin_ok(L.down)) return false;
-    if (L.has_sgate && (((uintptr_t)L.shared_gate.packed & 15) || L.shared_gate.bits != 8)) return false;
+    if (L.has_sgate && (((uintptr_t)L.shared_gate.packed & 15) || L.shared_gate.bits != 8 ||
+                        L.shared_gate.group % 32 || (L.shared_gate.group & (L.shared_gate.group - 1))))
+        return false;
     if (sh && (!cwin_ok(L.s_gate) || !cwin_ok(L.s_up) || !cwin_ok(L.s_down))) return false;
     if (L.router.bits != 8 || L.gate.bits != 4 || L.up.bits != 4 || L.down.bits != 4) return false;
     if (lora) {  // LoRA rows move by bulk copies: 16-byte aligned factors, rows of whole 16-byte pieces

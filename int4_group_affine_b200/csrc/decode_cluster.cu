@@ -55,7 +55,7 @@ constexpr int kQMaxGT = 8;    // gate/up tiles (8 h elements each) per CTA
 constexpr int kQGW = 12;      // h words per thread in the gather ((K+1) max(I, Is) <= 12 * 512)
 
 struct QPlan {
-    int CS, perA, perS, perO, perC, nSA, nRA, nDA, imx_sh;
+    int CS, perA, perS, perO, perC, nSA, nRA, nDA, imx_sh, i_sh;
     int gu_ns, gu_spg, gu_gsh;    // routed gate/up tensor-core tiles: K slices, groups per slice, log2(group / 32)
     int lean;                     // 1: the routed LoRA-A rows reuse the phase-R windows (copied once the
                                   // shared-expert rows are read) and the packed down rows reuse the
@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     const int s_lo = min(Is, cta * P.perS), nsr = min(Is, s_lo + P.perS) - s_lo;
     const int o_lo = min(H, cta * P.perO), no = min(H, o_lo + P.perO) - o_lo;
     const int nC = K * I, c_lo = min(nC, cta * P.perC), c_hi = min(nC, c_lo + P.perC), nrows = c_hi - c_lo;
-    const int cut = nrows > 0 ? min(c_hi, (c_lo / I + 1) * I) : c_lo;
+    const int Ish_ = P.i_sh;  // I = 1 << i_sh
+    const int cut = nrows > 0 ? min(c_hi, ((c_lo >> Ish_) + 1) << Ish_) : c_lo;
     const int nsa_here = (lora && sh) ? max(0, min(P.nSA, 2 * r - q * P.nSA)) : 0;
     const int nra_here = lora ? max(0, min(P.nRA, K * 2 * r - q * P.nRA)) : 0;
     const int nda_here = lora ? max(0, min(P.nDA, (K + (sh ? 1 : 0)) * r - q * P.nDA)) : 0;
@@ -540,7 +541,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
         const int ng = H / qt.group;
         for (int j = lane; j < nrows; j += 32) {
             const int qq = c_lo + j;
-            const int64_t row = (int64_t)s_idx[qq / I] * I + qq % I;
+            const int64_t row = ((int64_t)s_idx[qq >> Ish_] << Ish_) + (qq & (I - 1));
             winp(pol, sm + P.wc + P.c_off[3 * pj] + j * P.rrs, s_abort ? nullptr : qt.packed + row * (H / 8),
                  (uint32_t)(H / 2), &s_bar[3], &tx);
         }
@@ -550,10 +551,10 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
             const void* src = nullptr;
             uint32_t off = P.wc + P.c_off[part];
             if (q1 > q0 && s_abort == 0) {
-                const int64_t row = (int64_t)s_idx[q0 / I] * I + q0 % I;
+                const int64_t row = ((int64_t)s_idx[q0 >> Ish_] << Ish_) + (q0 & (I - 1));
                 src = (k == 1 ? qt.scales : qt.biases) + row * ng;
                 if (sgi == 1 && cut > c_lo) {  // segment 1's window follows segment 0's
-                    const int64_t row0 = (int64_t)s_idx[c_lo / I] * I + c_lo % I;
+                    const int64_t row0 = ((int64_t)s_idx[c_lo >> Ish_] << Ish_) + (c_lo & (I - 1));
                     off += win_span((k == 1 ? qt.scales : qt.biases) + row0 * ng, (uint32_t)(cut - c_lo) * ng * 2);
                 }
             }
@@ -562,7 +563,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
             const int sgi = (lane - 4) / 2, pb = (lane - 4) % 2;
             const int q0 = sgi == 0 ? c_lo : cut, q1 = sgi == 0 ? cut : c_hi;
             const moe_lora_proj* lp = (lora && q1 > q0 && s_abort == 0) ? dlora(L, ad, false, pb) : nullptr;
-            const int64_t row = q1 > q0 ? (int64_t)s_idx[q0 / I] * I + q0 % I : 0;
+            const int64_t row = q1 > q0 ? ((int64_t)s_idx[q0 >> Ish_] << Ish_) + (q0 & (I - 1)) : 0;
             s_rbw[sgi][pb] = winp(pol, sm + P.wrb + (lane - 4) * P.rb_stride, lp ? lp->B + row * r : nullptr,
                                   (uint32_t)((q1 - q0) * r * 2), &s_bar[3], &tx);
         }
@@ -704,7 +705,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
                 }
                 dst = a.hg + (int64_t)K * Imx + s_lo + j;
             } else {
-                const int jj = j - nsr, qq = c_lo + jj, k = qq / I, sg = qq < cut ? 0 : 1;
+                const int jj = j - nsr, qq = c_lo + jj, k = qq >> Ish_, sg = qq < cut ? 0 : 1;
                 const float* gp = reinterpret_cast<const float*>(sm + P.gpart) + (jj / 8) * P.gu_ns * 16 + jj % 8;
                 g = 0.0f;
                 u = 0.0f;
@@ -719,7 +720,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
                     tu = tg + r;
                     br = qq - (sg == 0 ? c_lo : cut);
                 }
-                dst = a.hg + (int64_t)k * Imx + qq % I;
+                dst = a.hg + (int64_t)k * Imx + (qq & (I - 1));
             }
             if (lora && bg && bu) {
                 float dg = 0.0f, du = 0.0f;
@@ -896,7 +897,8 @@ bool qwin_ok(const moe_qtensor& t) {
     const size_t rows = (size_t)t.n * t.out;
     const size_t pb = rows * (size_t)t.in * t.bits / 8, sb = rows * (size_t)(t.in / t.group) * 2;
     return ((uintptr_t)t.packed & 15) == 0 && ((uintptr_t)t.scales & 15) == 0 && ((uintptr_t)t.biases & 15) == 0 &&
-           pb % 16 == 0 && sb % 16 == 0 && t.group % 32 == 0;
+           pb % 16 == 0 && sb % 16 == 0 && t.group % 32 == 0 &&
+           (t.group & (t.group - 1)) == 0;
 }
 
 int q_optin_smem() {
@@ -927,7 +929,9 @@ bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P, bool lean
         return false;
     if (E > kQMaxE || H % 32 || H > 4096 || I % 32 || I > 4096 || (sh && (Is % 32 || Is > 4096))) return false;
     if (!qwin_ok(L.router) || !qwin_ok(L.gate) || !qwin_ok(L.up) || !qwin_ok(L.down)) return false;
-    if (L.has_sgate && (((uintptr_t)L.shared_gate.packed & 15) || L.shared_gate.bits != 8)) return false;
+    if (L.has_sgate && (((uintptr_t)L.shared_gate.packed & 15) || L.shared_gate.bits != 8 ||
+                        L.shared_gate.group % 32 || (L.shared_gate.group & (L.shared_gate.group - 1))))
+        return false;
     if (sh && (!qwin_ok(L.s_gate) || !qwin_ok(L.s_up) || !qwin_ok(L.s_down))) return false;
     if (L.router.bits != 8 || L.gate.bits != 4 || L.up.bits != 4 || L.down.bits != 4) return false;
     if (sh && (L.s_gate.bits != 4 || L.s_up.bits != 4 || L.s_down.bits != 4)) return false;
@@ -945,6 +949,9 @@ bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P, bool lean
     P->lean = lean ? 1 : 0;
     P->imx_sh = 0;
     while ((1 << P->imx_sh) < Imx) ++P->imx_sh;
+    if (I & (I - 1)) return false;  // (h elements are split into (expert, row) by shifts)
+    P->i_sh = 0;
+    while ((1 << P->i_sh) < I) ++P->i_sh;
     P->perA = cdivq(E, CS);
     P->perS = sh ? cdivq(Is, NB) : 0;
     P->perO = cdivq(H, NB);
