@@ -853,29 +853,28 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     }
     cl_wait();  // the down LoRA-A products of the whole cluster are here
     __syncthreads();
-    if (s_abort == 0 && tid < no) {  // combine, one thread per output row
-        const int ol = tid;
-        float acc = 0.0f;
-        for (int k = 0; k < KS; ++k) {
-            float v = sv[ol * KS + k];
-            if (lora) {
-                const uint16_t* bd = reinterpret_cast<const uint16_t*>(k < K ? s_rbdw[k] : s_sbw[2]);
-                if (bd) {
-                    float t = 0.0f;
-                    for (int c0 = 0; c0 < r; c0 += 8) {
-                        const uint4 wb = *reinterpret_cast<const uint4*>(bd + ol * r + c0);
-                        const uint32_t vb[4] = {wb.x, wb.y, wb.z, wb.w};
+    if (lora && s_abort == 0 && tid < no * KS) {  // per (output row, expert): the LoRA-B delta
+        const int ol = tid / KS, k = tid - ol * KS;
+        const uint16_t* bd = reinterpret_cast<const uint16_t*>(k < K ? s_rbdw[k] : s_sbw[2]);
+        if (bd) {
+            float t = 0.0f;
+            for (int c0 = 0; c0 < r; c0 += 8) {
+                const uint4 wb = *reinterpret_cast<const uint4*>(bd + ol * r + c0);
+                const uint32_t vb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-                        for (int q2 = 0; q2 < 4; ++q2) {
-                            t = fmaf(__uint_as_float(vb[q2] << 16), da[k * r + c0 + 2 * q2], t);
-                            t = fmaf(__uint_as_float(vb[q2] & 0xFFFF0000u), da[k * r + c0 + 2 * q2 + 1], t);
-                        }
-                    }
-                    v += L.scale * t;
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    t = fmaf(__uint_as_float(vb[q2] << 16), da[k * r + c0 + 2 * q2], t);
+                    t = fmaf(__uint_as_float(vb[q2] & 0xFFFF0000u), da[k * r + c0 + 2 * q2 + 1], t);
                 }
             }
-            acc = k < K ? fmaf(s_w[k], v, acc) : fmaf(s_sig, v, acc);
+            sv[tid] += L.scale * t;
         }
+    }
+    __syncthreads();
+    if (s_abort == 0 && tid < no) {  // combine in fixed order (k = 0..K-1, then the shared expert)
+        const int ol = tid;
+        float acc = 0.0f;
+        for (int k = 0; k < KS; ++k) acc = fmaf(k < K ? s_w[k] : s_sig, sv[ol * KS + k], acc);
         const int o = o_lo + ol;
         if (a.block) acc += bf16f(xr[o]);
         a.y[o] = f2bf16(acc);
