@@ -75,7 +75,7 @@ struct QPlan {
     uint32_t wd, d_off[3], d_stride;  // routed down rows of slot k at wd + k * d_stride
     uint32_t wrbd, rbd_stride;    // routed down LoRA-B rows [slot]
     uint32_t wda, da_stride;      // down LoRA-A rows
-    uint32_t sgu, gu, hs, hsum, sv;  // (hs, hsum reuse the routed gate/up windows)
+    uint32_t sgu, hs, hsum, sv;   // (hs, hsum reuse the routed gate/up windows)
     uint32_t total;
 };
 
@@ -244,13 +244,12 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     float* ra = reinterpret_cast<float*>(sm + P.ra);    // [K][2r] routed LoRA-A products (cluster)
     float* da = reinterpret_cast<float*>(sm + P.da);    // [K+1][r] down LoRA-A products (cluster)
     float* sgu = reinterpret_cast<float*>(sm + P.sgu);  // [perS][2] shared gate/up dots
-    float* gu = reinterpret_cast<float*>(sm + P.gu);    // [perC][2] routed gate/up dots
     float* hs = reinterpret_cast<float*>(sm + P.hs);    // [K+1][Imx] h (swizzled)
     float* hsum = reinterpret_cast<float*>(sm + P.hsum);
     float* sv = reinterpret_cast<float*>(sm + P.sv);    // [perO][K+1] per-expert outputs of the CTA's rows
 
     __shared__ __align__(8) uint64_t s_bar[6];
-    __shared__ int s_abort, s_aid;
+    __shared__ int s_abort, s_aid, s_gut;
     __shared__ uint32_t s_tag;
     __shared__ float s_inv, s_sig;
     __shared__ int32_t s_sel[kQMaxK];
@@ -274,6 +273,7 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     // (warp 1); 4: routed down rows + their LoRA-B rows (warp 2) + down LoRA-A rows (warp 4)
     if (tid == 0) {
         s_abort = 0;
+        s_gut = 0;
         s_sig = 1.0f;
         s_inv = 1.0f;
         for (int i = 0; i < 6; ++i) tc::mbar_init(&s_bar[i], (i == 3 || i == 4) ? 2u : 1u);
@@ -630,7 +630,9 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     }
 
     // ------------------------------------------------------------ phase G
-    for (int j = warp; j < nra_here; j += kCW) {  // routed LoRA-A rows -> products to the cluster
+    // routed LoRA-A rows -> products to the cluster, on the last warps (the first ones have just
+    // issued the copies and take gate/up tasks as soon as the rows land)
+    for (int j = kCW - 1 - warp; j < nra_here; j += kCW) {
         copies_landed(&s_bar[2], a.status, &s_abort, lim);
         float v = 0.0f;
         if (s_raw[j]) v = warp_sum(sdot_bf16(reinterpret_cast<const uint16_t*>(s_raw[j]), H, xs, lane));
@@ -643,7 +645,14 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
         const int NT = (nrows + 7) / 8, NS = P.gu_ns, spg = P.gu_spg, ngr = H / L.gate.group;
         const int g = lane >> 2, c = lane & 3, gsh = P.gu_gsh;
         float* gpart = reinterpret_cast<float*>(sm + P.gpart);
-        for (int t = warp; t < NT * NS; t += kCW) {
+        // tasks are taken from a counter as warps come free (their partial sums have fixed
+        // places, so the result does not depend on which warp took a task)
+        auto grab = [&]() {
+            int v = 0;
+            if (lane == 0) v = atomicAdd(&s_gut, 1);
+            return __shfl_sync(0xffffffffu, v, 0);
+        };
+        for (int t = grab(); t < NT * NS; t = grab()) {
             const int tile = t / NS, sl = t % NS, j = 8 * tile + g;
             copies_landed(&s_bar[3], a.status, &s_abort, lim);
             const bool live = j < nrows && s_cw[0][1];
@@ -799,15 +808,33 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
             if (i < nh && e < (slot < K ? I : Is) && !fresh(w[b], tag)) w[b] = peek(a.hg + i);
         }
         // (a warp's 32 elements of a pass are one 32-element chunk of one slot: I and Is are
-        // multiples of 32, so its chunk sum is one warp reduction)
+        // multiples of 32, so its chunk sum is one warp reduction).  The passes' values first,
+        // then their reductions side by side (one chain of five shuffle steps for all passes,
+        // not one chain per pass; the second half only when there are that many words)
+        float v[kQGW], cs[kQGW];
+#pragma unroll
+        for (int b = 0; b < kQGW; ++b) {
+            v[b] = fresh(w[b], tag) ? wval(w[b]) : 0.0f;  // (0 past the end: those words read as 0)
+            cs[b] = v[b];
+        }
+        constexpr int kH1 = kQGW / 2;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int b = 0; b < kH1; ++b) cs[b] += __shfl_xor_sync(0xffffffffu, cs[b], o);
+        if (nh > kH1 * kCT) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int b = kH1; b < kQGW; ++b) cs[b] += __shfl_xor_sync(0xffffffffu, cs[b], o);
+        }
 #pragma unroll
         for (int b = 0; b < kQGW; ++b) {
             const int i = b * kCT + tid, slot = i >> Ish, e = i & (Imx - 1);
-            if (i - lane >= nh || e - lane >= (slot < K ? I : Is)) continue;  // (uniform across the warp)
-            const float v = fresh(w[b], tag) ? wval(w[b]) : 0.0f;
-            hs[slot * Imx + swz(e)] = v;
-            const float cs = warp_sum(v);
-            if (lane == 0) hsum[slot * (Imx / 32) + (e >> 5)] = cs;
+            if (i - lane < nh && e - lane < (slot < K ? I : Is)) {  // (uniform across the warp)
+                hs[slot * Imx + swz(e)] = v[b];
+                if (lane == 0) hsum[slot * (Imx / 32) + (e >> 5)] = cs[b];
+            }
         }
         __syncthreads();
     }
@@ -1067,7 +1094,6 @@ bool plan_cluster(const LayerArgs& L, int T, int CS, int NB, QPlan* P, bool lean
         P->gpart = take((size_t)ntm * P->gu_ns * 16 * 4);
     }
     P->sgu = take((size_t)std::max(P->perS, 1) * 2 * 4);
-    P->gu = take((size_t)std::max(P->perC, 1) * 2 * 4);
     P->sv = take((size_t)P->perO * KS * 4);
     P->total = (uint32_t)o;
     const size_t limit = (size_t)q_optin_smem() > q_static_smem() ? (size_t)q_optin_smem() - q_static_smem() : 0;
