@@ -22,7 +22,9 @@
 //
 //  R  x; the CTA's router rows -> logits to the cluster; the shared-gate row (every
 //     CTA); the CTA's shared gate/up rows; shared LoRA-A rows -> products to the cluster.
-//  K  top-K in every CTA; the routed rows' bulk copies issued.
+//  K  top-K in every CTA; the routed rows' bulk copies issued.  With a given expert set
+//     (the prerouter's prediction) the copies go out as soon as the CTA's router rows are
+//     done, and the cluster's logits give only the weights.
 //  G  routed LoRA-A rows -> products to the cluster; routed gate/up dots; LoRA-B
 //     deltas and SwiGLU: h elements published (shared and routed).
 //  X  every CTA gathers h.
@@ -292,6 +294,114 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
     const int nra_here = lora ? max(0, min(P.nRA, K * 2 * r - q * P.nRA)) : 0;
     const int nda_here = lora ? max(0, min(P.nDA, (K + (sh ? 1 : 0)) * r - q * P.nDA)) : 0;
 
+    // The routed rows' bulk copies (warps 0..4; the routing in s_idx, the adapter ad):
+    // gate/up rows, their scales, biases and LoRA-B rows (warps 0, 1), down rows with theirs
+    // (warp 2), routed LoRA-A rows (warp 3), down LoRA-A rows (warp 4).
+    auto issue_routed = [&](const int ad) {
+        if (warp < 2) {
+            // routed gate (warp 0) | up (warp 1) rows: lane j copies the rows of h elements c_lo + j,
+            // c_lo + j + 32, .. to their own slots (stride rrs); lanes 0..3 copy the scales and
+            // biases of the two segments (rows of one expert each); warp 1 lanes 4..7 the LoRA-B rows
+            uint32_t tx = 0;
+            const int pj = warp;
+            const moe_qtensor& qt = pj ? L.up : L.gate;
+            const int ng = H / qt.group;
+            for (int j = lane; j < nrows; j += 32) {
+                const int qq = c_lo + j;
+                const int64_t row = ((int64_t)s_idx[qq >> Ish_] << Ish_) + (qq & (I - 1));
+                winp(pol, sm + P.wc + P.c_off[3 * pj] + j * P.rrs, s_abort ? nullptr : qt.packed + row * (H / 8),
+                     (uint32_t)(H / 2), &s_bar[3], &tx);
+            }
+            if (lane < 4) {  // scales | biases of the two segments: lane 2 s + (k - 1)
+                const int sgi = lane / 2, k = 1 + lane % 2, part = 3 * pj + k;
+                const int q0 = sgi == 0 ? c_lo : cut, q1 = sgi == 0 ? cut : c_hi;
+                const void* src = nullptr;
+                uint32_t off = P.wc + P.c_off[part];
+                if (q1 > q0 && s_abort == 0) {
+                    const int64_t row = ((int64_t)s_idx[q0 >> Ish_] << Ish_) + (q0 & (I - 1));
+                    src = (k == 1 ? qt.scales : qt.biases) + row * ng;
+                    if (sgi == 1 && cut > c_lo) {  // segment 1's window follows segment 0's
+                        const int64_t row0 = ((int64_t)s_idx[c_lo >> Ish_] << Ish_) + (c_lo & (I - 1));
+                        off += win_span((k == 1 ? qt.scales : qt.biases) + row0 * ng, (uint32_t)(cut - c_lo) * ng * 2);
+                    }
+                }
+                s_cw[sgi][part] = winp(pol, sm + off, src, (uint32_t)(q1 - q0) * ng * 2, &s_bar[3], &tx);
+            } else if (pj == 1 && lane < 8) {  // LoRA-B rows of the routed gate/up rows: lane 4 + 2 s + p
+                const int sgi = (lane - 4) / 2, pb = (lane - 4) % 2;
+                const int q0 = sgi == 0 ? c_lo : cut, q1 = sgi == 0 ? cut : c_hi;
+                const moe_lora_proj* lp = (lora && q1 > q0 && s_abort == 0) ? dlora(L, ad, false, pb) : nullptr;
+                const int64_t row = q1 > q0 ? ((int64_t)s_idx[q0 >> Ish_] << Ish_) + (q0 & (I - 1)) : 0;
+                s_rbw[sgi][pb] = winp(pol, sm + P.wrb + (lane - 4) * P.rb_stride, lp ? lp->B + row * r : nullptr,
+                                      (uint32_t)((q1 - q0) * r * 2), &s_bar[3], &tx);
+            }
+            tx = warp_total(tx);
+            if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[3], tx);
+        } else if (warp == 2) {  // routed down rows of the CTA's output range and their LoRA-B rows
+            uint32_t tx = 0;
+            const int ngd = I / L.down.group;
+            if (lane < 3 * K) {
+                const int k = lane / 3, part = lane % 3;
+                const int64_t row = (int64_t)s_idx[k] * H + o_lo;
+                const void* src = nullptr;
+                uint32_t bytes = 0;
+                if (no > 0 && s_abort == 0) {
+                    src = part == 0 ? (const void*)(L.down.packed + row * (I / 8))
+                                    : (const void*)((part == 1 ? L.down.scales : L.down.biases) + row * ngd);
+                    bytes = part == 0 ? (uint32_t)(no * I / 2) : (uint32_t)(no * ngd * 2);
+                }
+                if (part > 0 || !P.lean)
+                    s_dw[k][part] = winp(pol, sm + (part == 0 ? P.dp + k * P.dp_stride : P.wd + k * P.d_stride + P.d_off[part]),
+                                         src, bytes, &s_bar[4], &tx);
+            }
+            if (lane < K) {
+                const moe_lora_proj* lp = (lora && no > 0 && s_abort == 0) ? dlora(L, ad, false, 2) : nullptr;
+                const int64_t row = (int64_t)s_idx[lane] * H + o_lo;
+                s_rbdw[lane] = winp(pol, sm + P.wrbd + lane * P.rbd_stride, lp ? lp->B + row * r : nullptr,
+                                   (uint32_t)(no * r * 2), &s_bar[4], &tx);
+            }
+            tx = warp_total(tx);
+            if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[4], tx);
+        } else if (warp == 3) {  // routed LoRA-A rows: row d = q nRA + lane of [slot k][gate A | up A]
+            if (P.lean) {  // (their slots are the phase-R windows: wait for warps kQIssue.. to be done with them)
+                asm volatile("bar.sync 2, %0;" ::"n"((kCW - kQIssue + 1) * 32) : "memory");
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
+            uint32_t tx = 0;
+            if (lane < kQMaxRA) {
+                const int d = q * P.nRA + lane, k = d / max(2 * r, 1), c = d % max(2 * r, 1);
+                const moe_lora_proj* lp = (lane < nra_here && s_abort == 0) ? dlora(L, ad, false, c < r ? 0 : 1) : nullptr;
+                const int64_t row = lp ? ((int64_t)s_idx[k] * r + c % r) * H : 0;
+                s_raw[lane] = winp(pol, sm + P.wra + lane * P.ra_stride, lp ? lp->A + row : nullptr, (uint32_t)(H * 2),
+                                  &s_bar[2], &tx);
+            }
+            tx = warp_total(tx);
+            if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[2], tx);
+        } else if (warp == 4) {  // down LoRA-A rows: row d = q nDA + lane of [slot k][component]; slot K shared
+            uint32_t tx = 0;
+            if (lane < kQMaxDA) {
+                const int d = q * P.nDA + lane, k = d / max(r, 1), c = d % max(r, 1);
+                const moe_lora_proj* lp = nullptr;
+                const uint16_t* src = nullptr;
+                int n = I;
+                if (lane < nda_here && s_abort == 0) {
+                    lp = dlora(L, ad, k == K, 2);
+                    if (lp) {
+                        src = k < K ? lp->A + ((int64_t)s_idx[k] * r + c) * I : lp->A + (int64_t)c * Is;
+                        n = k < K ? I : Is;
+                    }
+                }
+                s_daw[lane] = winp(pol, sm + P.wda + lane * P.da_stride, src, (uint32_t)(n * 2), &s_bar[4], &tx);
+            }
+            tx = warp_total(tx);
+            if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[4], tx);
+        }
+    };
+    // A given expert set (the prerouter's prediction) needs no top-K: its rows are copied as
+    // soon as the CTA's router rows are done, while the cluster's logits (which give only the
+    // weights then) come together.  (Not in the lean layout, whose routed LoRA-A windows are
+    // free only after phase R.)
+    const bool early = a.select != nullptr && !P.lean;
+
     // ------------------------------------------------------------ phase R: issue
     // The weight rows of this phase depend on nothing the previous kernel on the stream
     // writes: their copies start before the grid-dependency wait.  Everything that reads
@@ -343,7 +453,14 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
             ad = -1;
         }
         if (lane == 0) s_aid = ad;
-        if (a.select && lane < K) s_sel[lane] = a.select[lane];
+        if (a.select) {  // the given set, repaired (an entry out of range or repeated: the lowest unused expert)
+            if (lane < K) s_sel[lane] = a.select[lane];
+            __syncwarp();
+            bool bad = false;
+            const int e = select_entry(s_sel, K, E, lane, &bad);
+            if (bad && lane == 0 && cta == 0) raise_status(a.status, MOE_ERR_DEVICE_INDEX);
+            if (lane < K) s_idx[lane] = e;
+        }
         uint32_t tx = 0;
         if (lane < 3) {  // shared down rows of the CTA's output range
             const void* src = nullptr;
@@ -464,169 +581,78 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
         }
     }
     cl_arrive();  // this CTA's logits are in every CTA of the cluster
-    // on warps kQIssue..: the shared-gate row, shared gate/up rows and shared LoRA-A rows
-    // (their products reach the cluster by the next cluster barrier), while warp 0 takes
-    // the top-K and warps 0..kQIssue-1 issue the routed rows' copies
-    for (int t = warp - kQIssue; warp >= kQIssue && t < 1 + nsr + nsa_here; t += kCW - kQIssue) {
-        if (t == 0) {
-            if (L.has_sgate) {
-                const float v = row8(nra);
-                if (lane == 0) s_sig = 1.0f / (1.0f + expf(-v));
-            }
-        } else if (t <= nsr) {
-            const int j = t - 1;
-            float ag[1] = {0.0f}, au[1] = {0.0f};
-            const int vid[1] = {0};
-            const int ngg = H / L.s_gate.group, ngu = H / L.s_up.group;
-            if (s_sgw[0] && s_sgw[3]) {
-                cdot_int4<1>(reinterpret_cast<const uint32_t*>(s_sgw[0] + (size_t)j * (H / 2)),
-                             reinterpret_cast<const uint16_t*>(s_sgw[1]) + j * ngg,
-                             reinterpret_cast<const uint16_t*>(s_sgw[2]) + j * ngg, L.s_gate.group, H, xs, xsum, vid, 1,
-                             ag, lane, 32);
-                cdot_int4<1>(reinterpret_cast<const uint32_t*>(s_sgw[3] + (size_t)j * (H / 2)),
-                             reinterpret_cast<const uint16_t*>(s_sgw[4]) + j * ngu,
-                             reinterpret_cast<const uint16_t*>(s_sgw[5]) + j * ngu, L.s_up.group, H, xs, xsum, vid, 1,
-                             au, lane, 32);
-            }
-            const float g = warp_sum(ag[0]), u = warp_sum(au[0]);
-            if (lane == 0) {
-                sgu[2 * j] = g;
-                sgu[2 * j + 1] = u;
-            }
-        } else {
-            const int jj = t - 1 - nsr;
-            copies_landed(&s_bar[1], a.status, &s_abort, lim);
-            float v = 0.0f;
-            if (s_saw[jj]) v = warp_sum(sdot_bf16(reinterpret_cast<const uint16_t*>(s_saw[jj]), H, xs, lane));
-            if (lane < CS) dsm_st(sa + q * P.nSA + jj, lane, v);
-        }
-    }
-    if (P.lean && warp >= kQIssue) asm volatile("bar.arrive 2, %0;" ::"n"((kCW - kQIssue + 1) * 32) : "memory");
-    cl_wait();  // the logits of the whole cluster are here
-
-    // ------------------------------------------------------------ phase K
-    if (warp == 0) {
-        if (a.select) {  // a caller-given set (the prerouter's prediction): only the weights come from z
-            bool bad = false;
-            const int e = select_entry(s_sel, K, E, lane, &bad);
-            if (bad && lane == 0 && cta == 0) raise_status(a.status, MOE_ERR_DEVICE_INDEX);
-            const float zk = e >= 0 ? z[e] : -INFINITY;
-            const float m = warp_max(zk);
-            const float ev = e >= 0 ? expf(zk - m) : 0.0f;
-            const float sum = warp_sum(ev);
-            if (lane < K) {
-                s_idx[lane] = e;
-                s_w[lane] = ev / sum;
-            }
-        } else {
-            warp_topk<kQMaxE / 32>(z, E, K, lane, s_idx, s_w);
-        }
-        __syncwarp();
-        if (cta == 0 && lane < K) {  // the routing this call used, for the caller's record
-            a.idx_out[lane] = s_idx[lane];
-            a.w_out[lane] = s_w[lane];
-        }
-    }
-    // the routing is known to the issuing warps (the others learn the window pointers
-    // through the copies' mbarriers)
-    if (warp < kQIssue) asm volatile("bar.sync 1, %0;" ::"n"(kQIssue * 32) : "memory");
-    const int ad = s_aid;
-    if (warp < 2) {
-        // routed gate (warp 0) | up (warp 1) rows: lane j copies the rows of h elements c_lo + j,
-        // c_lo + j + 32, .. to their own slots (stride rrs); lanes 0..3 copy the scales and
-        // biases of the two segments (rows of one expert each); warp 1 lanes 4..7 the LoRA-B rows
-        uint32_t tx = 0;
-        const int pj = warp;
-        const moe_qtensor& qt = pj ? L.up : L.gate;
-        const int ng = H / qt.group;
-        for (int j = lane; j < nrows; j += 32) {
-            const int qq = c_lo + j;
-            const int64_t row = ((int64_t)s_idx[qq >> Ish_] << Ish_) + (qq & (I - 1));
-            winp(pol, sm + P.wc + P.c_off[3 * pj] + j * P.rrs, s_abort ? nullptr : qt.packed + row * (H / 8),
-                 (uint32_t)(H / 2), &s_bar[3], &tx);
-        }
-        if (lane < 4) {  // scales | biases of the two segments: lane 2 s + (k - 1)
-            const int sgi = lane / 2, k = 1 + lane % 2, part = 3 * pj + k;
-            const int q0 = sgi == 0 ? c_lo : cut, q1 = sgi == 0 ? cut : c_hi;
-            const void* src = nullptr;
-            uint32_t off = P.wc + P.c_off[part];
-            if (q1 > q0 && s_abort == 0) {
-                const int64_t row = ((int64_t)s_idx[q0 >> Ish_] << Ish_) + (q0 & (I - 1));
-                src = (k == 1 ? qt.scales : qt.biases) + row * ng;
-                if (sgi == 1 && cut > c_lo) {  // segment 1's window follows segment 0's
-                    const int64_t row0 = ((int64_t)s_idx[c_lo >> Ish_] << Ish_) + (c_lo & (I - 1));
-                    off += win_span((k == 1 ? qt.scales : qt.biases) + row0 * ng, (uint32_t)(cut - c_lo) * ng * 2);
+    if (warp >= kQIssue) {
+        // the shared-gate row, shared gate/up rows and shared LoRA-A rows (their products
+        // reach the cluster by the next cluster barrier), while warps 0..kQIssue-1 route and
+        // issue the routed rows' copies
+        for (int t = warp - kQIssue; t < 1 + nsr + nsa_here; t += kCW - kQIssue) {
+            if (t == 0) {
+                if (L.has_sgate) {
+                    const float v = row8(nra);
+                    if (lane == 0) s_sig = 1.0f / (1.0f + expf(-v));
                 }
-            }
-            s_cw[sgi][part] = winp(pol, sm + off, src, (uint32_t)(q1 - q0) * ng * 2, &s_bar[3], &tx);
-        } else if (pj == 1 && lane < 8) {  // LoRA-B rows of the routed gate/up rows: lane 4 + 2 s + p
-            const int sgi = (lane - 4) / 2, pb = (lane - 4) % 2;
-            const int q0 = sgi == 0 ? c_lo : cut, q1 = sgi == 0 ? cut : c_hi;
-            const moe_lora_proj* lp = (lora && q1 > q0 && s_abort == 0) ? dlora(L, ad, false, pb) : nullptr;
-            const int64_t row = q1 > q0 ? ((int64_t)s_idx[q0 >> Ish_] << Ish_) + (q0 & (I - 1)) : 0;
-            s_rbw[sgi][pb] = winp(pol, sm + P.wrb + (lane - 4) * P.rb_stride, lp ? lp->B + row * r : nullptr,
-                                  (uint32_t)((q1 - q0) * r * 2), &s_bar[3], &tx);
-        }
-        tx = warp_total(tx);
-        if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[3], tx);
-    } else if (warp == 2) {  // routed down rows of the CTA's output range and their LoRA-B rows
-        uint32_t tx = 0;
-        const int ngd = I / L.down.group;
-        if (lane < 3 * K) {
-            const int k = lane / 3, part = lane % 3;
-            const int64_t row = (int64_t)s_idx[k] * H + o_lo;
-            const void* src = nullptr;
-            uint32_t bytes = 0;
-            if (no > 0 && s_abort == 0) {
-                src = part == 0 ? (const void*)(L.down.packed + row * (I / 8))
-                                : (const void*)((part == 1 ? L.down.scales : L.down.biases) + row * ngd);
-                bytes = part == 0 ? (uint32_t)(no * I / 2) : (uint32_t)(no * ngd * 2);
-            }
-            if (part > 0 || !P.lean)
-                s_dw[k][part] = winp(pol, sm + (part == 0 ? P.dp + k * P.dp_stride : P.wd + k * P.d_stride + P.d_off[part]),
-                                     src, bytes, &s_bar[4], &tx);
-        }
-        if (lane < K) {
-            const moe_lora_proj* lp = (lora && no > 0 && s_abort == 0) ? dlora(L, ad, false, 2) : nullptr;
-            const int64_t row = (int64_t)s_idx[lane] * H + o_lo;
-            s_rbdw[lane] = winp(pol, sm + P.wrbd + lane * P.rbd_stride, lp ? lp->B + row * r : nullptr,
-                               (uint32_t)(no * r * 2), &s_bar[4], &tx);
-        }
-        tx = warp_total(tx);
-        if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[4], tx);
-    } else if (warp == 3) {  // routed LoRA-A rows: row d = q nRA + lane of [slot k][gate A | up A]
-        if (P.lean) {  // (their slots are the phase-R windows: wait for warps kQIssue.. to be done with them)
-            asm volatile("bar.sync 2, %0;" ::"n"((kCW - kQIssue + 1) * 32) : "memory");
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        }
-        uint32_t tx = 0;
-        if (lane < kQMaxRA) {
-            const int d = q * P.nRA + lane, k = d / max(2 * r, 1), c = d % max(2 * r, 1);
-            const moe_lora_proj* lp = (lane < nra_here && s_abort == 0) ? dlora(L, ad, false, c < r ? 0 : 1) : nullptr;
-            const int64_t row = lp ? ((int64_t)s_idx[k] * r + c % r) * H : 0;
-            s_raw[lane] = winp(pol, sm + P.wra + lane * P.ra_stride, lp ? lp->A + row : nullptr, (uint32_t)(H * 2),
-                              &s_bar[2], &tx);
-        }
-        tx = warp_total(tx);
-        if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[2], tx);
-    } else if (warp == 4) {  // down LoRA-A rows: row d = q nDA + lane of [slot k][component]; slot K shared
-        uint32_t tx = 0;
-        if (lane < kQMaxDA) {
-            const int d = q * P.nDA + lane, k = d / max(r, 1), c = d % max(r, 1);
-            const moe_lora_proj* lp = nullptr;
-            const uint16_t* src = nullptr;
-            int n = I;
-            if (lane < nda_here && s_abort == 0) {
-                lp = dlora(L, ad, k == K, 2);
-                if (lp) {
-                    src = k < K ? lp->A + ((int64_t)s_idx[k] * r + c) * I : lp->A + (int64_t)c * Is;
-                    n = k < K ? I : Is;
+            } else if (t <= nsr) {
+                const int j = t - 1;
+                float ag[1] = {0.0f}, au[1] = {0.0f};
+                const int vid[1] = {0};
+                const int ngg = H / L.s_gate.group, ngu = H / L.s_up.group;
+                if (s_sgw[0] && s_sgw[3]) {
+                    cdot_int4<1>(reinterpret_cast<const uint32_t*>(s_sgw[0] + (size_t)j * (H / 2)),
+                                 reinterpret_cast<const uint16_t*>(s_sgw[1]) + j * ngg,
+                                 reinterpret_cast<const uint16_t*>(s_sgw[2]) + j * ngg, L.s_gate.group, H, xs, xsum, vid, 1,
+                                 ag, lane, 32);
+                    cdot_int4<1>(reinterpret_cast<const uint32_t*>(s_sgw[3] + (size_t)j * (H / 2)),
+                                 reinterpret_cast<const uint16_t*>(s_sgw[4]) + j * ngu,
+                                 reinterpret_cast<const uint16_t*>(s_sgw[5]) + j * ngu, L.s_up.group, H, xs, xsum, vid, 1,
+                                 au, lane, 32);
                 }
+                const float g = warp_sum(ag[0]), u = warp_sum(au[0]);
+                if (lane == 0) {
+                    sgu[2 * j] = g;
+                    sgu[2 * j + 1] = u;
+                }
+            } else {
+                const int jj = t - 1 - nsr;
+                copies_landed(&s_bar[1], a.status, &s_abort, lim);
+                float v = 0.0f;
+                if (s_saw[jj]) v = warp_sum(sdot_bf16(reinterpret_cast<const uint16_t*>(s_saw[jj]), H, xs, lane));
+                if (lane < CS) dsm_st(sa + q * P.nSA + jj, lane, v);
             }
-            s_daw[lane] = winp(pol, sm + P.wda + lane * P.da_stride, src, (uint32_t)(n * 2), &s_bar[4], &tx);
         }
-        tx = warp_total(tx);
-        if (lane == 0) tc::mbar_arrive_expect_tx(&s_bar[4], tx);
+        if (P.lean) asm volatile("bar.arrive 2, %0;" ::"n"((kCW - kQIssue + 1) * 32) : "memory");
+        cl_wait();  // the logits of the whole cluster are here
+    } else {
+        // ---------------------------------------------------------- phase K (issuing warps)
+        // Two rounds, one copy of the issue code: the routed rows' copies go out in round 0
+        // for a given set (before the cluster's logits, which then give only the weights),
+        // in round 1 after the top-K otherwise.
+#pragma unroll 1
+        for (int rnd = 0; rnd < 2; ++rnd) {
+            if (rnd == (early ? 0 : 1)) issue_routed(s_aid);
+            if (rnd == 0) {
+                cl_wait();  // the logits of the whole cluster are here
+                if (warp == 0) {
+                    if (a.select) {  // a caller-given set (repaired in the prologue): only the weights come from z
+                        const int e = lane < K ? s_idx[lane] : -1;
+                        const float zk = e >= 0 ? z[e] : -INFINITY;
+                        const float m = warp_max(zk);
+                        const float ev = e >= 0 ? expf(zk - m) : 0.0f;
+                        const float sum = warp_sum(ev);
+                        if (lane < K) s_w[lane] = ev / sum;
+                    } else {
+                        warp_topk<kQMaxE / 32>(z, E, K, lane, s_idx, s_w);
+                    }
+                    __syncwarp();
+                    if (cta == 0 && lane < K) {  // the routing this call used, for the caller's record
+                        a.idx_out[lane] = s_idx[lane];
+                        a.w_out[lane] = s_w[lane];
+                    }
+                }
+                // the routing is known to the issuing warps (the others learn the window
+                // pointers through the copies' mbarriers)
+                asm volatile("bar.sync 1, %0;" ::"n"(kQIssue * 32) : "memory");
+            }
+        }
     }
 
     // ------------------------------------------------------------ phase G
