@@ -251,8 +251,6 @@ NCU_TRAFFIC = {
     ("prefill", "tc_gate_up"): 333590784 + 9545728,
     # one gate/up launch of the mixed ternary/4-bit MLP, one token
     ("mixed_b1", "mixed_gate_up"): 2014976,
-    # one cluster decode launch, one token of the Edge0 layer (DRAM read; nothing written back)
-    ("decode_k4", "decode_cluster"): 10795776,
 }
 
 
