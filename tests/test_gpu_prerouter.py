@@ -136,6 +136,35 @@ def test_select_forward_every_path(layer, T, path):
     assert_close_output(y, y_ref, "select T=%d" % T)
 
 
+@pytest.fixture(scope="module")
+def layer8():
+    shape = dataclasses.replace(workloads.DECODE_K4, K=8, n_adapters=2, random_adapters=True)
+    t = quantize_layer(workloads.moe_weights(shape, seed=12))
+    return shape, t
+
+
+def test_select_forward_top8_cluster(layer8):
+    """One token at top-8 with a given set: the cluster kernel's lean layout, whose routed
+    rows are copied after the cluster's logits as on the router path (the set itself is
+    repaired in the kernel's prologue); one entry repeated."""
+    shape, t = layer8
+    x, aid = workloads.moe_inputs(shape, seed=740, T=1)
+    sel = np.argsort(synth.uniform(740, "sel", (1, shape.E)), axis=1, kind="stable")[:, :shape.K].astype(np.int32)
+    y, idx, wts, kinds, st = _select_forward(shape, t, x, aid, sel)
+    assert st == 0 and path_ran("cluster", kinds), kinds
+    assert np.array_equal(idx, sel)
+    y_ref, _, w_ref, _, _ = oracle_layer(shape, t).ffn(x, aid, select=sel)
+    assert np.allclose(wts, w_ref, rtol=2e-5, atol=1e-6)
+    assert_close_output(y, y_ref, "select top-8 T=1")
+    bad = sel.copy()
+    bad[0, 5] = bad[0, 2]  # a repeat: replaced by the lowest expert not in the set
+    y2, idx2, _, _, st2 = _select_forward(shape, t, x, aid, bad)
+    want = bad.copy()
+    want[0, 5] = min(set(range(shape.E)) - set(int(v) for v in bad[0]))
+    assert st2 == 5 and np.array_equal(idx2, want)
+    assert_close_output(y2, oracle_layer(shape, t).ffn(x, aid, select=want)[0], "repaired select top-8")
+
+
 @pytest.mark.parametrize("T", [1, 6])
 def test_select_repairs_bad_entries(layer, T):
     shape, t = layer
