@@ -623,13 +623,13 @@ __global__ void __launch_bounds__(kCT, 1) decode_cluster_kernel(const __grid_con
         cl_wait();  // the logits of the whole cluster are here
     } else {
         // ---------------------------------------------------------- phase K (issuing warps)
-        // Two rounds, one copy of the issue code: the routed rows' copies go out in round 0
-        // for a given set (before the cluster's logits, which then give only the weights),
-        // in round 1 after the top-K otherwise.
+        // Two passes, one copy of the issue code: the routed rows' copies go out in the first
+        // pass for a given set (before the cluster's logits, which then give only the
+        // weights), in the second after the top-K otherwise.
 #pragma unroll 1
-        for (int rnd = 0; rnd < 2; ++rnd) {
-            if (rnd == (early ? 0 : 1)) issue_routed(s_aid);
-            if (rnd == 0) {
+        for (int pass = 0; pass < 2; ++pass) {
+            if (pass == (early ? 0 : 1)) issue_routed(s_aid);
+            if (pass == 0) {
                 cl_wait();  // the logits of the whole cluster are here
                 if (warp == 0) {
                     if (a.select) {  // a caller-given set (repaired in the prologue): only the weights come from z
